@@ -1,0 +1,287 @@
+"""Pins of the CPU oracle against things other than itself.
+
+Each test ties one oracle function to the pages (worked example, printed bit
+order), to closed forms, to brute force on tiny inputs, or to an independent
+library routine, chosen so that a dropped term, a flipped sign, a wrong index or
+a transposed operand in the oracle fails at least one of them. No GPU needed.
+"""
+import itertools
+
+import numpy as np
+import pytest
+import torch
+
+import synth
+from conftest import read_golden
+
+
+# ---------------------------------------------------------------- weight quantiser
+
+def _worked():
+    g = read_golden("worked_example.txt")
+    return {k: v for k, v in g.items()}
+
+
+@pytest.mark.parametrize("per_row", [True, False])
+def test_worked_example_scale_and_ternary(oracle, per_row):
+    """The printed example of "BitNet 深度实战" §2.4: scale 0.8333, pre-clip, clamp."""
+    g = _worked()
+    W = np.array([[float(v) for v in g["weight"]]], dtype=np.float32)
+    s = oracle.absmean_scale(W, per_row)
+    assert s.shape == (1,)
+    assert round(float(s[0]), 4) == float(g["scale"][0])
+    # mean |W| = 5/6 exactly in real arithmetic; fp32 result within one ulp of it
+    assert abs(float(s[0]) - 5.0 / 6.0) <= np.spacing(np.float32(5.0 / 6.0))
+    t, r = oracle.ternarize(W, s, per_row, return_rounded=True)
+    assert r[0].tolist() == [int(v) for v in g["pre_clip"]]
+    assert t[0].tolist() == [int(v) for v in g["ternary"]]
+    deq = (t[0].astype(np.float64) * float(s[0])).round(4)
+    assert deq.tolist() == [float(v) for v in g["dequantized"]]
+
+
+def test_ternarize_half_even_ties(oracle):
+    """round() is half-to-even (torch.round): ties at 0.5, 1.5, 2.5 with scale exactly 1."""
+    W = np.array([[0.5, -0.5, 1.5, -1.5, 1.0, 1.0, 1.0, 1.0],
+                  [2.5, 0.5, 1.0, 0.0, 0.0, 0.0, 0.0, 0.0]], dtype=np.float32)
+    s = oracle.absmean_scale(W, per_row=True)
+    assert s.tolist() == [1.0, 0.5]  # (8/8) and (4/8)
+    t, r = oracle.ternarize(W, s, True, return_rounded=True)
+    # row 1: W / 0.5 = [5, 1, 2, 0, ...]
+    assert r[0].tolist() == [0, 0, 2, -2, 1, 1, 1, 1]
+    assert t[0].tolist() == [0, 0, 1, -1, 1, 1, 1, 1]
+    assert r[1].tolist() == [5, 1, 2, 0, 0, 0, 0, 0]
+    assert t[1].tolist() == [1, 1, 1, 0, 0, 0, 0, 0]
+    W2 = np.array([[2.5, 0.5, 1.0, 0.0]], dtype=np.float32)  # scale 1: 2.5 -> 2 (even) -> 1
+    s2 = oracle.absmean_scale(W2, True)
+    assert s2.tolist() == [1.0]
+    t2, r2 = oracle.ternarize(W2, s2, True, return_rounded=True)
+    assert r2[0].tolist() == [2, 0, 1, 0] and t2[0].tolist() == [1, 0, 1, 0]
+
+
+def test_absmean_eps_clamp(oracle):
+    W = np.zeros((2, 8), dtype=np.float32)
+    W[1, :] = 1e-7
+    s = oracle.absmean_scale(W, True)
+    assert s.tolist() == [np.float32(1e-5), np.float32(1e-5)]
+    t = oracle.ternarize(W, s, True)
+    assert not t.any()
+
+
+def test_absmean_against_numpy_mean(oracle):
+    """Per-row and per-tensor scales agree with numpy's fp64 mean to one fp32 rounding."""
+    g = np.random.default_rng(7)
+    W = (g.standard_normal((37, 96)) * g.uniform(0.01, 3, size=(37, 1))).astype(np.float32)
+    s_row = oracle.absmean_scale(W, True)
+    ref_row = np.abs(W.astype(np.float64)).mean(axis=1)
+    assert np.all(np.abs(s_row - ref_row) <= np.spacing(ref_row.astype(np.float32)))
+    s_t = oracle.absmean_scale(W, False)
+    ref_t = np.abs(W.astype(np.float64)).mean()
+    assert abs(float(s_t[0]) - ref_t) <= np.spacing(np.float32(ref_t))
+    # per-row scale of row n must not depend on the other rows (index bug guard)
+    s_row_sub = oracle.absmean_scale(W[5:9], True)
+    assert np.array_equal(s_row_sub, s_row[5:9])
+
+
+def test_ternarize_against_definition_by_interval(oracle):
+    """t = +1 exactly when W/s >= 0.5 (ties to even: 0.5 -> 0), -1 when <= -0.5."""
+    g = np.random.default_rng(3)
+    W = g.standard_normal((16, 64)).astype(np.float32)
+    s = oracle.absmean_scale(W, False)
+    t = oracle.ternarize(W, s, False)
+    ratio = W.astype(np.float64) / float(s[0])
+    assert np.all(t[ratio > 0.5000001] == 1)
+    assert np.all(t[ratio < -0.5000001] == -1)
+    assert np.all(t[np.abs(ratio) < 0.4999999] == 0)
+    # per-row with one row scaled by 8 gives the same ternary row (scale invariance)
+    W2 = W.copy()
+    W2[3] *= 8.0  # power of two: exact, so the row quantises identically
+    t_row = oracle.ternarize(W, oracle.absmean_scale(W, True), True)
+    t_row2 = oracle.ternarize(W2, oracle.absmean_scale(W2, True), True)
+    assert np.array_equal(t_row, t_row2)
+
+
+# ---------------------------------------------------------------- packing
+
+def test_pack_worked_example_bytes(oracle):
+    g = read_golden("pack_example.txt")
+    t = np.array([[int(v) for v in g["ternary"]]], dtype=np.int8)
+    p = oracle.pack(t)
+    assert [f"0x{b:02x}" for b in p[0]] == g["bytes"]
+    assert oracle.unpack(p, 8)[0].tolist() == t[0].tolist()
+
+
+def test_pack_bit_positions(oracle):
+    """Weight i of a group of four sits in bits 2i..2i+1 with code t+1; others are 0 -> 01."""
+    for i, w in itertools.product(range(4), (-1, 0, 1)):
+        t = np.zeros((1, 4), dtype=np.int8)
+        t[0, i] = w
+        expect = 0x55 & ~(3 << (2 * i)) | ((w + 1) << (2 * i))
+        assert int(oracle.pack(t)[0, 0]) == expect
+    # the second byte holds weights 4..7 (K ordering across bytes)
+    t = np.zeros((2, 8), dtype=np.int8)
+    t[1, 5] = -1
+    p = oracle.pack(t)
+    assert p.tolist() == [[0x55, 0x55], [0x55, 0x51]]
+
+
+def test_pack_roundtrip_and_code_range(oracle):
+    g = np.random.default_rng(11)
+    t = g.integers(-1, 2, size=(23, 128)).astype(np.int8)
+    p = oracle.pack(t)
+    assert p.shape == (23, 32)
+    codes = np.stack([(p >> (2 * i)) & 3 for i in range(4)])
+    assert codes.max() <= 2  # code 3 never produced
+    assert np.array_equal(oracle.unpack(p, 128), t)
+
+
+def test_unpack_rejects_code3_and_pack_rejects_bad_weight(oracle):
+    with pytest.raises(oracle.OracleError):
+        oracle.unpack(np.array([[0xC0]], dtype=np.uint8), 4)
+    with pytest.raises(oracle.OracleError):
+        oracle.pack(np.array([[0, 2, 0, 0]], dtype=np.int8))
+
+
+# ---------------------------------------------------------------- activation quantiser
+
+def test_quant_act_hand_example(oracle):
+    """amax = 1 -> s_x = 127; x*127 is exact in fp32 for these values, so q = rint(127 x)
+    with ties to even: -63.5 -> -64, 63.5 -> 64, 31.75 -> 32, 15.875 -> 16."""
+    xs = np.array([[1.0, -0.5, 0.25, 0.0, 0.75, -1.0, 0.125, 0.5]], dtype=np.float32)
+    q, s = oracle.quant_act(synth.to_bf16_bits(xs))
+    assert s.tolist() == [127.0]
+    assert q[0].tolist() == [127, -64, 32, 0, 95, -127, 16, 64]
+
+
+def test_quant_act_invariants(oracle):
+    g = np.random.default_rng(5)
+    x = synth.to_bf16_bits(g.standard_normal((9, 256)).astype(np.float32)
+                           * g.uniform(1e-3, 50, size=(9, 1)).astype(np.float32))
+    x[4] = 0  # an all-zero token
+    q, s = oracle.quant_act(x)
+    xf = synth.bf16_bits_to_f32(x).astype(np.float64)
+    assert np.abs(q.astype(int)).max() <= 127
+    for m in range(9):
+        if m == 4:
+            assert not q[m].any() and s[m] == np.float32(127.0) / np.float32(1e-5)
+            continue
+        amax = np.abs(xf[m]).max()
+        assert np.abs(q[m].astype(int)).max() == 127
+        assert s[m] == np.float32(127.0) / np.float32(amax)
+        # q is the nearest integer to x*s_x: error at most half a step (+ one fp32 rounding)
+        err = np.abs(q[m] - xf[m] * float(s[m]))
+        assert err.max() <= 0.5 + 127 * 2.0 ** -23
+        # the token's row does not leak into another token (index bug guard)
+        q1, s1 = oracle.quant_act(x[m:m + 1])
+        assert np.array_equal(q1[0], q[m]) and s1[0] == s[m]
+    # x -> -x gives q -> -q with the same scale
+    qn, sn = oracle.quant_act(x ^ np.uint16(0x8000))
+    assert np.array_equal(qn, -q) and np.array_equal(sn, s)
+
+
+# ---------------------------------------------------------------- contraction
+
+@pytest.mark.parametrize("M,N,K", [(1, 1, 4), (3, 5, 8), (8, 16, 64), (5, 2, 12), (2, 7, 40)])
+def test_ternary_matmul_brute_force(oracle, M, N, K):
+    """add/sub/skip loop == dense int64 matmul (numpy) on tiny non-square shapes."""
+    g = np.random.default_rng(M * 100 + N * 10 + K)
+    q = g.integers(-128, 128, size=(M, K)).astype(np.int8)
+    t = g.integers(-1, 2, size=(N, K)).astype(np.int8)
+    acc = oracle.ternary_matmul(q, t)
+    ref = q.astype(np.int64) @ t.astype(np.int64).T
+    assert acc.shape == (M, N)
+    assert np.array_equal(acc.astype(np.int64), ref)
+
+
+def test_ternary_matmul_exhaustive_tiny(oracle):
+    """Every ternary row of length 3 against a fixed int8 row set."""
+    rows = np.array(list(itertools.product((-1, 0, 1), repeat=3)), dtype=np.int8)
+    q = np.array([[127, -128, 5], [-7, 0, 99]], dtype=np.int8)
+    acc = oracle.ternary_matmul(q, rows)
+    for n, w in enumerate(rows):
+        for m in range(2):
+            assert acc[m, n] == sum(int(q[m, k]) * int(w[k]) for k in range(3))
+
+
+def test_ternary_matmul_closed_forms(oracle):
+    g = np.random.default_rng(9)
+    q = g.integers(-127, 128, size=(4, 32)).astype(np.int8)
+    rs = q.astype(np.int64).sum(axis=1)
+    assert np.array_equal(oracle.ternary_matmul(q, np.ones((3, 32), np.int8)),
+                          np.repeat(rs[:, None], 3, axis=1))
+    assert np.array_equal(oracle.ternary_matmul(q, -np.ones((3, 32), np.int8)),
+                          -np.repeat(rs[:, None], 3, axis=1))
+    assert not oracle.ternary_matmul(q, np.zeros((3, 32), np.int8)).any()
+    eye = np.eye(32, dtype=np.int8)[:6]  # t[n, k] = [k == n] selects activation column n
+    assert np.array_equal(oracle.ternary_matmul(q, eye), q[:, :6].astype(np.int32))
+
+
+def test_ternary_matmul_extreme_accumulator(oracle):
+    """|acc| reaches 128*K without overflow at the largest K in the workloads."""
+    K = 14336
+    q = np.full((1, K), -128, dtype=np.int8)
+    t = -np.ones((1, K), dtype=np.int8)
+    assert oracle.ternary_matmul(q, t)[0, 0] == 128 * K
+
+
+# ---------------------------------------------------------------- dequant and rounding
+
+def test_dequant_matches_float_linear(oracle):
+    """y equals the float form linear(q / s_x, t * s_w) of "BitNet 深度实战" §3.2 in fp64."""
+    g = np.random.default_rng(2)
+    M, N, K = 3, 6, 64
+    q = g.integers(-127, 128, size=(M, K)).astype(np.int8)
+    t = g.integers(-1, 2, size=(N, K)).astype(np.int8)
+    s_x = g.uniform(1, 100, size=M).astype(np.float32)
+    for per_row in (False, True):
+        s_w = g.uniform(0.5, 2, size=N if per_row else 1).astype(np.float32)
+        y = oracle.dequant(oracle.ternary_matmul(q, t), s_x, s_w, per_row)
+        sw = s_w.astype(np.float64) if per_row else np.full(N, float(s_w[0]))
+        ref = (q / s_x.astype(np.float64)[:, None]) @ (t * sw[:, None]).T
+        np.testing.assert_allclose(y, ref, rtol=1e-12, atol=1e-12)
+
+
+def test_round_bf16_matches_torch_for_fp32_values(oracle):
+    g = np.random.default_rng(4)
+    f = np.concatenate([g.standard_normal(20000).astype(np.float32) * 1e3,
+                        g.standard_normal(2000).astype(np.float32) * 1e-38,  # subnormal range
+                        np.array([0.0, -0.0, 3.3e38, -3.3e38, 1.0 + 2 ** -8, 1.0 + 3 * 2 ** -8],
+                                 dtype=np.float32)])
+    # ties: values exactly halfway between bf16 neighbours
+    ties = ((g.integers(0, 2 ** 15, size=5000).astype(np.uint32) << 16) | 0x8000).view(np.float32)
+    f = np.concatenate([f, ties[np.isfinite(ties)]])
+    ours = oracle.round_bf16(f.astype(np.float64))
+    ref = torch.from_numpy(f).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(ours, ref)
+
+
+def test_round_bf16_no_double_rounding(oracle):
+    # 1 + 2^-8 + 2^-30 lies above the tie 1 + 2^-8: nearest bf16 is 1 + 2^-7. Going through
+    # fp32 first would land on the tie and round to 1.0.
+    v = np.array([1.0 + 2.0 ** -8 + 2.0 ** -30, -(1.0 + 2.0 ** -8 + 2.0 ** -30)])
+    out = oracle.round_bf16(v)
+    assert out.tolist() == [0x3F81, 0xBF81]
+
+
+# ---------------------------------------------------------------- composite forward
+
+def test_bitlinear_composite_and_sampled(oracle):
+    cfg = synth.tiny(0)
+    packed, s_w = oracle.pack_weights(cfg["W"], cfg["per_row"])
+    K = cfg["K"]
+    full = oracle.bitlinear(cfg["x"], packed, s_w, cfg["per_row"], K)
+    assert full["y"].shape == (4, 256)
+    # composite equals the product of its parts
+    t = oracle.unpack(packed, K)
+    q, s_x = oracle.quant_act(cfg["x"])
+    ref = (q / s_x.astype(np.float64)[:, None]) @ (t.astype(np.float64) * float(s_w[0])).T
+    np.testing.assert_allclose(full["y"], ref, rtol=1e-12, atol=1e-12)
+    # sampled forward agrees with the full one on its sample
+    m_idx, n_idx = np.array([3, 0]), np.array([255, 7, 128])
+    smp = oracle.bitlinear_sampled(cfg["x"], packed, s_w, cfg["per_row"], K, m_idx, n_idx)
+    assert np.array_equal(smp["y"], full["y"][np.ix_(m_idx, n_idx)])
+    assert np.array_equal(smp["acc"], full["acc"][np.ix_(m_idx, n_idx)])
+    assert np.array_equal(smp["q"], full["q"][m_idx])
+    # the float product with the latent weights is close (quantisation error only)
+    xf = synth.bf16_bits_to_f32(cfg["x"]).astype(np.float64)
+    dense = xf @ cfg["W"].astype(np.float64).T
+    assert np.corrcoef(dense.ravel(), full["y"].ravel())[0, 1] > 0.8
