@@ -1,0 +1,410 @@
+"""Benchmark of the W2A8 BitLinear forward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Headline (value): decode GEMV throughput in algorithmic GB/s at M = 1 over the 2B-4T
+projection shapes (N, K) in {(2560,2560), (640,2560), (6912,2560), (2560,6912)}, ternary
+weights P(0) = 0.4, s_w ~ U(0.5, 2), x ~ N(0, 1). One step = bitnet_linear on every shape
+for each of R weight replicas (R chosen so the step's packed weights exceed 2x L2), run
+as one CUDA graph. Second number (gemm): prefill GEMM int8 TOPS at M = 2048 on the same
+shapes (Student-t activations with outlier channels, ternary P(0) = 0.5).
+
+Timing: W untimed warm-up steps, then K steps; L2 is flushed (a 256 MB write) before every
+step, outside the step's CUDA-event pair; per-step event times are summed; ranks meet at a
+barrier with a device synchronize on both sides and rank 0 reports the max over ranks.
+Multi-GPU (torchrun): every rank runs its own replica of the workload (weak scaling, no
+data-path collective).
+
+--impl reference times the CPU oracle (plain C, one thread) on a bounded sample of the same
+workload on this machine's host cores: the only reference implementation there is.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+METRIC = "W2A8 ternary GEMV HBM GB/s (M=1) and GEMM int8 TOPS (M>=512) vs roofline"
+L2_BYTES = 126 * 1024 * 1024
+DECODE_M = 1
+PREFILL_M = 2048
+# nominal dense int8 : bf16 tensor-core ratio on B200 (4.5 vs 2.25 PFLOP/s)
+INT8_PER_BF16 = 2.0
+
+
+def decode_bytes(M, N, K):
+    """Algorithmic bytes of one BitLinear call: packed W + x + y + s_w (per tensor)."""
+    return N * K // 4 + 2 * M * K + 2 * M * N + 4
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "bf16_tflops_sustained": float(d["bf16_tflops_sustained"]), "src": "measured"}
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                "src": "fallback"}
+
+
+# ---------------------------------------------------------------------------- ranks
+def dist_env():
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def reduce_over_ranks(local_ms: float, local_units: float, world: int):
+    """Max of the per-rank time and sum of the per-rank work (the job's aggregate)."""
+    if world <= 1:
+        return local_ms, local_units
+    import torch
+    import torch.distributed as dist
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([local_ms], dtype=torch.float64, device=dev)
+    u = torch.tensor([local_units], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    dist.all_reduce(u, op=dist.ReduceOp.SUM)
+    return float(t.item()), float(u.item())
+
+
+# ---------------------------------------------------------------------------- clocks
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML (read-only) every 50 ms."""
+
+    REASONS = {"hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
+               "sw_power_cap": 0x4}
+
+    def __init__(self, index: int):
+        self.index = index
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self._stop = None
+
+    def _run(self):
+        import pynvml
+        try:
+            pynvml.nvmlInit()
+            h = pynvml.nvmlDeviceGetHandleByIndex(self.index)
+            self.max_mhz = float(pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM))
+            while not self._stop.is_set():
+                self.samples.append(float(pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)))
+                bits = pynvml.nvmlDeviceGetCurrentClocksThrottleReasons(h)
+                for name, bit in self.REASONS.items():
+                    if bits & bit:
+                        self.reasons.add(name)
+                self._stop.wait(0.05)
+        except Exception as e:  # sampling is best effort; the line says so
+            self.error = repr(e)
+
+    def __enter__(self):
+        import threading
+        self._stop = threading.Event()
+        self._t = threading.Thread(target=self._run, daemon=True)
+        self._t.start()
+        return self
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        self._t.join(timeout=5)
+        return False
+
+    def summary(self):
+        d = {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+             "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+             "samples": len(self.samples)}
+        if getattr(self, "error", None):
+            d["error"] = self.error
+        return d
+
+
+# ---------------------------------------------------------------------------- workloads
+def build_decode(bn, torch, replicas: int, dev):
+    """Per replica and shape: packed weights, s_w, x, y (all resident in HBM)."""
+    calls = []
+    for r in range(replicas):
+        for si in range(len(synth.SWEEP_SHAPES)):
+            c = synth.decode_case(si, replica=r, M=DECODE_M)
+            packed = bn.bitnet_pack_ternary(torch.from_numpy(c["t"]).to(dev))
+            s_w = torch.from_numpy(c["s_w"]).to(dev)
+            x = torch.from_numpy(c["x"].view(np.int16).copy()).to(dev).view(torch.bfloat16)
+            y = torch.empty((DECODE_M, c["N"]), dtype=torch.bfloat16, device=dev)
+            calls.append({"x": x, "packed": packed, "s_w": s_w, "y": y, "N": c["N"], "K": c["K"]})
+    return calls
+
+
+def build_prefill(bn, torch, dev):
+    calls = []
+    for si in range(len(synth.SWEEP_SHAPES)):
+        c = synth.prefill_case(si, PREFILL_M)
+        packed = bn.bitnet_pack_ternary(torch.from_numpy(c["t"]).to(dev))
+        s_w = torch.from_numpy(c["s_w"]).to(dev)
+        x = torch.from_numpy(c["x"].view(np.int16).copy()).to(dev).view(torch.bfloat16)
+        y = torch.empty((PREFILL_M, c["N"]), dtype=torch.bfloat16, device=dev)
+        ws = bn.make_workspace(PREFILL_M, c["K"], dev)
+        calls.append({"x": x, "packed": packed, "s_w": s_w, "y": y, "N": c["N"], "K": c["K"],
+                      "ws": ws})
+    return calls
+
+
+def run_calls(bn, calls):
+    for c in calls:
+        bn.bitnet_linear(c["x"], c["packed"], c["s_w"], False, y=c["y"], workspace=c.get("ws"))
+
+
+def capture(torch, fn):
+    g = torch.cuda.CUDAGraph()
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        fn()  # warm the launch path outside capture
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    with torch.cuda.graph(g):
+        fn()
+    torch.cuda.synchronize()
+    return g
+
+
+def timed_steps(torch, step_fn, steps, warmup, flush_buf, world):
+    import torch.distributed as dist
+    for _ in range(warmup):
+        flush_buf.add_(1)
+        step_fn()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(steps)]
+    for a, b in ev:
+        flush_buf.add_(1)  # evict L2 (outside the step's events)
+        a.record()
+        step_fn()
+        b.record()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    return sum(a.elapsed_time(b) for a, b in ev)
+
+
+# ---------------------------------------------------------------------------- CPU oracle
+def oracle_sample(seconds_min: float):
+    """Times the oracle (as it stands, one thread) on whole decode sweeps at M = 1."""
+    import oracle
+    oracle.build()
+    cases = []
+    for si in range(len(synth.SWEEP_SHAPES)):
+        c = synth.decode_case(si, replica=0, M=DECODE_M)
+        cases.append((c, oracle.pack(c["t"])))
+    sweep_bytes = sum(decode_bytes(DECODE_M, c["N"], c["K"]) for c, _ in cases)
+    done, t0 = 0, time.perf_counter()
+    while True:
+        for c, packed in cases:
+            oracle.bitlinear(c["x"], packed, c["s_w"], False, c["K"])
+        done += 1
+        el = time.perf_counter() - t0
+        if el >= seconds_min:
+            break
+    return {"value": done * sweep_bytes / el / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "sample": f"{done} full decode sweeps (4 shapes, M=1), {el:.1f} s"}
+
+
+def run_reference(args):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return 0
+    import oracle
+    oracle.build()
+    cases = []
+    for si in range(len(synth.SWEEP_SHAPES)):
+        c = synth.decode_case(si, replica=0, M=DECODE_M)
+        cases.append((c, oracle.pack(c["t"])))
+    sweep_bytes = sum(decode_bytes(DECODE_M, c["N"], c["K"]) for c, _ in cases)
+
+    def step():
+        for c, packed in cases:
+            oracle.bitlinear(c["x"], packed, c["s_w"], False, c["K"])
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    el = time.perf_counter() - t0
+    value = args.steps * sweep_bytes / el / 1e9
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": el * 1e3 / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "s8xternary->s32", "data": "synthetic",
+        "config": {"workload": "decode GEMV sweep M=1, 2B-4T shapes (N,K) in "
+                               "{(2560,2560),(640,2560),(6912,2560),(2560,6912)}; one sweep "
+                               "(one weight replica) per step"},
+        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": 1, "kind": "oracle",
+                         "sample": f"{args.steps} sweeps of the 4 shapes at M=1"},
+        "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------------------- main arm
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    rank, world, local = dist_env()
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    import ternary_w2a8_linear_token_b200 as bn
+
+    peaks = load_peaks()
+    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+
+    # ---------------- decode GEMV sweep
+    per_replica = sum(N * K // 4 for N, K in synth.SWEEP_SHAPES)
+    replicas = args.replicas or max(1, -(-2 * L2_BYTES // per_replica))
+    calls = build_decode(bn, torch, replicas, dev)
+    launches_per_step = len(calls)
+    step_bytes = sum(decode_bytes(DECODE_M, c["N"], c["K"]) for c in calls)
+    g_dec = capture(torch, lambda: run_calls(bn, calls))
+    with ClockSampler(local) as clk:
+        dec_ms = timed_steps(torch, g_dec.replay, args.steps, args.warmup, flush, world)
+    assert bn.bitnet_check_device_errors() == 0
+    dec_ms_max, total_bytes = reduce_over_ranks(dec_ms, step_bytes * args.steps, world)
+    gbs = total_bytes / (dec_ms_max * 1e-3) / 1e9
+    per_launch_bytes = step_bytes / launches_per_step
+    avg_launch_s = dec_ms * 1e-3 / (args.steps * launches_per_step)
+    achieved = per_launch_bytes / avg_launch_s / 1e9
+
+    # ---------------- end to end: pinned host x -> device, forward, y -> pinned host
+    h_x = torch.empty(sum(c["x"].numel() for c in calls), dtype=torch.bfloat16).pin_memory()
+    h_y = torch.empty(sum(c["y"].numel() for c in calls), dtype=torch.bfloat16).pin_memory()
+    d_x = torch.empty_like(h_x, device=dev)
+    d_y = torch.empty_like(h_y, device=dev)
+    off = 0
+    e2e_calls = []
+    for c in calls:
+        n = c["x"].numel()
+        xv = d_x[off:off + n].view(c["x"].shape)
+        xv.copy_(c["x"])
+        e2e_calls.append(dict(c, x=xv))
+        off += n
+    h_x.copy_(d_x)
+    off = 0
+    for c in e2e_calls:
+        n = c["y"].numel()
+        c["y"] = d_y[off:off + n].view(c["y"].shape)
+        off += n
+    g_e2e = capture(torch, lambda: run_calls(bn, e2e_calls))
+
+    def e2e_step():
+        d_x.copy_(h_x, non_blocking=True)
+        g_e2e.replay()
+        h_y.copy_(d_y, non_blocking=True)
+
+    e2e_ms = timed_steps(torch, e2e_step, args.steps, args.warmup, flush, world)
+    e2e_ms_max, _ = reduce_over_ranks(e2e_ms, 0.0, world)
+    e2e_gbs = total_bytes / (e2e_ms_max * 1e-3) / 1e9
+
+    # ---------------- prefill GEMM
+    if args.only == "decode":
+        pcalls = []
+    else:
+        pcalls = build_prefill(bn, torch, dev)
+    gemm = None
+    g_pre = None
+    if pcalls:
+        g_pre = capture(torch, lambda: run_calls(bn, pcalls))
+        pre_ms = timed_steps(torch, g_pre.replay, args.steps, args.warmup, flush, world)
+        assert bn.bitnet_check_device_errors() == 0
+        ops_step = sum(2.0 * PREFILL_M * c["N"] * c["K"] for c in pcalls)
+        pre_ms_max, pre_ops = reduce_over_ranks(pre_ms, ops_step * args.steps, world)
+        tops = pre_ops / (pre_ms_max * 1e-3) / 1e12
+        int8_peak = peaks["bf16_tflops"] * INT8_PER_BF16
+        local_tops = ops_step * args.steps / (pre_ms * 1e-3) / 1e12
+        gemm = {"value": tops, "unit": "TOPS", "ms_per_step": pre_ms_max / args.steps,
+                "workload": f"prefill GEMM M={PREFILL_M} on the same 4 shapes, x = 0.5 t_4 "
+                            "with 1% x20 outlier channels, ternary P(0)=0.5",
+                "roofline": {"bound": "tensor", "achieved": local_tops, "peak": int8_peak,
+                             "unit": "TOPS", "frac": local_tops / int8_peak, "traffic": None,
+                             "peak_src": f"{peaks['src']} bf16 x {INT8_PER_BF16} "
+                                         "(nominal int8:bf16)",
+                             "note": "per-call time includes the quantiser launch"}}
+
+    cpu = oracle_sample(args.cpu_seconds) if (rank == 0 and world == 1 and args.cpu_seconds > 0) \
+        else None
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": gbs, "unit": "GB/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": dec_ms_max / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "s8xternary->s32",
+            "data": "synthetic",
+            "config": {
+                "workload": "decode GEMV sweep M=1, 2B-4T shapes (N,K) in {(2560,2560),"
+                            "(640,2560),(6912,2560),(2560,6912)}, ternary P(0)=0.4, "
+                            f"s_w~U(0.5,2), x~N(0,1); {replicas} weight replicas per step "
+                            f"({per_replica * replicas / 1e6:.0f} MB packed) as one CUDA graph",
+                "l2": "256 MB write before every step (outside the step's events); step "
+                      "weights exceed 2x L2",
+                "bytes_per_step": step_bytes, "launches_per_step": launches_per_step,
+                "parallelism": f"replica x{world}",
+            },
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"],
+                         "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
+                         "traffic": None, "peak_src": peaks["src"],
+                         "kernel": "gemv_w2a8_kernel"},
+            "e2e": {"value": e2e_gbs, "unit": "GB/s",
+                    "h2d_bytes_per_step": int(h_x.numel() * 2),
+                    "d2h_bytes_per_step": int(h_y.numel() * 2)},
+            "gpu_launches": args.steps * launches_per_step * 2 + args.steps * 2 * len(pcalls),
+            "clocks": clk.summary(),
+            "gemm": gemm,
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+    del g_dec, g_e2e, g_pre
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--only", choices=["all", "decode"], default="all",
+                    help="decode: skip the prefill GEMM part (small profiling runs)")
+    ap.add_argument("--replicas", type=int, default=0,
+                    help="weight replicas per decode step (0: enough to exceed 2x L2)")
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)  # at least 3 untimed warm-up steps
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,199 @@
+/*
+ * bitnet.h — C ABI of the B200 (sm_100a) W2A8 BitLinear library (libbitnet.so).
+ *
+ * The operation is the BitNet b1.58 BitLinear forward:
+ *   y[m, n] = (sum_k q[m, k] * t[n, k]) * s_w / s_x[m]
+ * with ternary weights t in {-1, 0, +1} and absmean scale s_w (page "BitNet 深度实战：
+ * 微软 32K Star 的 1-bit LLM 推理框架", section 2.4 "量化函数的细节" and section 3.2, where
+ * BitLinear computes linear(x, t * s_w)), weights stored 2-bit packed as (N, K/4) uint8
+ * with four weights per byte (page "BitNet-Triton：消费级GPU上的1.58-bit大模型推理加速方案",
+ * section "技术架构：融合内核的三重优化", item 1; bit order from "BitNet 深度实战" section
+ * 4.3 "位打包（Bit Packing）存储"), int8 activations quantised per token (BitNet-Triton,
+ * items 2 and 3; "BitNet 1-bit LLM推理优化：内存布局、量化策略与硬件加速", section 3.2
+ * "激活量化策略"), and an int32 accumulator ("BitNet 深度实战" section 4.4 "查找表加速").
+ *
+ * Conventions shared by every call:
+ *  - Data pointers are DEVICE pointers in the current CUDA context, owned by the
+ *    caller. The library keeps no pointer after a call returns.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = the legacy default stream).
+ *    Every call is asynchronous on that stream and returns once the work is queued.
+ *  - Arguments are checked on the host before anything is launched; a call that
+ *    returns an error status has launched nothing (except BITNET_ERR_CUDA, which
+ *    reports a failed launch).
+ *  - Layouts are dense row-major. bf16 values are passed as their uint16 bit
+ *    patterns. Base addresses of x, packed, q, y and t must be 16-byte aligned and
+ *    `workspace` 256-byte aligned (BITNET_ERR_ALIGN otherwise).
+ *  - Shapes: M, N >= 1; K >= 64 and K % 64 == 0 (BITNET_ERR_SHAPE if K % 4 != 0,
+ *    BITNET_ERR_UNSUPPORTED for other K); M, N, K < 2^31.
+ *  - NaN or Inf in x or W give unspecified (but memory-safe) results.
+ *  - Rounding: every float step is IEEE binary32 round-to-nearest-even, with no
+ *    contraction into FMA where the order below is stated.
+ *  - Thread safety: calls may be made from several host threads. The library
+ *    holds one piece of device state, the watchdog word read by
+ *    bitnet_check_device_errors().
+ */
+#ifndef BITNET_H
+#define BITNET_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    BITNET_OK = 0,
+    BITNET_ERR_NULL = 1,        /* a required pointer is NULL                                   */
+    BITNET_ERR_SHAPE = 2,       /* M, N or K out of range, or K not a multiple of 4             */
+    BITNET_ERR_ALIGN = 3,       /* a pointer is not aligned as stated above                     */
+    BITNET_ERR_UNSUPPORTED = 4, /* valid by the method but not by these kernels (e.g. K % 64)   */
+    BITNET_ERR_CUDA = 5,        /* a CUDA launch or query failed                                */
+    BITNET_ERR_TIMEOUT = 6,     /* a kernel's bounded wait expired (see bitnet_check_device_errors) */
+    BITNET_ERR_WORKSPACE = 7    /* workspace missing or smaller than bitnet_linear_workspace_size() */
+} bitnet_status;
+
+typedef enum {
+    BITNET_SCALE_PER_TENSOR = 0, /* s_w has 1 element (the BitNet b1.58 layout)                 */
+    BITNET_SCALE_PER_ROW = 1     /* s_w has N elements (mean along dim=-1, "BitNet 深度实战" 2.4) */
+} bitnet_scale_mode;
+
+typedef enum {
+    BITNET_OUT_BF16 = 0, /* y is (M, N) bf16, round-to-nearest-even of the fp32 value */
+    BITNET_OUT_F32 = 1   /* y is (M, N) fp32                                          */
+} bitnet_out_dtype;
+
+typedef enum {
+    BITNET_PATH_AUTO = 0, /* GEMV for M <= BITNET_GEMV_MAX_M, tensor-core GEMM above      */
+    BITNET_PATH_GEMV = 1, /* force the dp4a GEMV with fused activation quantisation      */
+    BITNET_PATH_TC = 2    /* force the tcgen05 GEMM (needs the workspace)                 */
+} bitnet_path;
+
+#define BITNET_GEMV_MAX_M 8
+#define BITNET_MAX_PROJ 8
+
+/*
+ * bitnet_pack_weights — the offline weight step ("BitNet 深度实战" section 2.4, packing
+ * per section 4.3): absmean scale, ternarise, pack.
+ *   W       [in]  (N, K) fp32 latent weights, device.
+ *   mode          BITNET_SCALE_PER_TENSOR or BITNET_SCALE_PER_ROW.
+ *   packed  [out] (N, K/4) uint8, device. Byte j of row n holds weights 4j..4j+3, weight
+ *                 4j+i in bits 2i..2i+1, code = t + 1 (00 = -1, 01 = 0, 10 = +1; 11 unused).
+ *                 Also used as scratch for the per-row sums before it is written.
+ *   s_w     [out] fp32, 1 element (per tensor) or N (per row), device.
+ * Order of operations (fixed, so results are bit-reproducible): r_n = binary64 sum of
+ * |W[n,k]| for k ascending; per row s_n = (float)(r_n / K); per tensor
+ * s = (float)((r_0 + r_1 + ... + r_{N-1}) / (N*K)) summed for n ascending; then
+ * s = max(s, 1e-5f). t = clamp(rint(W / s), -1, 1) with a binary32 divide, ties to even.
+ */
+bitnet_status bitnet_pack_weights(const float* W, int64_t N, int64_t K, bitnet_scale_mode mode,
+                                  uint8_t* packed, float* s_w, void* stream);
+
+/*
+ * bitnet_pack_ternary — pack weights that are already ternary (synthetic workloads draw
+ * t directly). t is (N, K) int8 with values in {-1, 0, +1} (other values give
+ * unspecified codes); packed is (N, K/4) uint8 in the layout above. No scale is made.
+ */
+bitnet_status bitnet_pack_ternary(const int8_t* t, int64_t N, int64_t K, uint8_t* packed,
+                                  void* stream);
+
+/*
+ * bitnet_quant_act — per-token absmax int8 activation quantiser (BitNet-Triton item 3
+ * "融合激活量化"; "BitNet 1-bit LLM推理优化" section 3.2). For each token m:
+ *   amax = max_k |x[m,k]|;  s_x[m] = 127 / max(amax, 1e-5)  (binary32 divide);
+ *   q[m,k] = clamp(rint(x[m,k] * s_x[m]), -128, 127)          (binary32 multiply).
+ *   x   [in]  (M, K) bf16 bits, device.   q [out] (M, K) int8.   s_x [out] (M) fp32.
+ * |q| <= 127 always (-128 is unreachable); every non-zero token has max |q| = 127.
+ */
+bitnet_status bitnet_quant_act(const uint16_t* x, int64_t M, int64_t K, int8_t* q, float* s_x,
+                               void* stream);
+
+/*
+ * Workspace bytes the tensor-core path of bitnet_linear / bitnet_linear_batch needs for
+ * M tokens of width K (quantised activations and per-token scales). The GEMV path
+ * (M <= BITNET_GEMV_MAX_M under BITNET_PATH_AUTO) uses none: callers that only run such
+ * M may pass workspace = NULL.
+ */
+size_t bitnet_linear_workspace_size(int64_t M, int64_t K);
+
+/*
+ * bitnet_linear — the BitLinear forward: per-token quantisation of x (as in
+ * bitnet_quant_act), unpacking of the 2-bit codes, int8 x ternary contraction with an
+ * int32 accumulator, and the dequant epilogue, all on the device.
+ *   x        [in]  (M, K) bf16 bits.        packed [in] (N, K/4) uint8 (layout above).
+ *   s_w      [in]  fp32, 1 or N elements by `mode`.
+ *   y        [out] (M, N) bf16 or fp32 by `out_dtype`.
+ *   workspace, workspace_bytes: device scratch of at least bitnet_linear_workspace_size(M, K)
+ *            bytes when the tensor-core path runs (M > BITNET_GEMV_MAX_M); its contents
+ *            on entry are ignored, and it must not be shared by calls that may overlap.
+ * Epilogue arithmetic: acc = exact int32 sum; r = 1/s_x[m] (binary32, rounded);
+ * y = (float)acc * (s_w[n or 0] * r), each product rounded; bf16 is RNE of that fp32
+ * value. The result differs from the exact acc * s_w / s_x by at most 3 binary32
+ * roundings (relative error < 2^-22), before the bf16 rounding.
+ */
+bitnet_status bitnet_linear(const uint16_t* x, int64_t M, int64_t K, const uint8_t* packed,
+                            const float* s_w, bitnet_scale_mode mode, int64_t N, void* y,
+                            bitnet_out_dtype out_dtype, void* workspace, size_t workspace_bytes,
+                            void* stream);
+
+/* bitnet_linear with an explicit choice of kernel path (testing and benchmarking). */
+bitnet_status bitnet_linear_ex(const uint16_t* x, int64_t M, int64_t K, const uint8_t* packed,
+                               const float* s_w, bitnet_scale_mode mode, int64_t N, void* y,
+                               bitnet_out_dtype out_dtype, void* workspace,
+                               size_t workspace_bytes, bitnet_path path, void* stream);
+
+/* One projection of a batch: its own packed weights, scale, width N and output (M, N). */
+typedef struct {
+    const uint8_t* packed; /* (N, K/4) uint8, device                  */
+    const float* s_w;      /* 1 or N fp32, device                      */
+    int32_t mode;          /* bitnet_scale_mode                        */
+    int32_t reserved;      /* must be 0                                */
+    int64_t N;             /* output width of this projection          */
+    void* y;               /* (M, N) output, device                    */
+} bitnet_proj;
+
+/*
+ * bitnet_linear_batch — several projections of one input x, e.g. q/k/v of one hidden
+ * state or gate/up of the MLP ("BitNet 深度实战" section 3.2, BitLlamaAttention and
+ * BitLlamaMLP). x is quantised once and all projections run in one GEMM/GEMV launch.
+ *   projs [in] HOST array of nproj (1..BITNET_MAX_PROJ) descriptors; all share K and M.
+ * Results equal nproj separate bitnet_linear calls bit for bit.
+ */
+bitnet_status bitnet_linear_batch(const uint16_t* x, int64_t M, int64_t K,
+                                  const bitnet_proj* projs, int32_t nproj,
+                                  bitnet_out_dtype out_dtype, void* workspace,
+                                  size_t workspace_bytes, void* stream);
+
+/* bitnet_linear_batch with an explicit kernel path. */
+bitnet_status bitnet_linear_batch_ex(const uint16_t* x, int64_t M, int64_t K,
+                                     const bitnet_proj* projs, int32_t nproj,
+                                     bitnet_out_dtype out_dtype, void* workspace,
+                                     size_t workspace_bytes, bitnet_path path, void* stream);
+
+/*
+ * bitnet_linear_i32 — the contraction alone, for bit-exact checks: acc[m, n] =
+ * sum_k q[m, k] * t[n, k] in int32 from int8 q (M, K) and packed weights (N, K/4).
+ * Runs the same GEMV / tensor-core main loops as bitnet_linear (chosen by `path`).
+ */
+bitnet_status bitnet_linear_i32(const int8_t* q, int64_t M, int64_t K, const uint8_t* packed,
+                                int64_t N, int32_t* acc, void* workspace, size_t workspace_bytes,
+                                bitnet_path path, void* stream);
+
+/*
+ * bitnet_check_device_errors — synchronises the current device, returns the library's
+ * watchdog word in *flags (0 = no kernel gave up a bounded wait since the last check)
+ * and clears it. Returns BITNET_ERR_TIMEOUT when the word was non-zero.
+ */
+bitnet_status bitnet_check_device_errors(int32_t* flags);
+
+/* Human-readable name of a status code (static storage). */
+const char* bitnet_status_string(bitnet_status status);
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+int32_t bitnet_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BITNET_H */

@@ -1,0 +1,221 @@
+"""Python binding of libbitnet (the B200 W2A8 BitLinear library).
+
+Argument marshalling only: every step of the forward runs in the CUDA kernels behind
+the C ABI declared in ``include/bitnet.h``. PyTorch supplies device memory (output and
+workspace tensors) and the current CUDA stream; nothing here computes on tensors.
+
+The shared library is built in-tree by ``python -m ternary_w2a8_linear_token_b200.build``.
+Importing this package without it raises ImportError: there is no fallback path.
+
+Functions keep the C names:
+    bitnet_pack_weights(W, per_row)            -> (packed, s_w)
+    bitnet_pack_ternary(t)                     -> packed
+    bitnet_quant_act(x)                        -> (q, s_x)
+    bitnet_linear(x, packed, s_w, per_row, ...) -> y
+    bitnet_linear_batch(x, projs, ...)         -> [y, ...]
+    bitnet_linear_i32(q, packed, ...)          -> acc (int32)
+    bitnet_check_device_errors()               -> watchdog word (0 = clean)
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Sequence
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libbitnet.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(
+        f"{LIB_PATH} is missing: build it with `python -m ternary_w2a8_linear_token_b200.build` "
+        "(there is no non-CUDA fallback)")
+
+lib = ctypes.CDLL(LIB_PATH)
+
+# ----------------------------------------------------------------------------- constants
+OK, ERR_NULL, ERR_SHAPE, ERR_ALIGN, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT, ERR_WORKSPACE = range(8)
+SCALE_PER_TENSOR, SCALE_PER_ROW = 0, 1
+OUT_BF16, OUT_F32 = 0, 1
+PATH_AUTO, PATH_GEMV, PATH_TC = 0, 1, 2
+GEMV_MAX_M = 8
+MAX_PROJ = 8
+
+_P, _I64, _I32, _SZ = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_size_t
+
+
+class bitnet_proj(ctypes.Structure):
+    _fields_ = [("packed", _P), ("s_w", _P), ("mode", _I32), ("reserved", _I32), ("N", _I64),
+                ("y", _P)]
+
+
+_SIGS = {
+    "bitnet_pack_weights": ([_P, _I64, _I64, ctypes.c_int, _P, _P, _P], ctypes.c_int),
+    "bitnet_pack_ternary": ([_P, _I64, _I64, _P, _P], ctypes.c_int),
+    "bitnet_quant_act": ([_P, _I64, _I64, _P, _P, _P], ctypes.c_int),
+    "bitnet_linear_workspace_size": ([_I64, _I64], _SZ),
+    "bitnet_linear": ([_P, _I64, _I64, _P, _P, ctypes.c_int, _I64, _P, ctypes.c_int, _P, _SZ, _P],
+                      ctypes.c_int),
+    "bitnet_linear_ex": ([_P, _I64, _I64, _P, _P, ctypes.c_int, _I64, _P, ctypes.c_int, _P, _SZ,
+                          ctypes.c_int, _P], ctypes.c_int),
+    "bitnet_linear_batch": ([_P, _I64, _I64, ctypes.POINTER(bitnet_proj), _I32, ctypes.c_int, _P,
+                             _SZ, _P], ctypes.c_int),
+    "bitnet_linear_batch_ex": ([_P, _I64, _I64, ctypes.POINTER(bitnet_proj), _I32, ctypes.c_int,
+                                _P, _SZ, ctypes.c_int, _P], ctypes.c_int),
+    "bitnet_linear_i32": ([_P, _I64, _I64, _P, _I64, _P, _P, _SZ, ctypes.c_int, _P], ctypes.c_int),
+    "bitnet_check_device_errors": ([ctypes.POINTER(_I32)], ctypes.c_int),
+    "bitnet_status_string": ([ctypes.c_int], ctypes.c_char_p),
+    "bitnet_version": ([], _I32),
+}
+for _name, (_args, _res) in _SIGS.items():
+    _f = getattr(lib, _name)
+    _f.argtypes = _args
+    _f.restype = _res
+
+
+class BitnetError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {lib.bitnet_status_string(status).decode()} ({status})")
+
+
+def _check(status: int, where: str):
+    if status != OK:
+        raise BitnetError(status, where)
+
+
+def _stream(stream: Optional[torch.cuda.Stream]) -> int:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return s.cuda_stream
+
+
+def _dev(t: torch.Tensor, dtype: torch.dtype, name: str) -> int:
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t.data_ptr()
+
+
+def _x_ptr(x: torch.Tensor) -> int:
+    if x.dtype == torch.bfloat16:
+        return _dev(x, torch.bfloat16, "x")
+    return _dev(x, torch.int16, "x (bf16 bits)")
+
+
+def workspace_size(M: int, K: int) -> int:
+    return int(lib.bitnet_linear_workspace_size(M, K))
+
+
+def make_workspace(M: int, K: int, device=None) -> torch.Tensor:
+    """A device buffer big enough for the tensor-core path at (M, K) (256-byte aligned)."""
+    n = workspace_size(M, K)
+    return torch.empty(max(n, 256), dtype=torch.uint8, device=device or "cuda")
+
+
+# ----------------------------------------------------------------------------- calls
+def bitnet_pack_weights(W: torch.Tensor, per_row: bool, stream=None):
+    N, K = W.shape
+    packed = torch.empty((N, K // 4), dtype=torch.uint8, device=W.device)
+    s_w = torch.empty(N if per_row else 1, dtype=torch.float32, device=W.device)
+    _check(lib.bitnet_pack_weights(_dev(W, torch.float32, "W"), N, K, int(bool(per_row)),
+                                   packed.data_ptr(), s_w.data_ptr(), _stream(stream)),
+           "bitnet_pack_weights")
+    return packed, s_w
+
+
+def bitnet_pack_ternary(t: torch.Tensor, stream=None) -> torch.Tensor:
+    N, K = t.shape
+    packed = torch.empty((N, K // 4), dtype=torch.uint8, device=t.device)
+    _check(lib.bitnet_pack_ternary(_dev(t, torch.int8, "t"), N, K, packed.data_ptr(),
+                                   _stream(stream)), "bitnet_pack_ternary")
+    return packed
+
+
+def bitnet_quant_act(x: torch.Tensor, stream=None):
+    M, K = x.shape
+    q = torch.empty((M, K), dtype=torch.int8, device=x.device)
+    s_x = torch.empty(M, dtype=torch.float32, device=x.device)
+    _check(lib.bitnet_quant_act(_x_ptr(x), M, K, q.data_ptr(), s_x.data_ptr(), _stream(stream)),
+           "bitnet_quant_act")
+    return q, s_x
+
+
+def _ws_args(workspace: Optional[torch.Tensor], M: int, K: int, path: int, device):
+    need_tc = path == PATH_TC or (path == PATH_AUTO and M > GEMV_MAX_M)
+    if workspace is None:
+        if not need_tc:
+            return None, 0, None
+        workspace = make_workspace(M, K, device)
+    return workspace.data_ptr(), workspace.numel() * workspace.element_size(), workspace
+
+
+def bitnet_linear(x: torch.Tensor, packed: torch.Tensor, s_w: torch.Tensor, per_row: bool,
+                  out_dtype: torch.dtype = torch.bfloat16, y: Optional[torch.Tensor] = None,
+                  workspace: Optional[torch.Tensor] = None, path: int = PATH_AUTO, stream=None):
+    M, K = x.shape
+    N = packed.shape[0]
+    if packed.shape[1] * 4 != K:
+        raise ValueError("packed must be (N, K/4)")
+    if y is None:
+        y = torch.empty((M, N), dtype=out_dtype, device=x.device)
+    od = OUT_BF16 if y.dtype == torch.bfloat16 else OUT_F32
+    wp, wb, _keep = _ws_args(workspace, M, K, path, x.device)
+    _check(lib.bitnet_linear_ex(_x_ptr(x), M, K, _dev(packed, torch.uint8, "packed"),
+                                _dev(s_w, torch.float32, "s_w"), int(bool(per_row)), N,
+                                _dev(y, y.dtype, "y"), od, wp, wb, path, _stream(stream)),
+           "bitnet_linear")
+    return y
+
+
+def bitnet_linear_batch(x: torch.Tensor, projs: Sequence, out_dtype: torch.dtype = torch.bfloat16,
+                        ys: Optional[Sequence[torch.Tensor]] = None,
+                        workspace: Optional[torch.Tensor] = None, path: int = PATH_AUTO,
+                        stream=None):
+    """projs: sequence of (packed, s_w, per_row). Returns the list of outputs (M, N_i)."""
+    M, K = x.shape
+    n = len(projs)
+    if not 1 <= n <= MAX_PROJ:
+        raise ValueError(f"1..{MAX_PROJ} projections")
+    if ys is None:
+        ys = [torch.empty((M, p[0].shape[0]), dtype=out_dtype, device=x.device) for p in projs]
+    od = OUT_BF16 if ys[0].dtype == torch.bfloat16 else OUT_F32
+    arr = (bitnet_proj * n)()
+    for i, (packed, s_w, per_row) in enumerate(projs):
+        arr[i].packed = _dev(packed, torch.uint8, "packed")
+        arr[i].s_w = _dev(s_w, torch.float32, "s_w")
+        arr[i].mode = int(bool(per_row))
+        arr[i].reserved = 0
+        arr[i].N = packed.shape[0]
+        arr[i].y = _dev(ys[i], ys[i].dtype, "y")
+    wp, wb, _keep = _ws_args(workspace, M, K, path, x.device)
+    _check(lib.bitnet_linear_batch_ex(_x_ptr(x), M, K, arr, n, od, wp, wb, path, _stream(stream)),
+           "bitnet_linear_batch")
+    return list(ys)
+
+
+def bitnet_linear_i32(q: torch.Tensor, packed: torch.Tensor, path: int = PATH_AUTO,
+                      workspace: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    M, K = q.shape
+    N = packed.shape[0]
+    acc = torch.empty((M, N), dtype=torch.int32, device=q.device)
+    wp, wb, _keep = _ws_args(workspace, M, K, path, q.device)
+    _check(lib.bitnet_linear_i32(_dev(q, torch.int8, "q"), M, K,
+                                 _dev(packed, torch.uint8, "packed"), N, acc.data_ptr(), wp, wb,
+                                 path, _stream(stream)), "bitnet_linear_i32")
+    return acc
+
+
+def bitnet_check_device_errors() -> int:
+    flags = _I32(0)
+    st = lib.bitnet_check_device_errors(ctypes.byref(flags))
+    if st not in (OK, ERR_TIMEOUT):
+        raise BitnetError(st, "bitnet_check_device_errors")
+    return int(flags.value)
+
+
+def bitnet_version() -> int:
+    return int(lib.bitnet_version())

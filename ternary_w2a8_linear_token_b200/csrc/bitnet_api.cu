@@ -1,0 +1,327 @@
+// C-ABI host layer of libbitnet: argument checks, kernel-path choice, TMA descriptor
+// encoding and launches on the caller's stream. Declarations and contracts: include/bitnet.h.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cstring>
+#include <mutex>
+
+#include "bitnet.h"
+#include "bitnet_internal.h"
+
+// The watchdog word every kernel reports bounded-wait expiries into.
+__device__ int32_t g_bitnet_watchdog;
+
+namespace bitnet {
+namespace {
+
+constexpr int kMaxDevices = 64;
+int32_t* g_err_ptr[kMaxDevices] = {};
+std::mutex g_err_mu;
+
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+bitnet_status from_cuda(cudaError_t e) { return e == cudaSuccess ? BITNET_OK : BITNET_ERR_CUDA; }
+
+// K, M, N shared checks.
+bitnet_status check_mk(int64_t M, int64_t K) {
+    if (M < 1 || K < 1 || M >= (int64_t(1) << 31) || K >= (int64_t(1) << 31)) return BITNET_ERR_SHAPE;
+    if (K % 4 != 0) return BITNET_ERR_SHAPE;
+    if (K % 64 != 0) return BITNET_ERR_UNSUPPORTED;
+    return BITNET_OK;
+}
+
+bitnet_status check_n(int64_t N) {
+    return (N < 1 || N >= (int64_t(1) << 31)) ? BITNET_ERR_SHAPE : BITNET_OK;
+}
+
+// Validated batch description shared by bitnet_linear and bitnet_linear_batch.
+struct Batch {
+    int nproj;
+    bitnet_proj proj[kMaxProj];
+};
+
+bitnet_status validate_batch(const void* x, int64_t M, int64_t K, const bitnet_proj* projs,
+                             int32_t nproj, int out_kind, Batch* b) {
+    if (!x || !projs) return BITNET_ERR_NULL;
+    bitnet_status st = check_mk(M, K);
+    if (st != BITNET_OK) return st;
+    if (nproj < 1 || nproj > kMaxProj) return BITNET_ERR_SHAPE;
+    if (out_kind < 0 || out_kind > 2) return BITNET_ERR_UNSUPPORTED;
+    if (!aligned(x, 16)) return BITNET_ERR_ALIGN;
+    b->nproj = nproj;
+    for (int i = 0; i < nproj; ++i) {
+        const bitnet_proj& pr = projs[i];
+        if (!pr.packed || !pr.y || (out_kind != 2 && !pr.s_w)) return BITNET_ERR_NULL;
+        if ((st = check_n(pr.N)) != BITNET_OK) return st;
+        if (pr.mode != BITNET_SCALE_PER_TENSOR && pr.mode != BITNET_SCALE_PER_ROW)
+            return BITNET_ERR_UNSUPPORTED;
+        if (pr.reserved != 0) return BITNET_ERR_UNSUPPORTED;
+        if (!aligned(pr.packed, 16) || !aligned(pr.y, 16) || (pr.s_w && !aligned(pr.s_w, 4)))
+            return BITNET_ERR_ALIGN;
+        b->proj[i] = pr;
+    }
+    return BITNET_OK;
+}
+
+bitnet_status check_workspace(void* ws, size_t bytes, int64_t M, int64_t K) {
+    if (!ws || bytes < ws_total_bytes(M, K)) return BITNET_ERR_WORKSPACE;
+    if (!aligned(ws, 256)) return BITNET_ERR_ALIGN;
+    return BITNET_OK;
+}
+
+bool use_gemv(int64_t M, int64_t K, bitnet_path path) {
+    if (path == BITNET_PATH_GEMV) return true;
+    if (path == BITNET_PATH_TC) return false;
+    return M <= BITNET_GEMV_MAX_M && gemv_supported(M, K);
+}
+
+// Runs a validated batch. x_bf16 or q_in (int8, contraction-only) is the input.
+bitnet_status run_batch(const uint16_t* x_bf16, const int8_t* q_in, int64_t M, int64_t K,
+                        const Batch& b, int out_kind, void* workspace, size_t workspace_bytes,
+                        bitnet_path path, cudaStream_t stream) {
+    if (use_gemv(M, K, path)) {
+        if (!gemv_supported(M, K)) return BITNET_ERR_UNSUPPORTED;
+        GemvParams p;
+        std::memset(&p, 0, sizeof(p));
+        p.x = x_bf16;
+        p.q_in = q_in;
+        p.K = K;
+        p.M = static_cast<int32_t>(M);
+        p.nproj = b.nproj;
+        p.out_kind = out_kind;
+        int64_t rows = 0;
+        for (int i = 0; i < b.nproj; ++i) {
+            p.proj[i].packed = b.proj[i].packed;
+            p.proj[i].s_w = b.proj[i].s_w;
+            p.proj[i].y = b.proj[i].y;
+            p.proj[i].N = b.proj[i].N;
+            p.proj[i].per_row = b.proj[i].mode == BITNET_SCALE_PER_ROW;
+            p.proj[i].row_begin = rows;
+            rows += b.proj[i].N;
+        }
+        p.total_rows = rows;
+        return from_cuda(launch_gemv(p, stream, /*pdl=*/true));
+    }
+
+    bitnet_status st = check_workspace(workspace, workspace_bytes, M, K);
+    if (st != BITNET_OK) return st;
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    int8_t* q_ws = reinterpret_cast<int8_t*>(ws);
+    float* s_x = reinterpret_cast<float*>(ws + ws_q_bytes(M, K));
+    float* r_x = reinterpret_cast<float*>(ws + ws_q_bytes(M, K) + ws_scale_bytes(M));
+
+    TcParams p;
+    std::memset(&p, 0, sizeof(p));
+    const int bn = tc_pick_bn(M);
+    if (!encode_tmap_2d_u8(&p.tmap_q, q_ws, uint64_t(K), uint64_t(M), uint64_t(K), 128,
+                           uint32_t(bn), /*swizzle128=*/true))
+        return BITNET_ERR_CUDA;
+    int tiles = 0;
+    for (int i = 0; i < b.nproj; ++i) {
+        const int64_t N = b.proj[i].N;
+        if (!encode_tmap_2d_u8(&p.tmap_w[i], b.proj[i].packed, uint64_t(K / 4), uint64_t(N),
+                               uint64_t(K / 4), 32, 128, /*swizzle128=*/false))
+            return BITNET_ERR_CUDA;
+        p.proj[i].s_w = b.proj[i].s_w;
+        p.proj[i].y = b.proj[i].y;
+        p.proj[i].N = N;
+        p.proj[i].per_row = b.proj[i].mode == BITNET_SCALE_PER_ROW;
+        p.proj[i].tile_begin = tiles;
+        tiles += static_cast<int>((N + 127) / 128);
+    }
+    p.r_x = r_x;
+    p.err = device_error_word();
+    if (!p.err) return BITNET_ERR_CUDA;
+    p.K = K;
+    p.M = static_cast<int32_t>(M);
+    p.nproj = b.nproj;
+    p.n_tiles_total = tiles;
+    p.out_kind = out_kind;
+
+    cudaError_t e = launch_quant(x_bf16, q_in, M, K, q_ws, q_in ? nullptr : s_x,
+                                 q_in ? nullptr : r_x, /*permuted=*/1, stream, /*pdl=*/true);
+    if (e != cudaSuccess) return BITNET_ERR_CUDA;
+    return from_cuda(launch_tc_gemm(p, bn, stream, /*pdl=*/true));
+}
+
+}  // namespace
+
+int32_t* device_error_word() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+    std::lock_guard<std::mutex> lk(g_err_mu);
+    if (!g_err_ptr[dev]) {
+        void* ptr = nullptr;
+        if (cudaGetSymbolAddress(&ptr, g_bitnet_watchdog) != cudaSuccess) return nullptr;
+        g_err_ptr[dev] = static_cast<int32_t*>(ptr);
+    }
+    return g_err_ptr[dev];
+}
+
+bool encode_tmap_2d_u8(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer,
+                       uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer,
+                       bool swizzle128) {
+    std::call_once(g_encode_once, [] {
+        void* fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    });
+    if (!g_encode) return false;
+    const cuuint64_t dims[2] = {inner, outer};
+    const cuuint64_t strides[1] = {row_stride_bytes};
+    const cuuint32_t box[2] = {box_inner, box_outer};
+    const cuuint32_t estride[2] = {1, 1};
+    const CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base),
+                                dims, strides, box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                                swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                                CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+}  // namespace bitnet
+
+using namespace bitnet;
+
+extern "C" {
+
+bitnet_status bitnet_pack_weights(const float* W, int64_t N, int64_t K, bitnet_scale_mode mode,
+                                  uint8_t* packed, float* s_w, void* stream) {
+    if (!W || !packed || !s_w) return BITNET_ERR_NULL;
+    bitnet_status st = check_mk(1, K);
+    if (st != BITNET_OK) return st;
+    if ((st = check_n(N)) != BITNET_OK) return st;
+    if (mode != BITNET_SCALE_PER_TENSOR && mode != BITNET_SCALE_PER_ROW) return BITNET_ERR_UNSUPPORTED;
+    if (!aligned(W, 16) || !aligned(packed, 16) || !aligned(s_w, 4)) return BITNET_ERR_ALIGN;
+    return from_cuda(launch_pack_weights(W, N, K, mode == BITNET_SCALE_PER_ROW, packed, s_w,
+                                         static_cast<cudaStream_t>(stream)));
+}
+
+bitnet_status bitnet_pack_ternary(const int8_t* t, int64_t N, int64_t K, uint8_t* packed,
+                                  void* stream) {
+    if (!t || !packed) return BITNET_ERR_NULL;
+    bitnet_status st = check_mk(1, K);
+    if (st != BITNET_OK) return st;
+    if ((st = check_n(N)) != BITNET_OK) return st;
+    if (!aligned(t, 16) || !aligned(packed, 16)) return BITNET_ERR_ALIGN;
+    return from_cuda(launch_pack_ternary(t, N, K, packed, static_cast<cudaStream_t>(stream)));
+}
+
+bitnet_status bitnet_quant_act(const uint16_t* x, int64_t M, int64_t K, int8_t* q, float* s_x,
+                               void* stream) {
+    if (!x || !q || !s_x) return BITNET_ERR_NULL;
+    bitnet_status st = check_mk(M, K);
+    if (st != BITNET_OK) return st;
+    if (!aligned(x, 16) || !aligned(q, 16) || !aligned(s_x, 4)) return BITNET_ERR_ALIGN;
+    return from_cuda(launch_quant(x, nullptr, M, K, q, s_x, nullptr, /*permuted=*/0,
+                                  static_cast<cudaStream_t>(stream), /*pdl=*/false));
+}
+
+size_t bitnet_linear_workspace_size(int64_t M, int64_t K) {
+    if (M < 1 || K < 1) return 0;
+    return ws_total_bytes(M, K);
+}
+
+bitnet_status bitnet_linear_batch_ex(const uint16_t* x, int64_t M, int64_t K,
+                                     const bitnet_proj* projs, int32_t nproj,
+                                     bitnet_out_dtype out_dtype, void* workspace,
+                                     size_t workspace_bytes, bitnet_path path, void* stream) {
+    if (out_dtype != BITNET_OUT_BF16 && out_dtype != BITNET_OUT_F32) return BITNET_ERR_UNSUPPORTED;
+    if (path != BITNET_PATH_AUTO && path != BITNET_PATH_GEMV && path != BITNET_PATH_TC)
+        return BITNET_ERR_UNSUPPORTED;
+    Batch b;
+    bitnet_status st = validate_batch(x, M, K, projs, nproj, int(out_dtype), &b);
+    if (st != BITNET_OK) return st;
+    return run_batch(x, nullptr, M, K, b, int(out_dtype), workspace, workspace_bytes, path,
+                     static_cast<cudaStream_t>(stream));
+}
+
+bitnet_status bitnet_linear_batch(const uint16_t* x, int64_t M, int64_t K,
+                                  const bitnet_proj* projs, int32_t nproj,
+                                  bitnet_out_dtype out_dtype, void* workspace,
+                                  size_t workspace_bytes, void* stream) {
+    return bitnet_linear_batch_ex(x, M, K, projs, nproj, out_dtype, workspace, workspace_bytes,
+                                  BITNET_PATH_AUTO, stream);
+}
+
+bitnet_status bitnet_linear_ex(const uint16_t* x, int64_t M, int64_t K, const uint8_t* packed,
+                               const float* s_w, bitnet_scale_mode mode, int64_t N, void* y,
+                               bitnet_out_dtype out_dtype, void* workspace,
+                               size_t workspace_bytes, bitnet_path path, void* stream) {
+    bitnet_proj pr;
+    pr.packed = packed;
+    pr.s_w = s_w;
+    pr.mode = int32_t(mode);
+    pr.reserved = 0;
+    pr.N = N;
+    pr.y = y;
+    return bitnet_linear_batch_ex(x, M, K, &pr, 1, out_dtype, workspace, workspace_bytes, path,
+                                  stream);
+}
+
+bitnet_status bitnet_linear(const uint16_t* x, int64_t M, int64_t K, const uint8_t* packed,
+                            const float* s_w, bitnet_scale_mode mode, int64_t N, void* y,
+                            bitnet_out_dtype out_dtype, void* workspace, size_t workspace_bytes,
+                            void* stream) {
+    return bitnet_linear_ex(x, M, K, packed, s_w, mode, N, y, out_dtype, workspace,
+                            workspace_bytes, BITNET_PATH_AUTO, stream);
+}
+
+bitnet_status bitnet_linear_i32(const int8_t* q, int64_t M, int64_t K, const uint8_t* packed,
+                                int64_t N, int32_t* acc, void* workspace, size_t workspace_bytes,
+                                bitnet_path path, void* stream) {
+    if (path != BITNET_PATH_AUTO && path != BITNET_PATH_GEMV && path != BITNET_PATH_TC)
+        return BITNET_ERR_UNSUPPORTED;
+    bitnet_proj pr;
+    pr.packed = packed;
+    pr.s_w = nullptr;
+    pr.mode = BITNET_SCALE_PER_TENSOR;
+    pr.reserved = 0;
+    pr.N = N;
+    pr.y = acc;
+    Batch b;
+    bitnet_status st = validate_batch(q, M, K, &pr, 1, /*out_kind=*/2, &b);
+    if (st != BITNET_OK) return st;
+    return run_batch(nullptr, q, M, K, b, 2, workspace, workspace_bytes, path,
+                     static_cast<cudaStream_t>(stream));
+}
+
+bitnet_status bitnet_check_device_errors(int32_t* flags) {
+    if (!flags) return BITNET_ERR_NULL;
+    int32_t* dptr = device_error_word();
+    if (!dptr) return BITNET_ERR_CUDA;
+    if (cudaDeviceSynchronize() != cudaSuccess) return BITNET_ERR_CUDA;
+    int32_t v = 0;
+    if (cudaMemcpy(&v, dptr, sizeof(v), cudaMemcpyDeviceToHost) != cudaSuccess) return BITNET_ERR_CUDA;
+    const int32_t zero = 0;
+    if (cudaMemcpy(dptr, &zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess)
+        return BITNET_ERR_CUDA;
+    *flags = v;
+    return v ? BITNET_ERR_TIMEOUT : BITNET_OK;
+}
+
+const char* bitnet_status_string(bitnet_status status) {
+    switch (status) {
+        case BITNET_OK: return "ok";
+        case BITNET_ERR_NULL: return "null pointer";
+        case BITNET_ERR_SHAPE: return "bad shape";
+        case BITNET_ERR_ALIGN: return "misaligned pointer";
+        case BITNET_ERR_UNSUPPORTED: return "unsupported argument";
+        case BITNET_ERR_CUDA: return "CUDA error";
+        case BITNET_ERR_TIMEOUT: return "kernel wait timed out";
+        case BITNET_ERR_WORKSPACE: return "workspace missing or too small";
+    }
+    return "unknown status";
+}
+
+int32_t bitnet_version(void) { return 100; }
+
+}  // extern "C"

@@ -1,0 +1,97 @@
+// Internal declarations shared by the kernel translation units and the C-ABI layer.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cstddef>
+#include <cstdint>
+
+#include "bitnet.h"
+
+namespace bitnet {
+
+constexpr int kMaxProj = BITNET_MAX_PROJ;
+
+// ----------------------------------------------------------------------------- workspace
+// Tensor-core path scratch: q (M, K) int8 in the in-group permuted K order, s_x (M) and
+// r_x = 1/s_x (M), each region 256-byte aligned.
+inline size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
+inline size_t ws_q_bytes(int64_t M, int64_t K) { return align256(size_t(M) * size_t(K)); }
+inline size_t ws_scale_bytes(int64_t M) { return align256(size_t(M) * 4); }
+inline size_t ws_total_bytes(int64_t M, int64_t K) {
+    return ws_q_bytes(M, K) + 2 * ws_scale_bytes(M);
+}
+
+// ----------------------------------------------------------------------------- GEMV
+struct GemvProj {
+    const uint8_t* packed;
+    const float* s_w;
+    void* y;
+    int64_t N;
+    int64_t row_begin;  // first global row of this projection
+    int32_t per_row;
+    int32_t pad;
+};
+
+struct GemvParams {
+    const uint16_t* x;   // (M, K) bf16 bits, or nullptr when q_in is used
+    const int8_t* q_in;  // (M, K) int8 natural order (contraction-only mode)
+    int64_t K;
+    int64_t total_rows;
+    int32_t M;
+    int32_t nproj;
+    int32_t out_kind;  // 0 bf16, 1 f32, 2 int32 accumulator
+    int32_t pad;
+    GemvProj proj[kMaxProj];
+};
+
+cudaError_t launch_gemv(const GemvParams& p, cudaStream_t stream, bool pdl);
+bool gemv_supported(int64_t M, int64_t K);
+
+// ----------------------------------------------------------------------------- quantisation
+// mode 0: natural-order q (public bitnet_quant_act); mode 1: permuted q + s_x + r_x for
+// the tensor-core path. q_in != nullptr: copy-permute given int8 q (no scales).
+cudaError_t launch_quant(const uint16_t* x, const int8_t* q_in, int64_t M, int64_t K, int8_t* q,
+                         float* s_x, float* r_x, int permuted, cudaStream_t stream, bool pdl);
+
+// ----------------------------------------------------------------------------- packing
+cudaError_t launch_pack_weights(const float* W, int64_t N, int64_t K, int per_row,
+                                uint8_t* packed, float* s_w, cudaStream_t stream);
+cudaError_t launch_pack_ternary(const int8_t* t, int64_t N, int64_t K, uint8_t* packed,
+                                cudaStream_t stream);
+
+// ----------------------------------------------------------------------------- tensor-core GEMM
+struct TcProj {
+    const float* s_w;
+    void* y;
+    int64_t N;
+    int32_t per_row;
+    int32_t tile_begin;  // first n-tile index of this projection in the flattened grid
+};
+
+struct alignas(64) TcParams {
+    CUtensorMap tmap_w[kMaxProj];  // packed weights (N, K/4) u8, box {32, 128}
+    CUtensorMap tmap_q;            // workspace q (M, K) s8, box {128, BN}, 128-byte swizzle
+    TcProj proj[kMaxProj];
+    const float* r_x;  // (M) 1 / s_x
+    int32_t* err;      // watchdog word
+    int64_t K;
+    int32_t M;
+    int32_t nproj;
+    int32_t n_tiles_total;
+    int32_t out_kind;  // 0 bf16, 1 f32, 2 int32
+};
+
+// Token-tile width chosen for M.
+int tc_pick_bn(int64_t M);
+cudaError_t launch_tc_gemm(const TcParams& p, int bn, cudaStream_t stream, bool pdl);
+
+// Encodes the TMA descriptors (driver entry point fetched through the runtime).
+bool encode_tmap_2d_u8(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer,
+                       uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer,
+                       bool swizzle128);
+
+// Device watchdog word of the current device.
+int32_t* device_error_word();
+
+}  // namespace bitnet

@@ -1,0 +1,137 @@
+// Per-token absmax int8 activation quantiser (page "BitNet-Triton", section
+// "技术架构：融合内核的三重优化", item 3 "融合激活量化": one launch instead of a chain of
+// framework ops; page "BitNet 1-bit LLM推理优化", section 3.2 "激活量化策略").
+//   amax = max_k |x[m,k]|, s_x = 127 / max(amax, 1e-5), q = clamp(rint(x * s_x), -128, 127).
+//
+// One CTA per token. Pass 1 reduces amax over the bf16 bit patterns (|x| ordered as an
+// unsigned integer), pass 2 re-reads x (an L2 hit) and writes q. Two output layouts:
+//  - natural (M, K) int8, the public bitnet_quant_act result;
+//  - permuted, the operand layout of the tensor-core path: inside every group of 16
+//    values along K, byte 4i + b holds k = 4b + i. That is the order in which a packed
+//    32-bit weight word unpacks with shifts and masks alone ((w >> 2i) & 0x03030303
+//    yields k = i, 4+i, 8+i, 12+i), so the weights need no byte shuffles. Adjacent lanes
+//    own the two 8-value halves of a group and swap 16-bit pieces with one shuffle.
+#include <cuda_runtime.h>
+
+#include "bitnet_device.cuh"
+#include "bitnet_internal.h"
+
+namespace bitnet {
+namespace {
+
+constexpr float kEps = 1e-5f;
+constexpr int kThreads = 256;
+
+__device__ __forceinline__ float bf16_bits_to_float(uint32_t b) {
+    return __uint_as_float(b << 16);
+}
+
+__device__ __forceinline__ uint32_t quant_pair(uint32_t two_bf16, float s) {
+    const int a = __float2int_rn(__fmul_rn(bf16_bits_to_float(two_bf16 & 0xFFFFu), s));
+    const int b = __float2int_rn(__fmul_rn(bf16_bits_to_float(two_bf16 >> 16), s));
+    const int qa = min(max(a, -128), 127);
+    const int qb = min(max(b, -128), 127);
+    return (static_cast<uint32_t>(qa) & 0xFFu) | ((static_cast<uint32_t>(qb) & 0xFFu) << 8);
+}
+
+// 8 bf16 (one uint4) -> 8 int8 as two 32-bit words (values k..k+3, k+4..k+7).
+__device__ __forceinline__ uint2 quant8(const uint4 v, float s) {
+    uint2 r;
+    r.x = quant_pair(v.x, s) | (quant_pair(v.y, s) << 16);
+    r.y = quant_pair(v.z, s) | (quant_pair(v.w, s) << 16);
+    return r;
+}
+
+__device__ __forceinline__ uint32_t absmax8_bits(const uint4 v) {
+    const uint32_t a = max(max(v.x & 0x7FFFu, v.x >> 16 & 0x7FFFu), max(v.y & 0x7FFFu, v.y >> 16 & 0x7FFFu));
+    const uint32_t b = max(max(v.z & 0x7FFFu, v.z >> 16 & 0x7FFFu), max(v.w & 0x7FFFu, v.w >> 16 & 0x7FFFu));
+    return max(a, b);
+}
+
+// Turns the natural-order words (lo = k..k+3, hi = k+4..k+7) held by lane pair
+// (2p, 2p+1) of one 16-group into that lane's 8 bytes of the permuted group.
+__device__ __forceinline__ uint2 permute_group_half(uint2 nat, int h) {
+    const uint32_t p01 = __byte_perm(nat.x, nat.y, 0x5140);  // pieces for words 0 and 1
+    const uint32_t p23 = __byte_perm(nat.x, nat.y, 0x7362);  // pieces for words 2 and 3
+    const uint32_t own = h ? p23 : p01;
+    const uint32_t send = h ? p01 : p23;
+    const uint32_t recv = __shfl_xor_sync(0xFFFFFFFFu, send, 1);
+    const uint32_t lo = h ? recv : own;  // pieces from the first 8 values of the group
+    const uint32_t hi = h ? own : recv;  // pieces from the last 8 values of the group
+    return make_uint2(__byte_perm(lo, hi, 0x5410), __byte_perm(lo, hi, 0x7632));
+}
+
+__global__ void __launch_bounds__(kThreads) quant_rows_kernel(const uint16_t* __restrict__ x,
+                                                              const int8_t* __restrict__ q_in,
+                                                              int64_t K, int8_t* __restrict__ q,
+                                                              float* __restrict__ s_x,
+                                                              float* __restrict__ r_x,
+                                                              int permuted) {
+    __shared__ uint32_t s_red[kThreads / 32];
+    const int64_t m = blockIdx.x;
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int64_t pieces = K / 8;  // 8 values per piece; K % 64 == 0 so pieces is even
+
+    pdl_wait();
+    pdl_trigger();
+
+    float s = 0.0f;
+    if (q_in == nullptr) {
+        const uint4* xr = reinterpret_cast<const uint4*>(x + m * K);
+        uint32_t mx = 0;
+        for (int64_t c = threadIdx.x; c < pieces; c += kThreads) mx = max(mx, absmax8_bits(xr[c]));
+        mx = __reduce_max_sync(0xFFFFFFFFu, mx);
+        if (lane == 0) s_red[warp] = mx;
+        __syncthreads();
+        uint32_t all = s_red[0];
+#pragma unroll
+        for (int w = 1; w < kThreads / 32; ++w) all = max(all, s_red[w]);
+        const float amax = bf16_bits_to_float(all);
+        s = __fdiv_rn(127.0f, fmaxf(amax, kEps));
+        if (threadIdx.x == 0) {
+            if (s_x) s_x[m] = s;
+            if (r_x) r_x[m] = __frcp_rn(s);
+        }
+    }
+
+    int8_t* qr = q + m * K;
+    // Warp-uniform trip count so the pair shuffle always has both lanes present.
+    for (int64_t base = int64_t(warp) * 32; base < pieces; base += kThreads) {
+        const int64_t c = base + lane;
+        const bool valid = c < pieces;
+        uint2 nat = make_uint2(0u, 0u);
+        if (valid) {
+            if (q_in == nullptr) {
+                nat = quant8(reinterpret_cast<const uint4*>(x + m * K)[c], s);
+            } else {
+                nat = reinterpret_cast<const uint2*>(q_in + m * K)[c];
+            }
+        }
+        if (!permuted) {
+            if (valid) reinterpret_cast<uint2*>(qr)[c] = nat;
+        } else {
+            const uint2 out = permute_group_half(nat, lane & 1);
+            if (valid) reinterpret_cast<uint2*>(qr)[c] = out;  // group c/2, half c%2
+        }
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_quant(const uint16_t* x, const int8_t* q_in, int64_t M, int64_t K, int8_t* q,
+                         float* s_x, float* r_x, int permuted, cudaStream_t stream, bool pdl) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(M));
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, quant_rows_kernel, x, q_in, K, q, s_x, r_x, permuted);
+}
+
+}  // namespace bitnet

@@ -1,0 +1,126 @@
+"""Host-side checks of the C ABI: the library loads, exports every declared call, and
+rejects bad arguments before any launch. No GPU is needed: every call here fails its
+argument checks, which run before the library touches CUDA (fake pointers below are
+never dereferenced)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "bitnet.h")
+
+
+@pytest.fixture(scope="module")
+def bn():
+    import ternary_w2a8_linear_token_b200 as bn
+    return bn
+
+
+def declared_functions():
+    src = open(HEADER, encoding="utf-8").read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(bitnet_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for required in ("bitnet_pack_weights", "bitnet_quant_act", "bitnet_linear",
+                     "bitnet_linear_batch"):
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol(bn):
+    missing = [n for n in declared_functions() if not hasattr(bn.lib, n)]
+    assert not missing, f"not exported: {missing}"
+
+
+def test_status_strings_and_version(bn):
+    for code in range(8):
+        assert bn.lib.bitnet_status_string(code)
+    assert bn.lib.bitnet_status_string(99) == b"unknown status"
+    assert bn.bitnet_version() >= 100
+
+
+def test_proj_struct_layout(bn):
+    assert ctypes.sizeof(bn.bitnet_proj) == 40
+    assert bn.bitnet_proj.N.offset == 24 and bn.bitnet_proj.y.offset == 32
+
+
+def test_workspace_size(bn):
+    assert bn.workspace_size(0, 64) == 0
+    ws = bn.workspace_size(300, 2560)
+    assert ws >= 300 * 2560 + 2 * 300 * 4 and ws % 256 == 0
+
+
+FAKE = 0x7F0000000000  # 256-byte aligned, never dereferenced (every call below fails checks)
+
+
+def _linear(bn, x=FAKE, M=256, K=512, packed=FAKE, s_w=FAKE, mode=0, N=128, y=FAKE, od=0,
+            ws=FAKE, wsb=1 << 30, path=0):
+    return bn.lib.bitnet_linear_ex(x, M, K, packed, s_w, mode, N, y, od, ws, wsb, path, None)
+
+
+def test_linear_argument_errors(bn):
+    assert _linear(bn, x=None) == bn.ERR_NULL
+    assert _linear(bn, packed=None) == bn.ERR_NULL
+    assert _linear(bn, s_w=None) == bn.ERR_NULL
+    assert _linear(bn, y=None) == bn.ERR_NULL
+    assert _linear(bn, M=0) == bn.ERR_SHAPE
+    assert _linear(bn, N=0) == bn.ERR_SHAPE
+    assert _linear(bn, K=510) == bn.ERR_SHAPE
+    assert _linear(bn, K=520) == bn.ERR_UNSUPPORTED  # K % 4 == 0 but K % 64 != 0
+    assert _linear(bn, M=1 << 31) == bn.ERR_SHAPE
+    assert _linear(bn, x=FAKE + 8) == bn.ERR_ALIGN
+    assert _linear(bn, packed=FAKE + 4) == bn.ERR_ALIGN
+    assert _linear(bn, y=FAKE + 2) == bn.ERR_ALIGN
+    assert _linear(bn, mode=2) == bn.ERR_UNSUPPORTED
+    assert _linear(bn, od=3) == bn.ERR_UNSUPPORTED
+    assert _linear(bn, path=7) == bn.ERR_UNSUPPORTED
+    # tensor-core path (M > 8): workspace checked before any launch
+    assert _linear(bn, ws=None) == bn.ERR_WORKSPACE
+    assert _linear(bn, wsb=1024) == bn.ERR_WORKSPACE
+    assert _linear(bn, ws=FAKE + 16) == bn.ERR_ALIGN
+    assert _linear(bn, M=4, path=2, ws=None) == bn.ERR_WORKSPACE
+
+
+def test_batch_argument_errors(bn):
+    arr = (bn.bitnet_proj * 9)()
+    for i in range(9):
+        arr[i].packed, arr[i].s_w, arr[i].mode, arr[i].N, arr[i].y = FAKE, FAKE, 0, 64, FAKE
+    f = bn.lib.bitnet_linear_batch
+    assert f(FAKE, 256, 512, arr, 0, 0, FAKE, 1 << 30, None) == bn.ERR_SHAPE
+    assert f(FAKE, 256, 512, arr, 9, 0, FAKE, 1 << 30, None) == bn.ERR_SHAPE
+    arr[1].reserved = 1
+    assert f(FAKE, 256, 512, arr, 2, 0, FAKE, 1 << 30, None) == bn.ERR_UNSUPPORTED
+    arr[1].reserved = 0
+    arr[1].N = -3
+    assert f(FAKE, 256, 512, arr, 2, 0, FAKE, 1 << 30, None) == bn.ERR_SHAPE
+    arr[1].N = 64
+    arr[1].packed = None
+    assert f(FAKE, 256, 512, arr, 2, 0, FAKE, 1 << 30, None) == bn.ERR_NULL
+    arr[1].packed = FAKE
+    assert f(None, 256, 512, arr, 2, 0, FAKE, 1 << 30, None) == bn.ERR_NULL
+    assert f(FAKE, 256, 512, None, 2, 0, FAKE, 1 << 30, None) == bn.ERR_NULL
+    assert f(FAKE, 256, 512, arr, 2, 0, None, 0, None) == bn.ERR_WORKSPACE
+
+
+def test_other_calls_argument_errors(bn):
+    L = bn.lib
+    assert L.bitnet_pack_weights(None, 4, 64, 0, FAKE, FAKE, None) == bn.ERR_NULL
+    assert L.bitnet_pack_weights(FAKE, 4, 66, 0, FAKE, FAKE, None) == bn.ERR_SHAPE
+    assert L.bitnet_pack_weights(FAKE, 4, 96, 0, FAKE, FAKE, None) == bn.ERR_UNSUPPORTED
+    assert L.bitnet_pack_weights(FAKE, 0, 64, 0, FAKE, FAKE, None) == bn.ERR_SHAPE
+    assert L.bitnet_pack_weights(FAKE, 4, 64, 5, FAKE, FAKE, None) == bn.ERR_UNSUPPORTED
+    assert L.bitnet_pack_weights(FAKE + 4, 4, 64, 0, FAKE, FAKE, None) == bn.ERR_ALIGN
+    assert L.bitnet_pack_ternary(FAKE, 4, 60, FAKE, None) == bn.ERR_UNSUPPORTED
+    assert L.bitnet_pack_ternary(FAKE, 4, 64, None, None) == bn.ERR_NULL
+    assert L.bitnet_quant_act(FAKE, 0, 64, FAKE, FAKE, None) == bn.ERR_SHAPE
+    assert L.bitnet_quant_act(FAKE, 3, 64, FAKE + 1, FAKE, None) == bn.ERR_ALIGN
+    assert L.bitnet_quant_act(FAKE, 3, 64, FAKE, None, None) == bn.ERR_NULL
+    assert L.bitnet_linear_i32(FAKE, 16, 64, FAKE, 16, None, FAKE, 1 << 30, 0, None) == bn.ERR_NULL
+    assert L.bitnet_linear_i32(FAKE, 16, 64, FAKE, 16, FAKE, None, 0, 0, None) == bn.ERR_WORKSPACE
+    assert L.bitnet_linear_i32(FAKE, 16, 64, FAKE, 16, FAKE, FAKE, 1 << 30, 9, None) == \
+        bn.ERR_UNSUPPORTED
+    assert L.bitnet_check_device_errors(None) == bn.ERR_NULL

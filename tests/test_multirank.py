@@ -1,0 +1,55 @@
+"""The N > 1 benchmark plumbing on CPU: two gloo ranks, each with its own replica of the
+workload (weak scaling, no data-path collective). The job's time is the max over ranks
+and its work the sum, as bench.py reports it."""
+import os
+import socket
+
+import pytest
+import torch.multiprocessing as mp
+
+
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    return port
+
+
+def _worker(rank, world, port, out):
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    sys.path.insert(0, root)
+    import torch.distributed as dist
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world), LOCAL_RANK=str(rank))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    import bench
+    r, w, lr = bench.dist_env()
+    assert (r, w, lr) == (rank, world, rank)
+    # rank-specific time and work
+    ms, units = bench.reduce_over_ranks(10.0 + 5.0 * rank, 100.0 * (rank + 1), world)
+    out[rank] = (ms, units)
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+def test_two_rank_max_time_sum_work():
+    world = 2
+    port = _free_port()
+    mgr = mp.Manager()
+    out = mgr.dict()
+    ctx = mp.get_context("spawn")
+    procs = [ctx.Process(target=_worker, args=(r, world, port, out)) for r in range(world)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=120)
+    assert all(p.exitcode == 0 for p in procs), [p.exitcode for p in procs]
+    for r in range(world):
+        assert out[r] == (15.0, 300.0)
+
+
+def test_single_rank_is_identity():
+    import bench
+    assert bench.reduce_over_ranks(3.5, 7.0, 1) == (3.5, 7.0)
