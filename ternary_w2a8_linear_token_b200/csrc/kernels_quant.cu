@@ -3,8 +3,8 @@
 // framework ops; page "BitNet 1-bit LLM推理优化", section 3.2 "激活量化策略").
 //   amax = max_k |x[m,k]|, s_x = 127 / max(amax, 1e-5), q = clamp(rint(x * s_x), -128, 127).
 //
-// One CTA per token. Pass 1 reduces amax over the bf16 bit patterns (|x| ordered as an
-// unsigned integer), pass 2 re-reads x (an L2 hit) and writes q. Two output layouts:
+// One warp per token. Pass 1 reduces amax over the bf16 bit patterns (|x| ordered as an
+// unsigned integer), pass 2 re-reads x (an L1/L2 hit) and writes q. Two output layouts:
 //  - natural (M, K) int8, the public bitnet_quant_act result;
 //  - permuted, the operand layout of the tensor-core path: inside every group of 16
 //    values along K, byte 4i + b holds k = 4b + i. That is the order in which a packed
@@ -61,58 +61,74 @@ __device__ __forceinline__ uint2 permute_group_half(uint2 nat, int h) {
     return make_uint2(__byte_perm(lo, hi, 0x5410), __byte_perm(lo, hi, 0x7632));
 }
 
+// One warp per token row; each lane keeps 8 loads in flight. Pass 1 finds amax, pass 2
+// re-reads the row (an L1/L2 hit) and writes q.
+constexpr int kRowsPerCta = kThreads / 32;
+constexpr int kUnroll = 8;
+
 __global__ void __launch_bounds__(kThreads) quant_rows_kernel(const uint16_t* __restrict__ x,
                                                               const int8_t* __restrict__ q_in,
-                                                              int64_t K, int8_t* __restrict__ q,
+                                                              int64_t M, int64_t K,
+                                                              int8_t* __restrict__ q,
                                                               float* __restrict__ s_x,
                                                               float* __restrict__ r_x,
                                                               int permuted) {
-    __shared__ uint32_t s_red[kThreads / 32];
-    const int64_t m = blockIdx.x;
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int64_t pieces = K / 8;  // 8 values per piece; K % 64 == 0 so pieces is even
+    const int64_t m = int64_t(blockIdx.x) * kRowsPerCta + warp;
+    const int64_t pieces = K / 8;  // 8 values per piece; K % 64 == 0 so pieces % 8 == 0
 
     pdl_wait();
     pdl_trigger();
+    if (m >= M) return;  // whole warp leaves together
 
     float s = 0.0f;
+    const uint4* xr = reinterpret_cast<const uint4*>(x + m * K);
     if (q_in == nullptr) {
-        const uint4* xr = reinterpret_cast<const uint4*>(x + m * K);
         uint32_t mx = 0;
-        for (int64_t c = threadIdx.x; c < pieces; c += kThreads) mx = max(mx, absmax8_bits(xr[c]));
-        mx = __reduce_max_sync(0xFFFFFFFFu, mx);
-        if (lane == 0) s_red[warp] = mx;
-        __syncthreads();
-        uint32_t all = s_red[0];
+        for (int64_t c0 = 0; c0 < pieces; c0 += 32 * kUnroll) {
+            uint4 v[kUnroll];
 #pragma unroll
-        for (int w = 1; w < kThreads / 32; ++w) all = max(all, s_red[w]);
-        const float amax = bf16_bits_to_float(all);
-        s = __fdiv_rn(127.0f, fmaxf(amax, kEps));
-        if (threadIdx.x == 0) {
+            for (int u = 0; u < kUnroll; ++u) {
+                const int64_t c = c0 + u * 32 + lane;
+                v[u] = c < pieces ? xr[c] : make_uint4(0u, 0u, 0u, 0u);
+            }
+#pragma unroll
+            for (int u = 0; u < kUnroll; ++u) mx = max(mx, absmax8_bits(v[u]));
+        }
+        mx = __reduce_max_sync(0xFFFFFFFFu, mx);
+        s = __fdiv_rn(127.0f, fmaxf(bf16_bits_to_float(mx), kEps));
+        if (lane == 0) {
             if (s_x) s_x[m] = s;
             if (r_x) r_x[m] = __frcp_rn(s);
         }
     }
 
     int8_t* qr = q + m * K;
-    // Warp-uniform trip count so the pair shuffle always has both lanes present.
-    for (int64_t base = int64_t(warp) * 32; base < pieces; base += kThreads) {
-        const int64_t c = base + lane;
-        const bool valid = c < pieces;
-        uint2 nat = make_uint2(0u, 0u);
-        if (valid) {
-            if (q_in == nullptr) {
-                nat = quant8(reinterpret_cast<const uint4*>(x + m * K)[c], s);
-            } else {
-                nat = reinterpret_cast<const uint2*>(q_in + m * K)[c];
+    for (int64_t c0 = 0; c0 < pieces; c0 += 32 * kUnroll) {
+        uint2 nat[kUnroll];
+        if (q_in == nullptr) {
+            uint4 v[kUnroll];
+#pragma unroll
+            for (int u = 0; u < kUnroll; ++u) {
+                const int64_t c = c0 + u * 32 + lane;
+                v[u] = c < pieces ? xr[c] : make_uint4(0u, 0u, 0u, 0u);
+            }
+#pragma unroll
+            for (int u = 0; u < kUnroll; ++u) nat[u] = quant8(v[u], s);
+        } else {
+#pragma unroll
+            for (int u = 0; u < kUnroll; ++u) {
+                const int64_t c = c0 + u * 32 + lane;
+                nat[u] = c < pieces ? reinterpret_cast<const uint2*>(q_in + m * K)[c]
+                                    : make_uint2(0u, 0u);
             }
         }
-        if (!permuted) {
-            if (valid) reinterpret_cast<uint2*>(qr)[c] = nat;
-        } else {
-            const uint2 out = permute_group_half(nat, lane & 1);
-            if (valid) reinterpret_cast<uint2*>(qr)[c] = out;  // group c/2, half c%2
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) {
+            const int64_t c = c0 + u * 32 + lane;  // c0 + u*32 is even: lane pairs share a group
+            const uint2 out = permuted ? permute_group_half(nat[u], lane & 1) : nat[u];
+            if (c < pieces) reinterpret_cast<uint2*>(qr)[c] = out;
         }
     }
 }
@@ -122,7 +138,7 @@ __global__ void __launch_bounds__(kThreads) quant_rows_kernel(const uint16_t* __
 cudaError_t launch_quant(const uint16_t* x, const int8_t* q_in, int64_t M, int64_t K, int8_t* q,
                          float* s_x, float* r_x, int permuted, cudaStream_t stream, bool pdl) {
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(static_cast<unsigned>(M));
+    cfg.gridDim = dim3(static_cast<unsigned>((M + kRowsPerCta - 1) / kRowsPerCta));
     cfg.blockDim = dim3(kThreads);
     cfg.dynamicSmemBytes = 0;
     cfg.stream = stream;
@@ -131,7 +147,7 @@ cudaError_t launch_quant(const uint16_t* x, const int8_t* q_in, int64_t M, int64
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = pdl ? 1 : 0;
-    return cudaLaunchKernelEx(&cfg, quant_rows_kernel, x, q_in, K, q, s_x, r_x, permuted);
+    return cudaLaunchKernelEx(&cfg, quant_rows_kernel, x, q_in, M, K, q, s_x, r_x, permuted);
 }
 
 }  // namespace bitnet

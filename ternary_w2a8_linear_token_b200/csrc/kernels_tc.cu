@@ -47,11 +47,28 @@ struct TcLayout {
     static constexpr int kStages = (200 * 1024) / kStage > 6 ? 6 : (200 * 1024) / kStage;
     static constexpr int kBarOff = kStages * kStage;
     static constexpr int kBarBytes = (3 * kStages + 1) * 8 + 16;  // + TMEM slot, abort flag
-    static constexpr int kSmem = kBarOff + kBarBytes + 1024;  // + alignment slack
+    static constexpr int kRxOff = kBarOff + kBarBytes;             // BN floats: 1/s_x of the tile
+    static constexpr int kSmem = kRxOff + BN * 4 + 1024;           // + alignment slack
+    static_assert(BN * kBM * 4 <= kStages * kStage, "output staging must fit the stage area");
     static constexpr uint32_t kTmemCols = BN < 32 ? 32 : BN;
     static_assert(kStage % 1024 == 0, "stage must keep 1024-byte alignment");
     static_assert(kStages >= 2, "need at least two stages");
 };
+
+// Barrier among the 8 unpack/epilogue warps only (named barrier 1).
+__device__ __forceinline__ void epilogue_bar_sync() {
+    asm volatile("bar.sync 1, %0;" ::"n"(kUnpackWarps * 32) : "memory");
+}
+
+template <int N>
+__device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, uint32_t (&v)[N]) {
+    static_assert(N % 8 == 0, "columns in multiples of 8");
+#pragma unroll
+    for (int i = 0; i < N / 8; ++i) {
+        uint32_t (&r)[8] = *reinterpret_cast<uint32_t(*)[8]>(&v[8 * i]);
+        tmem_ld_32x32b_x8(taddr + uint32_t(8 * i), r);
+    }
+}
 
 template <int BN>
 __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_constant__ TcParams p) {
@@ -119,6 +136,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
                                   kErrWaitDrain, nullptr);
             }
         }
+        __syncwarp();  // lanes 1-31 wait for the producer lane: the CTA barrier below is aligned
     } else if (warp == 1) {
         if (lane == 0) {
             // ---------------- MMA issuer
@@ -143,6 +161,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
             // Drain: no tensor-core operation may still be running when TMEM is freed.
             mbar_wait_bounded(acc_full, 0, p.err, kErrWaitDrain, nullptr);
         }
+        __syncwarp();  // reconverge before the aligned CTA barrier below
     } else {
         // ---------------- unpack warps
         const int ut = threadIdx.x - 64;  // 0 .. 255
@@ -174,11 +193,22 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
         }
 
         // ---------------- epilogue
+        // 1/s_x of the tile's tokens -> shared memory while the last MMAs run.
         pdl_wait();  // r_x comes from the quantiser grid; y may be read by earlier grids
+        const int et = threadIdx.x - 64;  // 0 .. 255
+        float* s_rx = reinterpret_cast<float*>(smem + L::kRxOff);
+        for (int i = et; i < BN; i += kUnpackWarps * 32) {
+            const int64_t m = int64_t(m0) + i;
+            s_rx[i] = (p.out_kind != 2 && m < p.M) ? p.r_x[m] : 0.0f;
+        }
+        epilogue_bar_sync();
         mbar_wait_bounded(acc_full, 0, p.err, kErrWaitAccum, abort_flag);
         tc_fence_after();
-        const int quarter = warp & 3;               // TMEM lanes 32*quarter ... +31
-        const int colhalf = (warp - 2) >> 2;        // which half of the BN columns
+
+        // TMEM (lane = weight row, column = token) -> registers -> dequantised values staged in
+        // the idle stage area as rows of the output: stage[token][weight row].
+        const int quarter = warp & 3;         // TMEM lanes 32*quarter ... +31
+        const int colhalf = (warp - 2) >> 2;  // which half of the BN columns
         const int n_local = quarter * 32 + lane;
         const TcProj& pr = p.proj[j];
         const int64_t n = int64_t(n0) + n_local;
@@ -187,29 +217,57 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
         const float sw = p.out_kind == 2 ? 0.0f
                          : pr.per_row   ? (nvalid ? pr.s_w[n] : 0.0f)
                                         : pr.s_w[0];
+        const int esz = p.out_kind == 0 ? 2 : 4;
+        uint8_t* stage = smem;
         constexpr int kHalfCols = BN / 2;
-        constexpr int kChunks = kHalfCols >= 8 ? kHalfCols / 8 : 1;
+        constexpr int kLd = kHalfCols >= 32 ? 32 : kHalfCols;  // columns per TMEM load
 #pragma unroll 1
-        for (int cc = 0; cc < kChunks; ++cc) {
-            const int col0 = colhalf * kHalfCols + cc * 8;
-            uint32_t v[8];
-            tmem_ld_32x32b_x8(tmem_d + (uint32_t(quarter * 32) << 16) + uint32_t(col0), v);
+        for (int cc = 0; cc < kHalfCols; cc += kLd) {
+            const int col0 = colhalf * kHalfCols + cc;
+            uint32_t v[kLd];
+            tmem_ld_cols<kLd>(tmem_d + (uint32_t(quarter * 32) << 16) + uint32_t(col0), v);
             tmem_ld_wait();
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const int64_t m = int64_t(m0) + col0 + i;
-                if (nvalid && m < p.M) {
-                    const int32_t a = static_cast<int32_t>(v[i]);
-                    const int64_t o = m * pr.N + n;
-                    if (p.out_kind == 2) {
-                        reinterpret_cast<int32_t*>(pr.y)[o] = a;
-                    } else {
-                        const float yv = __fmul_rn(__int2float_rn(a), __fmul_rn(sw, p.r_x[m]));
-                        if (p.out_kind == 0)
-                            reinterpret_cast<__nv_bfloat16*>(pr.y)[o] = __float2bfloat16_rn(yv);
-                        else
-                            reinterpret_cast<float*>(pr.y)[o] = yv;
-                    }
+            for (int i = 0; i < kLd; ++i) {
+                const int col = col0 + i;
+                const int32_t a = static_cast<int32_t>(v[i]);
+                uint8_t* dst = stage + (size_t(col) * kBM + n_local) * esz;
+                if (p.out_kind == 2) {
+                    *reinterpret_cast<int32_t*>(dst) = a;
+                } else {
+                    const float yv = __fmul_rn(__int2float_rn(a), __fmul_rn(sw, s_rx[col]));
+                    if (p.out_kind == 0)
+                        *reinterpret_cast<__nv_bfloat16*>(dst) = __float2bfloat16_rn(yv);
+                    else
+                        *reinterpret_cast<float*>(dst) = yv;
+                }
+            }
+        }
+        epilogue_bar_sync();
+
+        // Coalesced copy-out: each token row of the tile is 128 contiguous outputs.
+        const int row_bytes = kBM * esz;
+        const int chunks_per_row = row_bytes / 16;
+        const int vals_per_chunk = 16 / esz;
+        const bool vec_ok = ((pr.N * esz) % 16) == 0;  // every row start 16-byte aligned
+        uint8_t* ybase = static_cast<uint8_t*>(pr.y);
+        for (int c = et; c < BN * chunks_per_row; c += kUnpackWarps * 32) {
+            const int row = c / chunks_per_row;
+            const int ch = c - row * chunks_per_row;
+            const int64_t m = int64_t(m0) + row;
+            if (m >= p.M) continue;
+            const int64_t nn = int64_t(n0) + int64_t(ch) * vals_per_chunk;
+            const uint8_t* src = stage + size_t(row) * row_bytes + size_t(ch) * 16;
+            uint8_t* dst = ybase + (m * pr.N + nn) * esz;
+            if (vec_ok && nn + vals_per_chunk <= pr.N) {
+                *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(src);
+            } else {
+                for (int e = 0; e < vals_per_chunk; ++e) {
+                    if (nn + e >= pr.N) break;
+                    if (esz == 2)
+                        reinterpret_cast<uint16_t*>(dst)[e] = reinterpret_cast<const uint16_t*>(src)[e];
+                    else
+                        reinterpret_cast<uint32_t*>(dst)[e] = reinterpret_cast<const uint32_t*>(src)[e];
                 }
             }
         }
