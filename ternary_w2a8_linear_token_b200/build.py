@@ -1,6 +1,6 @@
 """Builds libbitnet.so in-tree with nvcc for sm_100a.
 
-    python -m ternary_w2a8_linear_token_b200.build [--force] [--verbose-ptxas]
+    python ternary_w2a8_linear_token_b200/build.py [--force] [--verbose-ptxas]
 
 Each .cu file under csrc/ is compiled to an object (in parallel), then linked into one
 shared library next to this file. CUDA runtime is linked statically; the driver entry
