@@ -180,6 +180,31 @@ bitnet_status bitnet_linear_i32(const int8_t* q, int64_t M, int64_t K, const uin
                                 bitnet_path path, void* stream);
 
 /*
+ * bitnet_linear_noalloc — bitnet_linear for callers that cannot allocate device memory.
+ * The pages have no counterpart to this call; it exists for callers such as a serving
+ * loop in which cudaMalloc could synchronise the device and stall other streams, a plug-in
+ * whose host runtime owns all device memory, or code running while its stream is captured
+ * into a graph. It takes the same arguments as bitnet_linear minus the workspace: the
+ * tensor-core path's scratch is a fixed device array of BITNET_NOALLOC_SCRATCH_BYTES inside
+ * the library, which every GPU that loads the library holds until the process exits.
+ *  - Sizes whose scratch (bitnet_linear_workspace_size(M, K)) exceeds that array are
+ *    rejected with BITNET_ERR_WORKSPACE before anything is launched (M <= BITNET_GEMV_MAX_M
+ *    runs the GEMV, which needs no scratch).
+ *  - The first call on each device looks the array's address up (cudaGetSymbolAddress);
+ *    make that first call before any stream capture on that device.
+ *  - All calls share the one array and it keeps the last call's contents (nothing in it
+ *    needs to start at zero). Calls that may overlap on the GPU — on different streams, or
+ *    from different threads without ordering — race on it and give wrong results.
+ *  - It calls no cudaMalloc, cudaFree or allocating library routine.
+ * Results equal bitnet_linear's bit for bit.
+ */
+#define BITNET_NOALLOC_SCRATCH_BYTES (16 * 1024 * 1024)
+bitnet_status bitnet_linear_noalloc(const uint16_t* x, int64_t M, int64_t K,
+                                    const uint8_t* packed, const float* s_w,
+                                    bitnet_scale_mode mode, int64_t N, void* y,
+                                    bitnet_out_dtype out_dtype, void* stream);
+
+/*
  * bitnet_check_device_errors — synchronises the current device, returns the library's
  * watchdog word in *flags (0 = no kernel gave up a bounded wait since the last check)
  * and clears it. Returns BITNET_ERR_TIMEOUT when the word was non-zero.

@@ -4,7 +4,7 @@ Argument marshalling only: every step of the forward runs in the CUDA kernels be
 the C ABI declared in ``include/bitnet.h``. PyTorch supplies device memory (output and
 workspace tensors) and the current CUDA stream; nothing here computes on tensors.
 
-The shared library is built in-tree by ``python -m ternary_w2a8_linear_token_b200.build``.
+The shared library is built in-tree by ``python ternary_w2a8_linear_token_b200/build.py``.
 Importing this package without it raises ImportError: there is no fallback path.
 
 Functions keep the C names:
@@ -29,7 +29,7 @@ LIB_PATH = os.path.join(_PKG, "libbitnet.so")
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(
-        f"{LIB_PATH} is missing: build it with `python -m ternary_w2a8_linear_token_b200.build` "
+        f"{LIB_PATH} is missing: build it with `python ternary_w2a8_linear_token_b200/build.py` "
         "(there is no non-CUDA fallback)")
 
 lib = ctypes.CDLL(LIB_PATH)
@@ -64,6 +64,8 @@ _SIGS = {
     "bitnet_linear_batch_ex": ([_P, _I64, _I64, ctypes.POINTER(bitnet_proj), _I32, ctypes.c_int,
                                 _P, _SZ, ctypes.c_int, _P], ctypes.c_int),
     "bitnet_linear_i32": ([_P, _I64, _I64, _P, _I64, _P, _P, _SZ, ctypes.c_int, _P], ctypes.c_int),
+    "bitnet_linear_noalloc": ([_P, _I64, _I64, _P, _P, ctypes.c_int, _I64, _P, ctypes.c_int, _P],
+                              ctypes.c_int),
     "bitnet_check_device_errors": ([ctypes.POINTER(_I32)], ctypes.c_int),
     "bitnet_status_string": ([ctypes.c_int], ctypes.c_char_p),
     "bitnet_version": ([], _I32),
@@ -207,6 +209,27 @@ def bitnet_linear_i32(q: torch.Tensor, packed: torch.Tensor, path: int = PATH_AU
                                  _dev(packed, torch.uint8, "packed"), N, acc.data_ptr(), wp, wb,
                                  path, _stream(stream)), "bitnet_linear_i32")
     return acc
+
+
+NOALLOC_SCRATCH_BYTES = 16 * 1024 * 1024
+
+
+def bitnet_linear_noalloc(x: torch.Tensor, packed: torch.Tensor, s_w: torch.Tensor,
+                          per_row: bool, out_dtype: torch.dtype = torch.bfloat16,
+                          y: Optional[torch.Tensor] = None, stream=None):
+    """bitnet_linear without a workspace: for callers that cannot allocate device memory
+    during execution. Uses the library's fixed 16 MiB device scratch array; calls that can
+    overlap on the GPU race on it. Sizes beyond the array raise BitnetError (workspace)."""
+    M, K = x.shape
+    N = packed.shape[0]
+    if y is None:
+        y = torch.empty((M, N), dtype=out_dtype, device=x.device)
+    od = OUT_BF16 if y.dtype == torch.bfloat16 else OUT_F32
+    _check(lib.bitnet_linear_noalloc(_x_ptr(x), M, K, _dev(packed, torch.uint8, "packed"),
+                                     _dev(s_w, torch.float32, "s_w"), int(bool(per_row)), N,
+                                     _dev(y, y.dtype, "y"), od, _stream(stream)),
+           "bitnet_linear_noalloc")
+    return y
 
 
 def bitnet_check_device_errors() -> int:
