@@ -41,7 +41,7 @@ struct GemvParams {
     int32_t M;
     int32_t nproj;
     int32_t out_kind;  // 0 bf16, 1 f32, 2 int32 accumulator
-    int32_t pad;
+    int32_t stage_x;   // set by the launcher: stage x in shared memory
     GemvProj proj[kMaxProj];
 };
 

@@ -57,9 +57,9 @@ __device__ __forceinline__ uint2 permute_group_half(uint2 nat, int h) {
 }
 
 // MT: token capacity (compile time); p.M <= MT tokens are real, the rest are zero.
-// CPL: 16-byte chunks per lane (K <= CPL * 32 * 64). One weight row per warp.
-template <int MT, int CPL>
-__global__ void __launch_bounds__(kThreads) gemv_w2a8_kernel(const __grid_constant__ GemvParams p) {
+// CPL: 16-byte chunks per lane (K <= CPL * 32 * 64). RW: weight rows per warp.
+template <int MT, int CPL, int RW>
+__global__ void __launch_bounds__(kThreads, MT <= 2 ? 2 : 1) gemv_w2a8_kernel(const __grid_constant__ GemvParams p) {
     extern __shared__ uint4 s_q[];  // [MT][4][C] permuted q: word i of group 4c + j
     __shared__ uint32_t s_red[kWarps][MT];  // per-warp amax bits
     __shared__ int32_t s_qsum[kWarps][MT];  // per-warp partial sums of q
@@ -70,26 +70,33 @@ __global__ void __launch_bounds__(kThreads) gemv_w2a8_kernel(const __grid_consta
     const int C = static_cast<int>(K >> 6);  // 16-byte chunks per packed row
     const int Mreal = p.M;
 
-    // ---- 1. this warp's weight row -> registers (no dependency on earlier grids)
-    const int64_t gr = int64_t(blockIdx.x) * kWarps + warp;
-    const bool rvalid = gr < p.total_rows;
-    int pj = 0;
+    // ---- 1. this warp's weight rows -> registers (no dependency on earlier grids)
+    int64_t gr[RW];
+    bool rvalid[RW];
+    int pj[RW];
+    int64_t nrow[RW];
+    uint4 w[RW][CPL];
+    float sw[RW];
 #pragma unroll
-    for (int jj = 1; jj < kMaxProj; ++jj)
-        if (jj < p.nproj && gr >= p.proj[jj].row_begin) pj = jj;
-    const int64_t nrow = gr - p.proj[pj].row_begin;
-    uint4 w[CPL];
-    {
-        const uint8_t* rowp = p.proj[pj].packed + nrow * (K >> 2);
+    for (int r = 0; r < RW; ++r) {
+        gr[r] = (int64_t(blockIdx.x) * kWarps + warp) * RW + r;
+        rvalid[r] = gr[r] < p.total_rows;
+        pj[r] = 0;
+#pragma unroll
+        for (int jj = 1; jj < kMaxProj; ++jj)
+            if (jj < p.nproj && gr[r] >= p.proj[jj].row_begin) pj[r] = jj;
+        nrow[r] = gr[r] - p.proj[pj[r]].row_begin;
+        const uint8_t* rowp = p.proj[pj[r]].packed + nrow[r] * (K >> 2);
 #pragma unroll
         for (int c = 0; c < CPL; ++c) {
             const int chunk = lane + 32 * c;
-            w[c] = (rvalid && chunk < C) ? ldg_stream_v4(rowp + int64_t(chunk) * 16)
-                                         : make_uint4(0u, 0u, 0u, 0u);
+            w[r][c] = (rvalid[r] && chunk < C) ? ldg_stream_v4(rowp + int64_t(chunk) * 16)
+                                               : make_uint4(0u, 0u, 0u, 0u);
         }
+        sw[r] = 0.0f;
+        if (rvalid[r] && p.out_kind != 2)
+            sw[r] = p.proj[pj[r]].per_row ? p.proj[pj[r]].s_w[nrow[r]] : p.proj[pj[r]].s_w[0];
     }
-    float sw = 0.0f;
-    if (rvalid && p.out_kind != 2) sw = p.proj[pj].per_row ? p.proj[pj].s_w[nrow] : p.proj[pj].s_w[0];
 
     pdl_trigger();
     pdl_wait();
@@ -97,10 +104,15 @@ __global__ void __launch_bounds__(kThreads) gemv_w2a8_kernel(const __grid_consta
     // ---- 2. quantise the tokens into shared memory (pieces of 8 values; pieces % 8 == 0)
     const int64_t pieces = K >> 3;
     float s_tok[MT];
+    // x is staged in shared memory (after q) during the amax pass when it fits, so the
+    // quantising pass never goes back to global memory.
+    uint4* s_x = reinterpret_cast<uint4*>(reinterpret_cast<uint8_t*>(s_q) + int64_t(MT) * K);
+    const bool stage_x = p.stage_x != 0;
     if (p.q_in == nullptr) {
         uint32_t mx[MT];
 #pragma unroll
         for (int m = 0; m < MT; ++m) mx[m] = 0;
+#pragma unroll 2
         for (int64_t c = threadIdx.x; c < pieces; c += kThreads) {
             uint4 v[MT];
 #pragma unroll
@@ -109,6 +121,7 @@ __global__ void __launch_bounds__(kThreads) gemv_w2a8_kernel(const __grid_consta
                                  : make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
             for (int m = 0; m < MT; ++m) {
+                if (stage_x) s_x[int64_t(m) * pieces + c] = v[m];
                 const uint32_t a = max(max(v[m].x & 0x7FFFu, v[m].x >> 16 & 0x7FFFu),
                                        max(v[m].y & 0x7FFFu, v[m].y >> 16 & 0x7FFFu));
                 const uint32_t b = max(max(v[m].z & 0x7FFFu, v[m].z >> 16 & 0x7FFFu),
@@ -147,8 +160,10 @@ __global__ void __launch_bounds__(kThreads) gemv_w2a8_kernel(const __grid_consta
             uint4 v[MT];
 #pragma unroll
             for (int m = 0; m < MT; ++m)
-                v[m] = (valid && m < Mreal) ? reinterpret_cast<const uint4*>(p.x + int64_t(m) * K)[c]
-                                            : make_uint4(0u, 0u, 0u, 0u);
+                v[m] = (valid && m < Mreal)
+                           ? (stage_x ? s_x[int64_t(m) * pieces + c]
+                                      : reinterpret_cast<const uint4*>(p.x + int64_t(m) * K)[c])
+                           : make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
             for (int m = 0; m < MT; ++m) {
                 const float s = s_tok[m];
@@ -182,70 +197,103 @@ __global__ void __launch_bounds__(kThreads) gemv_w2a8_kernel(const __grid_consta
     }
     __syncthreads();
 
-    // ---- 3. dp4a over the register-resident chunks: sum_k q * code
-    int32_t acc[MT];
+    // ---- 3. dp4a over the register-resident chunks: sum_k q * code, two independent
+    //         accumulator chains per output
+    int32_t acc[RW][MT][2];
 #pragma unroll
-    for (int m = 0; m < MT; ++m) acc[m] = 0;
+    for (int r = 0; r < RW; ++r)
+#pragma unroll
+        for (int m = 0; m < MT; ++m) acc[r][m][0] = acc[r][m][1] = 0;
 #pragma unroll
     for (int c = 0; c < CPL; ++c) {
         const int chunk = lane + 32 * c;
         if (chunk < C) {
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
-                const uint32_t word = j == 0 ? w[c].x : j == 1 ? w[c].y : j == 2 ? w[c].z : w[c].w;
-                const int e0 = int(word & 0x03030303u);
-                const int e1 = int((word >> 2) & 0x03030303u);
-                const int e2 = int((word >> 4) & 0x03030303u);
-                const int e3 = int((word >> 6) & 0x03030303u);
+                int e[RW][4];
+#pragma unroll
+                for (int r = 0; r < RW; ++r) {
+                    const uint32_t word = j == 0 ? w[r][c].x : j == 1 ? w[r][c].y
+                                        : j == 2 ? w[r][c].z : w[r][c].w;
+                    e[r][0] = int(word & 0x03030303u);
+                    e[r][1] = int((word >> 2) & 0x03030303u);
+                    e[r][2] = int((word >> 4) & 0x03030303u);
+                    e[r][3] = int((word >> 6) & 0x03030303u);
+                }
 #pragma unroll
                 for (int m = 0; m < MT; ++m) {
                     const uint4 qv = s_q[(m * 4 + j) * C + chunk];
-                    int a = acc[m];
-                    a = __dp4a(e0, int(qv.x), a);
-                    a = __dp4a(e1, int(qv.y), a);
-                    a = __dp4a(e2, int(qv.z), a);
-                    a = __dp4a(e3, int(qv.w), a);
-                    acc[m] = a;
+#pragma unroll
+                    for (int r = 0; r < RW; ++r) {
+                        acc[r][m][0] = __dp4a(e[r][0], int(qv.x), acc[r][m][0]);
+                        acc[r][m][1] = __dp4a(e[r][1], int(qv.y), acc[r][m][1]);
+                        acc[r][m][0] = __dp4a(e[r][2], int(qv.z), acc[r][m][0]);
+                        acc[r][m][1] = __dp4a(e[r][3], int(qv.w), acc[r][m][1]);
+                    }
                 }
             }
         }
     }
 
     // ---- 4. reduce across the warp, remove the code offset (sum q), dequantise, write
+    int32_t qs_tot[MT];
 #pragma unroll
     for (int m = 0; m < MT; ++m) {
-        const int32_t total = __reduce_add_sync(0xFFFFFFFFu, acc[m]);
-        if (lane == m && rvalid && m < Mreal) {
-            int32_t qs = 0;
+        int32_t t = 0;
 #pragma unroll
-            for (int ww = 0; ww < kWarps; ++ww) qs += s_qsum[ww][m];
-            const GemvProj& pr = p.proj[pj];
-            const int32_t v = total - qs;
-            const int64_t o = int64_t(m) * pr.N + nrow;
-            if (p.out_kind == 2) {
-                reinterpret_cast<int32_t*>(pr.y)[o] = v;
-            } else {
-                const float rx = __frcp_rn(s_tok[m]);
-                const float yv = __fmul_rn(__int2float_rn(v), __fmul_rn(sw, rx));
-                if (p.out_kind == 0)
-                    reinterpret_cast<__nv_bfloat16*>(pr.y)[o] = __float2bfloat16_rn(yv);
-                else
-                    reinterpret_cast<float*>(pr.y)[o] = yv;
+        for (int ww = 0; ww < kWarps; ++ww) t += s_qsum[ww][m];
+        qs_tot[m] = t;
+    }
+#pragma unroll
+    for (int r = 0; r < RW; ++r) {
+#pragma unroll
+        for (int m = 0; m < MT; ++m) {
+            const int32_t total = __reduce_add_sync(0xFFFFFFFFu, acc[r][m][0] + acc[r][m][1]);
+            if (lane == r * MT + m && rvalid[r] && m < Mreal) {
+                const GemvProj& pr = p.proj[pj[r]];
+                const int32_t v = total - qs_tot[m];
+                const int64_t o = int64_t(m) * pr.N + nrow[r];
+                if (p.out_kind == 2) {
+                    reinterpret_cast<int32_t*>(pr.y)[o] = v;
+                } else {
+                    const float rx = __frcp_rn(s_tok[m]);
+                    const float yv = __fmul_rn(__int2float_rn(v), __fmul_rn(sw[r], rx));
+                    if (p.out_kind == 0)
+                        reinterpret_cast<__nv_bfloat16*>(pr.y)[o] = __float2bfloat16_rn(yv);
+                    else
+                        reinterpret_cast<float*>(pr.y)[o] = yv;
+                }
             }
         }
     }
 }
 
-template <int MT, int CPL>
+int num_sms() {
+    static int cached[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+    if (!cached[dev]) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+            n = 148;
+        cached[dev] = n;
+    }
+    return cached[dev];
+}
+
+template <int MT, int CPL, int RW>
 cudaError_t launch_one(const GemvParams& p, cudaStream_t stream, bool pdl) {
-    const size_t smem = size_t(MT) * size_t(p.K);
-    auto kern = gemv_w2a8_kernel<MT, CPL>;
+    // q (MT*K bytes) plus, when it fits, the staged bf16 activations (2*MT*K bytes)
+    GemvParams q = p;
+    q.stage_x = (p.q_in == nullptr && 3 * int64_t(MT) * p.K <= 96 * 1024) ? 1 : 0;
+    const size_t smem = size_t(MT) * size_t(p.K) * (q.stage_x ? 3 : 1);
+    auto kern = gemv_w2a8_kernel<MT, CPL, RW>;
     if (smem > 48 * 1024) {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              static_cast<int>(smem));
         if (e != cudaSuccess) return e;
     }
-    const int64_t rows_per_cta = kWarps;
+    const int64_t rows_per_cta = int64_t(kWarps) * RW;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>((p.total_rows + rows_per_cta - 1) / rows_per_cta));
     cfg.blockDim = dim3(kThreads);
@@ -256,18 +304,31 @@ cudaError_t launch_one(const GemvParams& p, cudaStream_t stream, bool pdl) {
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = pdl ? 1 : 0;
-    return cudaLaunchKernelEx(&cfg, kern, p);
+    return cudaLaunchKernelEx(&cfg, kern, q);
+}
+
+// Rows per warp: two for short rows when the grid would exceed one CTA per SM, which
+// keeps more of this grid and the next one (started early by programmatic dependent
+// launch) resident together; more rows per warp lengthen the work left after the wait
+// for the previous grid, which costs more than it saves (measured on B200).
+template <int MT, int CPL>
+cudaError_t launch_cpl(const GemvParams& p, cudaStream_t stream, bool pdl) {
+    const int64_t slots = int64_t(num_sms()) * kWarps;  // warps of one CTA per SM
+    if constexpr (CPL <= 2 && MT <= 2) {
+        if (p.total_rows > slots) return launch_one<MT, CPL, 2>(p, stream, pdl);
+    }
+    return launch_one<MT, CPL, 1>(p, stream, pdl);
 }
 
 template <int MT>
 cudaError_t launch_mt(const GemvParams& p, cudaStream_t stream, bool pdl) {
     const int64_t C = p.K >> 6;
     const int cpl = static_cast<int>((C + 31) / 32);
-    if (cpl <= 1) return launch_one<MT, 1>(p, stream, pdl);
-    if (cpl <= 2) return launch_one<MT, 2>(p, stream, pdl);
-    if (cpl <= 4) return launch_one<MT, 4>(p, stream, pdl);
-    if (cpl <= 8) return launch_one<MT, 8>(p, stream, pdl);
-    return launch_one<MT, 16>(p, stream, pdl);
+    if (cpl <= 1) return launch_cpl<MT, 1>(p, stream, pdl);
+    if (cpl <= 2) return launch_cpl<MT, 2>(p, stream, pdl);
+    if (cpl <= 4) return launch_cpl<MT, 4>(p, stream, pdl);
+    if (cpl <= 8) return launch_cpl<MT, 8>(p, stream, pdl);
+    return launch_cpl<MT, 16>(p, stream, pdl);
 }
 
 }  // namespace
