@@ -73,6 +73,8 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
     uint32_t spins = 0;
     while (true) {
         if (mbar_try_wait(bar, parity)) return true;
+        // Long waits back off, so waiting warps leave issue slots to co-resident work.
+        if (spins > 256u) __nanosleep(spins > 4096u ? 256u : 64u);
         if ((++spins & 63u) == 0u) {
             if (abort && *abort) return false;
             if (global_timer_ns() - t0 > kWaitLimitNs) {

@@ -65,6 +65,7 @@ __device__ __forceinline__ uint2 permute_group_half(uint2 nat, int h) {
 // re-reads the row (an L1/L2 hit) and writes q.
 constexpr int kRowsPerCta = kThreads / 32;
 constexpr int kUnroll = 8;
+constexpr int kRegPieces = 16;  // rows of up to 32 * 16 pieces (K <= 4096) stay in registers
 
 __global__ void __launch_bounds__(kThreads) quant_rows_kernel(const uint16_t* __restrict__ x,
                                                               const int8_t* __restrict__ q_in,
@@ -84,6 +85,34 @@ __global__ void __launch_bounds__(kThreads) quant_rows_kernel(const uint16_t* __
 
     float s = 0.0f;
     const uint4* xr = reinterpret_cast<const uint4*>(x + m * K);
+    int8_t* qr = q + m * K;
+    if (q_in == nullptr && pieces <= 32 * kRegPieces) {
+        // Short rows (K <= 4096): the whole row stays in registers; one read of x.
+        uint4 v[kRegPieces];
+#pragma unroll
+        for (int u = 0; u < kRegPieces; ++u) {
+            const int64_t c = u * 32 + lane;
+            v[u] = c < pieces ? xr[c] : make_uint4(0u, 0u, 0u, 0u);
+        }
+        uint32_t mx = 0;
+#pragma unroll
+        for (int u = 0; u < kRegPieces; ++u) mx = max(mx, absmax8_bits(v[u]));
+        mx = __reduce_max_sync(0xFFFFFFFFu, mx);
+        s = __fdiv_rn(127.0f, fmaxf(bf16_bits_to_float(mx), kEps));
+        if (lane == 0) {
+            if (s_x) s_x[m] = s;
+            if (r_x) r_x[m] = __frcp_rn(s);
+        }
+#pragma unroll
+        for (int u = 0; u < kRegPieces; ++u) {
+            if (u * 32 >= pieces) break;  // warp-uniform
+            const int64_t c = u * 32 + lane;
+            const uint2 nat = quant8(v[u], s);
+            const uint2 out = permuted ? permute_group_half(nat, lane & 1) : nat;
+            if (c < pieces) reinterpret_cast<uint2*>(qr)[c] = out;
+        }
+        return;
+    }
     if (q_in == nullptr) {
         uint32_t mx = 0;
         for (int64_t c0 = 0; c0 < pieces; c0 += 32 * kUnroll) {
@@ -104,7 +133,6 @@ __global__ void __launch_bounds__(kThreads) quant_rows_kernel(const uint16_t* __
         }
     }
 
-    int8_t* qr = q + m * K;
     for (int64_t c0 = 0; c0 < pieces; c0 += 32 * kUnroll) {
         uint2 nat[kUnroll];
         if (q_in == nullptr) {

@@ -1,4 +1,4 @@
-// Tensor-core W2A8 GEMM for sm_100a (tcgen05 + TMA + TMEM).
+// Tensor-core W2A8 GEMM for sm_100a (tcgen05 + TMA + TMEM), persistent.
 //
 // The contraction acc[m, n] = sum_k q[m, k] t[n, k] ("BitNet 深度实战", section 4.4
 // "查找表加速": int8 activations, ternary weights, int32 accumulation) runs as an int8
@@ -10,20 +10,27 @@
 // That keeps small token counts efficient and re-unpacks each weight tile once per
 // token tile of up to 256 tokens.
 //
-// Per CTA: one 128 x BN output tile (weight rows x tokens), K streamed in 128-byte stages.
-//  warp 0      TMEM allocation; lane 0 issues TMA loads of the packed weight tile
-//              (128 rows x 32 bytes) and the quantised token tile (BN rows x 128 bytes,
-//              128-byte swizzle) for each stage;
-//  warp 1      lane 0 issues 4 tcgen05.mma.kind::i8 (K = 32 each) per stage and commits
-//              them to the stage's "empty" barrier;
-//  warps 2-9   unpack each packed stage into the int8 A tile in shared memory (128-byte
-//              swizzled K-major, codes - 1 per byte), then run the epilogue: TMEM -> regs,
-//              y = acc * (s_w * 1/s_x), store.
-// The activation tile arrives already in the permuted in-group K order produced by the
-// quantiser, which is the order a packed word unpacks into with shifts and masks alone.
+// One CTA per SM walks a static list of 128 x BN output tiles. Three shared-memory rings
+// decouple the stages of the main loop, and two TMEM accumulators let the epilogue of one
+// tile overlap the main loop of the next:
+//  warp 0      TMEM allocation; lane 0 loads token tiles (BN rows x 128 bytes, 128-byte
+//              swizzle) into ring B with TMA;
+//  warp 1      lane 0 issues 4 tcgen05.mma.kind::i8 (K = 32 each) per 128-byte K stage and
+//              commits them to the A/B slots they read and, per tile, to the accumulator;
+//  warp 2      lane 0 loads packed weight tiles (128 rows x 32 bytes) into ring P with TMA;
+//  warps 3-10  epilogue, two warps per TMEM lane quarter splitting the columns: TMEM ->
+//              registers -> y = acc * (s_w * 1/s_x) -> staged rows -> coalesced 16-byte
+//              stores; then the accumulator goes back to the MMA warp;
+//  warps 11-18 unpack ring P into ring A: codes - 1 per byte, written as the 128-byte
+//              swizzled K-major operand tile.
+// The token tile arrives in the permuted in-group K order produced by the quantiser, which
+// is the order a packed word unpacks into with shifts and masks alone.
 //
+// Under programmatic dependent launch the weight producer and the unpack warps start
+// before the quantiser grid has finished; only the token producer and the epilogue wait.
 // Every mbarrier wait is bounded (bitnet_device.cuh): on expiry the kernel records a
-// watchdog code and runs on to its end, so it always returns and frees its TMEM.
+// watchdog code, the other waits return at once, and the CTA drains its copies and MMAs
+// and frees its TMEM before it exits.
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
 
@@ -33,31 +40,40 @@
 namespace bitnet {
 namespace {
 
-constexpr int kBM = 128;          // weight rows per tile (MMA M)
-constexpr int kBK = 128;          // K bytes per stage
-constexpr int kUnpackWarps = 8;
-constexpr int kThreads = 64 + kUnpackWarps * 32;  // 320
+constexpr int kBM = 128;  // weight rows per tile (MMA M)
+constexpr int kBK = 128;  // K bytes per stage
+constexpr int kWarpB = 0, kWarpMma = 1, kWarpP = 2, kEpiWarp0 = 3, kEpiWarps = 8,
+              kUnpWarp0 = 11, kUnpWarps = 8;
+constexpr int kThreads = (kUnpWarp0 + kUnpWarps) * 32;  // 608
+constexpr int kEpiThreads = kEpiWarps * 32;
+constexpr int kHalfCols = 16;                           // columns per epilogue warp per round
+constexpr int kStagingBytes = 2 * kHalfCols * kBM * 4;  // one staging buffer (fp32 / int32)
 
 template <int BN>
 struct TcLayout {
-    static constexpr int kA = kBM * kBK;        // unpacked weights, 16 KB
-    static constexpr int kB = BN * kBK;         // token tile
-    static constexpr int kP = kBM * kBK / 4;    // packed weights, 4 KB
-    static constexpr int kStage = kA + kB + kP;  // multiple of 1024
-    static constexpr int kStages = (200 * 1024) / kStage > 6 ? 6 : (200 * 1024) / kStage;
-    static constexpr int kBarOff = kStages * kStage;
-    static constexpr int kBarBytes = (3 * kStages + 1) * 8 + 16;  // + TMEM slot, abort flag
-    static constexpr int kRxOff = kBarOff + kBarBytes;             // BN floats: 1/s_x of the tile
-    static constexpr int kSmem = kRxOff + BN * 4 + 1024;           // + alignment slack
-    static_assert(BN * kBM * 4 <= kStages * kStage, "output staging must fit the stage area");
-    static constexpr uint32_t kTmemCols = BN < 32 ? 32 : BN;
-    static_assert(kStage % 1024 == 0, "stage must keep 1024-byte alignment");
-    static_assert(kStages >= 2, "need at least two stages");
+    static constexpr int kA = kBM * kBK;      // unpacked weights, 16 KB
+    static constexpr int kB = BN * kBK;       // token tile
+    static constexpr int kP = kBM * kBK / 4;  // packed weights, 4 KB
+    // Ring depths: the token ring is as deep as shared memory allows, since its TMA round
+    // trip (about 1 - 1.5 us measured on B200) sets the main-loop cadence.
+    static constexpr int kDA = BN >= 256 ? 3 : 4;
+    static constexpr int kDB = BN >= 256 ? 4 : BN >= 128 ? 6 : 8;
+    static constexpr int kDP = BN >= 256 ? 4 : 8;
+    static constexpr int kOffA = 0;
+    static constexpr int kOffB = kOffA + kDA * kA;
+    static constexpr int kOffP = kOffB + kDB * kB;
+    static constexpr int kOffStage = kOffP + kDP * kP;
+    static constexpr int kOffBar = kOffStage + 2 * kStagingBytes;
+    static constexpr int kNumBars = 2 * (kDA + kDB + kDP) + 4;
+    static constexpr int kSmem = kOffBar + kNumBars * 8 + 16 + 1024;  // + slot, flag, align
+    static constexpr uint32_t kAccCols = BN;  // columns per accumulator buffer
+    static constexpr uint32_t kTmemCols = 2 * BN < 32 ? 32 : 2 * BN;
+    static_assert(kA % 1024 == 0 && kB % 1024 == 0, "swizzled tiles need 1024-byte alignment");
+    static_assert(kSmem <= 232448, "shared memory budget");
 };
 
-// Barrier among the 8 unpack/epilogue warps only (named barrier 1).
 __device__ __forceinline__ void epilogue_bar_sync() {
-    asm volatile("bar.sync 1, %0;" ::"n"(kUnpackWarps * 32) : "memory");
+    asm volatile("bar.sync 1, %0;" ::"n"(kEpiThreads) : "memory");
 }
 
 template <int N>
@@ -65,9 +81,36 @@ __device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, uint32_t (&v)[N]) {
     static_assert(N % 8 == 0, "columns in multiples of 8");
 #pragma unroll
     for (int i = 0; i < N / 8; ++i) {
-        uint32_t (&r)[8] = *reinterpret_cast<uint32_t(*)[8]>(&v[8 * i]);
+        uint32_t(&r)[8] = *reinterpret_cast<uint32_t(*)[8]>(&v[8 * i]);
         tmem_ld_32x32b_x8(taddr + uint32_t(8 * i), r);
     }
+}
+
+struct TileCoord {
+    int proj;
+    int n0;   // first weight row of the tile within its projection
+    int m0;   // first token of the tile
+    int kt0;  // first K stage of the tile's main loop
+};
+
+__device__ __forceinline__ int num_k_of(const TcParams& p) {
+    return static_cast<int>((p.K + kBK - 1) / kBK);
+}
+
+__device__ __forceinline__ TileCoord tile_coord(const TcParams& p, int t, int bn) {
+    const int nt = t % p.n_tiles_total;
+    TileCoord c;
+    c.proj = 0;
+#pragma unroll
+    for (int jj = 1; jj < kMaxProj; ++jj)
+        if (jj < p.nproj && nt >= p.proj[jj].tile_begin) c.proj = jj;
+    c.n0 = (nt - p.proj[c.proj].tile_begin) * kBM;
+    c.m0 = (t / p.n_tiles_total) * bn;
+    // Tiles that share a token tile run at the same time on different SMs; starting their K
+    // loops at different stages spreads their reads of that tile over L2. The int32 sum is
+    // exact, so the order of the K stages does not change the result.
+    c.kt0 = static_cast<int>((int64_t(nt) * 7) % num_k_of(p));
+    return c;
 }
 
 template <int BN>
@@ -76,36 +119,44 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~uintptr_t(1023));
-    uint64_t* full_tma = reinterpret_cast<uint64_t*>(smem + L::kBarOff);
-    uint64_t* full_unp = full_tma + L::kStages;
-    uint64_t* empty = full_unp + L::kStages;
-    uint64_t* acc_full = empty + L::kStages;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_full + 1);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kOffBar);
+    uint64_t* p_full = bars;
+    uint64_t* p_empty = p_full + L::kDP;
+    uint64_t* a_full = p_empty + L::kDP;
+    uint64_t* a_empty = a_full + L::kDA;
+    uint64_t* b_full = a_empty + L::kDA;
+    uint64_t* b_empty = b_full + L::kDB;
+    uint64_t* acc_full = b_empty + L::kDB;  // [2]
+    uint64_t* acc_empty = acc_full + 2;     // [2]
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
     volatile int32_t* abort_flag = reinterpret_cast<volatile int32_t*>(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-
-    // tile -> (projection, weight-row block, token block)
-    int j = 0;
-#pragma unroll
-    for (int jj = 1; jj < kMaxProj; ++jj)
-        if (jj < p.nproj && int(blockIdx.x) >= p.proj[jj].tile_begin) j = jj;
-    const int n0 = (int(blockIdx.x) - p.proj[j].tile_begin) * kBM;
-    const int m0 = int(blockIdx.y) * BN;
     const int num_k = static_cast<int>((p.K + kBK - 1) / kBK);
+    const int m_tiles = (p.M + BN - 1) / BN;
+    const int num_tiles = m_tiles * p.n_tiles_total;
 
-    if (warp == 0) {
+    if (warp == kWarpB) {
         if (lane == 0) {
-            for (int s = 0; s < L::kStages; ++s) {
-                mbar_init(&full_tma[s], 1);
-                mbar_init(&full_unp[s], kUnpackWarps);
-                mbar_init(&empty[s], 1);
+            for (int s = 0; s < L::kDP; ++s) {
+                mbar_init(&p_full[s], 1);
+                mbar_init(&p_empty[s], kUnpWarps);
             }
-            mbar_init(acc_full, 1);
+            for (int s = 0; s < L::kDA; ++s) {
+                mbar_init(&a_full[s], kUnpWarps);
+                mbar_init(&a_empty[s], 1);
+            }
+            for (int s = 0; s < L::kDB; ++s) {
+                mbar_init(&b_full[s], 1);
+                mbar_init(&b_empty[s], 1);
+            }
+            for (int b = 0; b < 2; ++b) {
+                mbar_init(&acc_full[b], 1);
+                mbar_init(&acc_empty[b], kEpiWarps);
+            }
             *abort_flag = 0;
             fence_mbar_init();
-            tma_prefetch_desc(&p.tmap_w[j]);
             tma_prefetch_desc(&p.tmap_q);
         }
         __syncwarp();
@@ -115,170 +166,248 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    const uint32_t tmem_d = *tmem_slot;
+    const uint32_t tmem_base = *tmem_slot;
+    pdl_trigger();
 
-    if (warp == 0) {
+    if (warp == kWarpB) {
         if (lane == 0) {
-            // ---------------- TMA producer
-            pdl_wait();  // the token tile is written by the quantiser grid
-            for (int kt = 0; kt < num_k; ++kt) {
-                const int s = kt % L::kStages;
-                const uint32_t ph = (kt / L::kStages) & 1;
-                mbar_wait_bounded(&empty[s], ph ^ 1, p.err, kErrWaitEmpty, abort_flag);
-                uint8_t* st = smem + s * L::kStage;
-                mbar_arrive_expect_tx(&full_tma[s], L::kB + L::kP);
-                tma_load_2d(st + L::kA + L::kB, &p.tmap_w[j], &full_tma[s], kt * (kBK / 4), n0);
-                tma_load_2d(st + L::kA, &p.tmap_q, &full_tma[s], kt * kBK, m0);
+            // ---------------- token tiles (written by the quantiser grid)
+            pdl_wait();
+            int kc = 0;
+            for (int t = blockIdx.x; t < num_tiles; t += gridDim.x) {
+                const TileCoord tc = tile_coord(p, t, BN);
+                for (int kt = 0; kt < num_k; ++kt, ++kc) {
+                    const int s = kc % L::kDB;
+                    const uint32_t ph = (kc / L::kDB) & 1;
+                    mbar_wait_bounded(&b_empty[s], ph ^ 1, p.err, kErrWaitEmpty, abort_flag);
+                    mbar_arrive_expect_tx(&b_full[s], L::kB);
+                    const int kr = (tc.kt0 + kt) % num_k;
+                    tma_load_2d(smem + L::kOffB + s * L::kB, &p.tmap_q, &b_full[s], kr * kBK, tc.m0);
+                }
             }
-            // Drain: every issued stage must have landed before the CTA may exit.
-            for (int kt = num_k > L::kStages ? num_k - L::kStages : 0; kt < num_k; ++kt) {
-                mbar_wait_bounded(&full_tma[kt % L::kStages], (kt / L::kStages) & 1, p.err,
-                                  kErrWaitDrain, nullptr);
-            }
+            for (int k = kc > L::kDB ? kc - L::kDB : 0; k < kc; ++k)  // drain
+                mbar_wait_bounded(&b_full[k % L::kDB], (k / L::kDB) & 1, p.err, kErrWaitDrain, nullptr);
         }
-        __syncwarp();  // lanes 1-31 wait for the producer lane: the CTA barrier below is aligned
-    } else if (warp == 1) {
+        __syncwarp();
+    } else if (warp == kWarpP) {
+        if (lane == 0) {
+            // ---------------- packed weight tiles (independent of earlier grids)
+            for (int j = 0; j < p.nproj; ++j) tma_prefetch_desc(&p.tmap_w[j]);
+            int kc = 0;
+            for (int t = blockIdx.x; t < num_tiles; t += gridDim.x) {
+                const TileCoord tc = tile_coord(p, t, BN);
+                for (int kt = 0; kt < num_k; ++kt, ++kc) {
+                    const int s = kc % L::kDP;
+                    const uint32_t ph = (kc / L::kDP) & 1;
+                    mbar_wait_bounded(&p_empty[s], ph ^ 1, p.err, kErrWaitEmpty, abort_flag);
+                    mbar_arrive_expect_tx(&p_full[s], L::kP);
+                    const int kr = (tc.kt0 + kt) % num_k;
+                    tma_load_2d(smem + L::kOffP + s * L::kP, &p.tmap_w[tc.proj], &p_full[s],
+                                kr * (kBK / 4), tc.n0);
+                }
+            }
+            for (int k = kc > L::kDP ? kc - L::kDP : 0; k < kc; ++k)  // drain
+                mbar_wait_bounded(&p_full[k % L::kDP], (k / L::kDP) & 1, p.err, kErrWaitDrain, nullptr);
+        }
+        __syncwarp();
+    } else if (warp == kWarpMma) {
         if (lane == 0) {
             // ---------------- MMA issuer
             constexpr uint32_t idesc = idesc_i8(kBM, BN);
-            for (int kt = 0; kt < num_k; ++kt) {
-                const int s = kt % L::kStages;
-                const uint32_t ph = (kt / L::kStages) & 1;
-                mbar_wait_bounded(&full_tma[s], ph, p.err, kErrWaitTmaFull, abort_flag);
-                mbar_wait_bounded(&full_unp[s], ph, p.err, kErrWaitUnpack, abort_flag);
+            int kc = 0, i = 0;
+            for (int t = blockIdx.x; t < num_tiles; t += gridDim.x, ++i) {
+                const int buf = i & 1;
+                mbar_wait_bounded(&acc_empty[buf], ((i >> 1) & 1) ^ 1, p.err, kErrWaitAccum,
+                                  abort_flag);
                 tc_fence_after();
-                const uint32_t a_base = smem_addr(smem + s * L::kStage);
-                const uint32_t b_base = a_base + L::kA;
+                const uint32_t d = tmem_base + uint32_t(buf) * L::kAccCols;
+                for (int kt = 0; kt < num_k; ++kt, ++kc) {
+                    const int sa = kc % L::kDA, sb = kc % L::kDB;
+                    mbar_wait_bounded(&a_full[sa], (kc / L::kDA) & 1, p.err, kErrWaitUnpack, abort_flag);
+                    mbar_wait_bounded(&b_full[sb], (kc / L::kDB) & 1, p.err, kErrWaitTmaFull, abort_flag);
+                    tc_fence_after();
+                    const uint32_t a_base = smem_addr(smem + L::kOffA + sa * L::kA);
+                    const uint32_t b_base = smem_addr(smem + L::kOffB + sb * L::kB);
 #pragma unroll
-                for (int kk = 0; kk < kBK / 32; ++kk) {
-                    const uint64_t ad = smem_desc_k_sw128(a_base + kk * 32);
-                    const uint64_t bd = smem_desc_k_sw128(b_base + kk * 32);
-                    mma_i8(tmem_d, ad, bd, idesc, (kt | kk) != 0 ? 1u : 0u);
+                    for (int kk = 0; kk < kBK / 32; ++kk)
+                        mma_i8(d, smem_desc_k_sw128(a_base + kk * 32),
+                               smem_desc_k_sw128(b_base + kk * 32), idesc, (kt | kk) != 0 ? 1u : 0u);
+                    mma_commit(&a_empty[sa]);
+                    mma_commit(&b_empty[sb]);
                 }
-                mma_commit(&empty[s]);
+                mma_commit(&acc_full[buf]);
             }
-            mma_commit(acc_full);
-            // Drain: no tensor-core operation may still be running when TMEM is freed.
-            mbar_wait_bounded(acc_full, 0, p.err, kErrWaitDrain, nullptr);
+            if (i > 0)  // drain: no tensor-core operation may run when TMEM is freed
+                mbar_wait_bounded(&acc_full[(i - 1) & 1], ((i - 1) >> 1) & 1, p.err, kErrWaitDrain,
+                                  nullptr);
         }
-        __syncwarp();  // reconverge before the aligned CTA barrier below
+        __syncwarp();
+    } else if (warp >= kUnpWarp0) {
+        // ---------------- unpack: ring P -> ring A
+        const int ut = threadIdx.x - kUnpWarp0 * 32;  // 0 .. 255
+        const int row = ut >> 1;                      // weight row of the tile
+        const int half = ut & 1;                      // which 16 packed bytes (64 weights)
+        int kc = 0;
+        for (int t = blockIdx.x; t < num_tiles; t += gridDim.x) {
+            for (int kt = 0; kt < num_k; ++kt, ++kc) {
+                const int sp = kc % L::kDP, sa = kc % L::kDA;
+                mbar_wait_bounded(&p_full[sp], (kc / L::kDP) & 1, p.err, kErrWaitTmaFull, abort_flag);
+                const uint4 pk = *reinterpret_cast<const uint4*>(smem + L::kOffP + sp * L::kP +
+                                                                 row * 32 + half * 16);
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&p_empty[sp]);
+                mbar_wait_bounded(&a_empty[sa], ((kc / L::kDA) & 1) ^ 1, p.err, kErrWaitEmpty,
+                                  abort_flag);
+                uint8_t* arow = smem + L::kOffA + sa * L::kA + row * kBK;
+                const uint32_t words[4] = {pk.x, pk.y, pk.z, pk.w};
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    const uint32_t wv = words[c];
+                    uint4 tv;
+                    tv.x = codes_to_ternary_s8x4(wv & 0x03030303u);
+                    tv.y = codes_to_ternary_s8x4((wv >> 2) & 0x03030303u);
+                    tv.z = codes_to_ternary_s8x4((wv >> 4) & 0x03030303u);
+                    tv.w = codes_to_ternary_s8x4((wv >> 6) & 0x03030303u);
+                    const int chunk = half * 4 + c;  // 16-byte chunk of the 128-byte row
+                    *reinterpret_cast<uint4*>(arow + ((chunk ^ (row & 7)) << 4)) = tv;
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&a_full[sa]);
+            }
+        }
     } else {
-        // ---------------- unpack warps
-        const int ut = threadIdx.x - 64;  // 0 .. 255
-        const int row = ut >> 1;         // weight row of the tile
-        const int half = ut & 1;         // which 16 packed bytes (64 weights) of the stage
-        for (int kt = 0; kt < num_k; ++kt) {
-            const int s = kt % L::kStages;
-            const uint32_t ph = (kt / L::kStages) & 1;
-            mbar_wait_bounded(&full_tma[s], ph, p.err, kErrWaitTmaFull, abort_flag);
-            uint8_t* st = smem + s * L::kStage;
-            const uint4 pk = *reinterpret_cast<const uint4*>(st + L::kA + L::kB + row * 32 +
-                                                             half * 16);
-            const uint32_t words[4] = {pk.x, pk.y, pk.z, pk.w};
-            uint8_t* arow = st + row * kBK;
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                const uint32_t wv = words[c];
-                uint4 t;
-                t.x = codes_to_ternary_s8x4(wv & 0x03030303u);
-                t.y = codes_to_ternary_s8x4((wv >> 2) & 0x03030303u);
-                t.z = codes_to_ternary_s8x4((wv >> 4) & 0x03030303u);
-                t.w = codes_to_ternary_s8x4((wv >> 6) & 0x03030303u);
-                const int chunk = half * 4 + c;  // 16-byte chunk of the 128-byte row
-                *reinterpret_cast<uint4*>(arow + ((chunk ^ (row & 7)) << 4)) = t;
-            }
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&full_unp[s]);
-        }
-
-        // ---------------- epilogue
-        // 1/s_x of the tile's tokens -> shared memory while the last MMAs run.
+        // ---------------- epilogue (warps 3-10: TMEM lane quarter warp % 4, column half)
         pdl_wait();  // r_x comes from the quantiser grid; y may be read by earlier grids
-        const int et = threadIdx.x - 64;  // 0 .. 255
-        float* s_rx = reinterpret_cast<float*>(smem + L::kRxOff);
-        for (int i = et; i < BN; i += kUnpackWarps * 32) {
-            const int64_t m = int64_t(m0) + i;
-            s_rx[i] = (p.out_kind != 2 && m < p.M) ? p.r_x[m] : 0.0f;
-        }
-        epilogue_bar_sync();
-        mbar_wait_bounded(acc_full, 0, p.err, kErrWaitAccum, abort_flag);
-        tc_fence_after();
-
-        // TMEM (lane = weight row, column = token) -> registers -> dequantised values staged in
-        // the idle stage area as rows of the output: stage[token][weight row].
-        const int quarter = warp & 3;         // TMEM lanes 32*quarter ... +31
-        const int colhalf = (warp - 2) >> 2;  // which half of the BN columns
+        const int quarter = warp & 3;
+        const int colhalf = (warp - kEpiWarp0) >> 2;
         const int n_local = quarter * 32 + lane;
-        const TcProj& pr = p.proj[j];
-        const int64_t n = int64_t(n0) + n_local;
-        const bool nvalid = n < pr.N;
-        // s_w is absent (nullptr) when the raw int32 accumulator is the output.
-        const float sw = p.out_kind == 2 ? 0.0f
-                         : pr.per_row   ? (nvalid ? pr.s_w[n] : 0.0f)
-                                        : pr.s_w[0];
+        const int et = threadIdx.x - kEpiWarp0 * 32;  // 0 .. 255
         const int esz = p.out_kind == 0 ? 2 : 4;
-        uint8_t* stage = smem;
-        constexpr int kHalfCols = BN / 2;
-        constexpr int kLd = kHalfCols >= 32 ? 32 : kHalfCols;  // columns per TMEM load
-#pragma unroll 1
-        for (int cc = 0; cc < kHalfCols; cc += kLd) {
-            const int col0 = colhalf * kHalfCols + cc;
-            uint32_t v[kLd];
-            tmem_ld_cols<kLd>(tmem_d + (uint32_t(quarter * 32) << 16) + uint32_t(col0), v);
-            tmem_ld_wait();
+        constexpr int kHC = BN / 2 < kHalfCols ? BN / 2 : kHalfCols;  // columns per warp per round
+        constexpr int kRounds = BN / (2 * kHC);
+        // Staging buffers alternate on a round counter that runs across tiles, so a buffer is
+        // rewritten only after the barrier that follows every thread's copy-out of it.
+        int round_run = 0;
+        int i = 0;
+        for (int t = blockIdx.x; t < num_tiles; t += gridDim.x, ++i) {
+            const TileCoord tc = tile_coord(p, t, BN);
+            const TcProj& pr = p.proj[tc.proj];
+            const int64_t n = int64_t(tc.n0) + n_local;
+            const bool nvalid = n < pr.N;
+            // s_w is absent (nullptr) when the raw int32 accumulator is the output.
+            const float sw = p.out_kind == 2 ? 0.0f
+                             : pr.per_row   ? (nvalid ? pr.s_w[n] : 0.0f)
+                                            : pr.s_w[0];
+            const int buf = i & 1;
+            // 1/s_x of this warp's columns, fetched before the accumulator is ready: lane l
+            // holds token (round r, column l % kHC) for r = l / kHC (+ rounds of 32 / kHC).
+            constexpr int kPre = (kRounds * kHC + 31) / 32;
+            float rx_pre[kPre];
 #pragma unroll
-            for (int i = 0; i < kLd; ++i) {
-                const int col = col0 + i;
-                const int32_t a = static_cast<int32_t>(v[i]);
-                uint8_t* dst = stage + (size_t(col) * kBM + n_local) * esz;
+            for (int u = 0; u < kPre; ++u) {
+                const int slot = u * 32 + lane;  // = round * kHC + column
+                const int rr = slot / kHC, cc = slot % kHC;
+                const int64_t m = int64_t(tc.m0) + rr * 2 * kHC + colhalf * kHC + cc;
+                rx_pre[u] = (p.out_kind != 2 && rr < kRounds && m < p.M) ? p.r_x[m] : 0.0f;
+            }
+            mbar_wait_bounded(&acc_full[buf], (i >> 1) & 1, p.err, kErrWaitAccum, abort_flag);
+            tc_fence_after();
+            const uint32_t d = tmem_base + uint32_t(buf) * L::kAccCols + (uint32_t(quarter * 32) << 16);
+            const bool vec_ok = ((pr.N * esz) % 16) == 0;  // every output row 16-byte aligned
+            uint8_t* ybase = static_cast<uint8_t*>(pr.y);
+#pragma unroll 1
+            for (int r = 0; r < kRounds; ++r, ++round_run) {
+                uint8_t* stage = smem + L::kOffStage + (round_run & 1) * kStagingBytes;
+                const int col0 = r * 2 * kHC + colhalf * kHC;  // this warp's first column
+                uint32_t v[kHC];
+                tmem_ld_cols<kHC>(d + uint32_t(col0), v);
+                float rx[kHC];
+#pragma unroll
+                for (int c = 0; c < kHC; ++c) {
+                    const int slot = r * kHC + c;
+                    float mine = 0.0f;
+#pragma unroll
+                    for (int u = 0; u < kPre; ++u)
+                        if (u == slot / 32) mine = rx_pre[u];
+                    rx[c] = __shfl_sync(0xFFFFFFFFu, mine, slot % 32);
+                }
+                tmem_ld_wait();
+                // staged row index = column within the round (0 .. 2*kHC-1)
+                const int srow0 = colhalf * kHC;
                 if (p.out_kind == 2) {
-                    *reinterpret_cast<int32_t*>(dst) = a;
+#pragma unroll
+                    for (int c = 0; c < kHC; ++c)
+                        reinterpret_cast<int32_t*>(stage)[(srow0 + c) * kBM + n_local] = int32_t(v[c]);
+                } else if (p.out_kind == 0) {
+                    __nv_bfloat16 yb[kHC];
+#pragma unroll
+                    for (int c = 0; c < kHC; ++c)
+                        yb[c] = __float2bfloat16_rn(
+                            __fmul_rn(__int2float_rn(int32_t(v[c])), __fmul_rn(sw, rx[c])));
+#pragma unroll
+                    for (int c = 0; c < kHC; ++c)
+                        reinterpret_cast<__nv_bfloat16*>(stage)[(srow0 + c) * kBM + n_local] = yb[c];
                 } else {
-                    const float yv = __fmul_rn(__int2float_rn(a), __fmul_rn(sw, s_rx[col]));
-                    if (p.out_kind == 0)
-                        *reinterpret_cast<__nv_bfloat16*>(dst) = __float2bfloat16_rn(yv);
-                    else
-                        *reinterpret_cast<float*>(dst) = yv;
+                    float yf[kHC];
+#pragma unroll
+                    for (int c = 0; c < kHC; ++c)
+                        yf[c] = __fmul_rn(__int2float_rn(int32_t(v[c])), __fmul_rn(sw, rx[c]));
+#pragma unroll
+                    for (int c = 0; c < kHC; ++c)
+                        reinterpret_cast<float*>(stage)[(srow0 + c) * kBM + n_local] = yf[c];
+                }
+                epilogue_bar_sync();
+                // coalesced copy-out: 2*kHC token rows of 128 contiguous outputs
+                const int row_bytes = kBM * esz;
+                const int chunks_per_row = row_bytes / 16;
+                const int vals_per_chunk = 16 / esz;
+                for (int q = et; q < 2 * kHC * chunks_per_row; q += kEpiThreads) {
+                    const int rrow = q / chunks_per_row;
+                    const int ch = q - rrow * chunks_per_row;
+                    const int64_t m = int64_t(tc.m0) + r * 2 * kHC + rrow;
+                    if (m >= p.M) continue;
+                    const int64_t nn = int64_t(tc.n0) + int64_t(ch) * vals_per_chunk;
+                    const uint8_t* src = stage + size_t(rrow) * row_bytes + size_t(ch) * 16;
+                    uint8_t* dst = ybase + (m * pr.N + nn) * esz;
+                    if (vec_ok && nn + vals_per_chunk <= pr.N) {
+                        *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(src);
+                    } else {
+                        for (int e = 0; e < vals_per_chunk && nn + e < pr.N; ++e) {
+                            if (esz == 2)
+                                reinterpret_cast<uint16_t*>(dst)[e] = reinterpret_cast<const uint16_t*>(src)[e];
+                            else
+                                reinterpret_cast<uint32_t*>(dst)[e] = reinterpret_cast<const uint32_t*>(src)[e];
+                        }
+                    }
                 }
             }
-        }
-        epilogue_bar_sync();
-
-        // Coalesced copy-out: each token row of the tile is 128 contiguous outputs.
-        const int row_bytes = kBM * esz;
-        const int chunks_per_row = row_bytes / 16;
-        const int vals_per_chunk = 16 / esz;
-        const bool vec_ok = ((pr.N * esz) % 16) == 0;  // every row start 16-byte aligned
-        uint8_t* ybase = static_cast<uint8_t*>(pr.y);
-        for (int c = et; c < BN * chunks_per_row; c += kUnpackWarps * 32) {
-            const int row = c / chunks_per_row;
-            const int ch = c - row * chunks_per_row;
-            const int64_t m = int64_t(m0) + row;
-            if (m >= p.M) continue;
-            const int64_t nn = int64_t(n0) + int64_t(ch) * vals_per_chunk;
-            const uint8_t* src = stage + size_t(row) * row_bytes + size_t(ch) * 16;
-            uint8_t* dst = ybase + (m * pr.N + nn) * esz;
-            if (vec_ok && nn + vals_per_chunk <= pr.N) {
-                *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(src);
-            } else {
-                for (int e = 0; e < vals_per_chunk; ++e) {
-                    if (nn + e >= pr.N) break;
-                    if (esz == 2)
-                        reinterpret_cast<uint16_t*>(dst)[e] = reinterpret_cast<const uint16_t*>(src)[e];
-                    else
-                        reinterpret_cast<uint32_t*>(dst)[e] = reinterpret_cast<const uint32_t*>(src)[e];
-                }
-            }
+            // accumulator read out: hand it back to the MMA warp
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&acc_empty[buf]);
         }
     }
 
     tc_fence_before();
     __syncthreads();
-    if (warp == 0) {
+    if (warp == kWarpB) {
         __syncwarp();
-        tmem_dealloc(tmem_d, L::kTmemCols);
+        tmem_dealloc(tmem_base, L::kTmemCols);
     }
+}
+
+int num_sms_cached() {
+    static int cached[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+    if (!cached[dev]) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+            n = 148;
+        cached[dev] = n;
+    }
+    return cached[dev];
 }
 
 template <int BN>
@@ -287,9 +416,10 @@ cudaError_t launch_bn(const TcParams& p, cudaStream_t stream, bool pdl) {
     auto kern = tc_gemm_kernel<BN>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kSmem);
     if (e != cudaSuccess) return e;
+    const int tiles = ((p.M + BN - 1) / BN) * p.n_tiles_total;
+    const int grid = tiles < num_sms_cached() ? tiles : num_sms_cached();
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(static_cast<unsigned>(p.n_tiles_total),
-                       static_cast<unsigned>((p.M + BN - 1) / BN));
+    cfg.gridDim = dim3(static_cast<unsigned>(grid));
     cfg.blockDim = dim3(kThreads);
     cfg.dynamicSmemBytes = L::kSmem;
     cfg.stream = stream;
