@@ -144,15 +144,15 @@ def build_decode(bn, torch, replicas: int, dev):
     return calls
 
 
-def build_prefill(bn, torch, dev):
+def build_prefill(bn, torch, dev, M):
     calls = []
     for si in range(len(synth.SWEEP_SHAPES)):
-        c = synth.prefill_case(si, PREFILL_M)
+        c = synth.prefill_case(si, M)
         packed = bn.bitnet_pack_ternary(torch.from_numpy(c["t"]).to(dev))
         s_w = torch.from_numpy(c["s_w"]).to(dev)
         x = torch.from_numpy(c["x"].view(np.int16).copy()).to(dev).view(torch.bfloat16)
-        y = torch.empty((PREFILL_M, c["N"]), dtype=torch.bfloat16, device=dev)
-        ws = bn.make_workspace(PREFILL_M, c["K"], dev)
+        y = torch.empty((M, c["N"]), dtype=torch.bfloat16, device=dev)
+        ws = bn.make_workspace(M, c["K"], dev)
         calls.append({"x": x, "packed": packed, "s_w": s_w, "y": y, "N": c["N"], "K": c["K"],
                       "ws": ws})
     return calls
@@ -327,20 +327,20 @@ def run_ours(args):
     if args.only == "decode":
         pcalls = []
     else:
-        pcalls = build_prefill(bn, torch, dev)
+        pcalls = build_prefill(bn, torch, dev, args.prefill_m)
     gemm = None
     g_pre = None
     if pcalls:
         g_pre = capture(torch, lambda: run_calls(bn, pcalls))
         pre_ms = timed_steps(torch, g_pre.replay, args.steps, args.warmup, flush, world)
         assert bn.bitnet_check_device_errors() == 0
-        ops_step = sum(2.0 * PREFILL_M * c["N"] * c["K"] for c in pcalls)
+        ops_step = sum(2.0 * args.prefill_m * c["N"] * c["K"] for c in pcalls)
         pre_ms_max, pre_ops = reduce_over_ranks(pre_ms, ops_step * args.steps, world)
         tops = pre_ops / (pre_ms_max * 1e-3) / 1e12
         int8_peak = peaks["bf16_tflops"] * INT8_PER_BF16
         local_tops = ops_step * args.steps / (pre_ms * 1e-3) / 1e12
         gemm = {"value": tops, "unit": "TOPS", "ms_per_step": pre_ms_max / args.steps,
-                "workload": f"prefill GEMM M={PREFILL_M} on the same 4 shapes, x = 0.5 t_4 "
+                "workload": f"prefill GEMM M={args.prefill_m} on the same 4 shapes, x = 0.5 t_4 "
                             "with 1% x20 outlier channels, ternary P(0)=0.5",
                 "roofline": {"bound": "tensor", "achieved": local_tops, "peak": int8_peak,
                              "unit": "TOPS", "frac": local_tops / int8_peak, "traffic": None,
@@ -399,6 +399,8 @@ def main():
                     help="decode: skip the prefill GEMM part (small profiling runs)")
     ap.add_argument("--replicas", type=int, default=0,
                     help="weight replicas per decode step (0: enough to exceed 2x L2)")
+    ap.add_argument("--prefill-m", type=int, default=PREFILL_M,
+                    help="tokens of the prefill GEMM part")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)  # at least 3 untimed warm-up steps
     if args.impl == "reference":

@@ -19,8 +19,9 @@
 //              commits them to the A/B slots they read and, per tile, to the accumulator;
 //  warp 2      lane 0 loads packed weight tiles (128 rows x 32 bytes) into ring P with TMA;
 //  warps 3-10  epilogue, two warps per TMEM lane quarter splitting the columns: TMEM ->
-//              registers -> y = acc * (s_w * 1/s_x) -> staged rows -> coalesced 16-byte
-//              stores; then the accumulator goes back to the MMA warp;
+//              registers -> y = acc * (s_w * 1/s_x) -> stores (a warp writes 32 adjacent
+//              outputs of one token per store); then the accumulator goes back to the MMA
+//              warp;
 //  warps 11-18 unpack ring P into ring A: codes - 1 per byte, written as the 128-byte
 //              swizzled K-major operand tile.
 // The token tile arrives in the permuted in-group K order produced by the quantiser, which
@@ -47,7 +48,6 @@ constexpr int kWarpB = 0, kWarpMma = 1, kWarpP = 2, kEpiWarp0 = 3, kEpiWarps = 8
 constexpr int kThreads = (kUnpWarp0 + kUnpWarps) * 32;  // 608
 constexpr int kEpiThreads = kEpiWarps * 32;
 constexpr int kHalfCols = 16;                           // columns per epilogue warp per round
-constexpr int kStagingBytes = 2 * kHalfCols * kBM * 4;  // one staging buffer (fp32 / int32)
 
 template <int BN>
 struct TcLayout {
@@ -57,13 +57,12 @@ struct TcLayout {
     // Ring depths: the token ring is as deep as shared memory allows, since its TMA round
     // trip (about 1 - 1.5 us measured on B200) sets the main-loop cadence.
     static constexpr int kDA = BN >= 256 ? 3 : 4;
-    static constexpr int kDB = BN >= 256 ? 4 : BN >= 128 ? 6 : 8;
+    static constexpr int kDB = BN >= 256 ? 5 : BN >= 128 ? 8 : 8;
     static constexpr int kDP = BN >= 256 ? 4 : 8;
     static constexpr int kOffA = 0;
     static constexpr int kOffB = kOffA + kDA * kA;
     static constexpr int kOffP = kOffB + kDB * kB;
-    static constexpr int kOffStage = kOffP + kDP * kP;
-    static constexpr int kOffBar = kOffStage + 2 * kStagingBytes;
+    static constexpr int kOffBar = kOffP + kDP * kP;
     static constexpr int kNumBars = 2 * (kDA + kDB + kDP) + 4;
     static constexpr int kSmem = kOffBar + kNumBars * 8 + 16 + 1024;  // + slot, flag, align
     static constexpr uint32_t kAccCols = BN;  // columns per accumulator buffer
@@ -71,10 +70,6 @@ struct TcLayout {
     static_assert(kA % 1024 == 0 && kB % 1024 == 0, "swizzled tiles need 1024-byte alignment");
     static_assert(kSmem <= 232448, "shared memory budget");
 };
-
-__device__ __forceinline__ void epilogue_bar_sync() {
-    asm volatile("bar.sync 1, %0;" ::"n"(kEpiThreads) : "memory");
-}
 
 template <int N>
 __device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, uint32_t (&v)[N]) {
@@ -282,13 +277,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
         const int quarter = warp & 3;
         const int colhalf = (warp - kEpiWarp0) >> 2;
         const int n_local = quarter * 32 + lane;
-        const int et = threadIdx.x - kEpiWarp0 * 32;  // 0 .. 255
-        const int esz = p.out_kind == 0 ? 2 : 4;
         constexpr int kHC = BN / 2 < kHalfCols ? BN / 2 : kHalfCols;  // columns per warp per round
         constexpr int kRounds = BN / (2 * kHC);
-        // Staging buffers alternate on a round counter that runs across tiles, so a buffer is
-        // rewritten only after the barrier that follows every thread's copy-out of it.
-        int round_run = 0;
         int i = 0;
         for (int t = blockIdx.x; t < num_tiles; t += gridDim.x, ++i) {
             const TileCoord tc = tile_coord(p, t, BN);
@@ -314,11 +304,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
             mbar_wait_bounded(&acc_full[buf], (i >> 1) & 1, p.err, kErrWaitAccum, abort_flag);
             tc_fence_after();
             const uint32_t d = tmem_base + uint32_t(buf) * L::kAccCols + (uint32_t(quarter * 32) << 16);
-            const bool vec_ok = ((pr.N * esz) % 16) == 0;  // every output row 16-byte aligned
-            uint8_t* ybase = static_cast<uint8_t*>(pr.y);
 #pragma unroll 1
-            for (int r = 0; r < kRounds; ++r, ++round_run) {
-                uint8_t* stage = smem + L::kOffStage + (round_run & 1) * kStagingBytes;
+            for (int r = 0; r < kRounds; ++r) {
                 const int col0 = r * 2 * kHC + colhalf * kHC;  // this warp's first column
                 uint32_t v[kHC];
                 tmem_ld_cols<kHC>(d + uint32_t(col0), v);
@@ -333,54 +320,33 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
                     rx[c] = __shfl_sync(0xFFFFFFFFu, mine, slot % 32);
                 }
                 tmem_ld_wait();
-                // staged row index = column within the round (0 .. 2*kHC-1)
-                const int srow0 = colhalf * kHC;
-                if (p.out_kind == 2) {
+                // Lanes hold adjacent weight rows n, so each store of column c writes 32
+                // adjacent outputs of token m0 + col0 + c. (Structured branch: the warp
+                // reconverges before the next aligned TMEM load.)
+                if (nvalid) {
+                    const int64_t mbase = int64_t(tc.m0) + col0;
+                    if (p.out_kind == 2) {
+                        int32_t* yp = static_cast<int32_t*>(pr.y) + mbase * pr.N + n;
 #pragma unroll
-                    for (int c = 0; c < kHC; ++c)
-                        reinterpret_cast<int32_t*>(stage)[(srow0 + c) * kBM + n_local] = int32_t(v[c]);
-                } else if (p.out_kind == 0) {
-                    __nv_bfloat16 yb[kHC];
+                        for (int c = 0; c < kHC; ++c)
+                            if (mbase + c < p.M) yp[int64_t(c) * pr.N] = int32_t(v[c]);
+                    } else if (p.out_kind == 0) {
+                        __nv_bfloat16* yp = static_cast<__nv_bfloat16*>(pr.y) + mbase * pr.N + n;
 #pragma unroll
-                    for (int c = 0; c < kHC; ++c)
-                        yb[c] = __float2bfloat16_rn(
-                            __fmul_rn(__int2float_rn(int32_t(v[c])), __fmul_rn(sw, rx[c])));
-#pragma unroll
-                    for (int c = 0; c < kHC; ++c)
-                        reinterpret_cast<__nv_bfloat16*>(stage)[(srow0 + c) * kBM + n_local] = yb[c];
-                } else {
-                    float yf[kHC];
-#pragma unroll
-                    for (int c = 0; c < kHC; ++c)
-                        yf[c] = __fmul_rn(__int2float_rn(int32_t(v[c])), __fmul_rn(sw, rx[c]));
-#pragma unroll
-                    for (int c = 0; c < kHC; ++c)
-                        reinterpret_cast<float*>(stage)[(srow0 + c) * kBM + n_local] = yf[c];
-                }
-                epilogue_bar_sync();
-                // coalesced copy-out: 2*kHC token rows of 128 contiguous outputs
-                const int row_bytes = kBM * esz;
-                const int chunks_per_row = row_bytes / 16;
-                const int vals_per_chunk = 16 / esz;
-                for (int q = et; q < 2 * kHC * chunks_per_row; q += kEpiThreads) {
-                    const int rrow = q / chunks_per_row;
-                    const int ch = q - rrow * chunks_per_row;
-                    const int64_t m = int64_t(tc.m0) + r * 2 * kHC + rrow;
-                    if (m >= p.M) continue;
-                    const int64_t nn = int64_t(tc.n0) + int64_t(ch) * vals_per_chunk;
-                    const uint8_t* src = stage + size_t(rrow) * row_bytes + size_t(ch) * 16;
-                    uint8_t* dst = ybase + (m * pr.N + nn) * esz;
-                    if (vec_ok && nn + vals_per_chunk <= pr.N) {
-                        *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(src);
+                        for (int c = 0; c < kHC; ++c)
+                            if (mbase + c < p.M)
+                                yp[int64_t(c) * pr.N] = __float2bfloat16_rn(
+                                    __fmul_rn(__int2float_rn(int32_t(v[c])), __fmul_rn(sw, rx[c])));
                     } else {
-                        for (int e = 0; e < vals_per_chunk && nn + e < pr.N; ++e) {
-                            if (esz == 2)
-                                reinterpret_cast<uint16_t*>(dst)[e] = reinterpret_cast<const uint16_t*>(src)[e];
-                            else
-                                reinterpret_cast<uint32_t*>(dst)[e] = reinterpret_cast<const uint32_t*>(src)[e];
-                        }
+                        float* yp = static_cast<float*>(pr.y) + mbase * pr.N + n;
+#pragma unroll
+                        for (int c = 0; c < kHC; ++c)
+                            if (mbase + c < p.M)
+                                yp[int64_t(c) * pr.N] =
+                                    __fmul_rn(__int2float_rn(int32_t(v[c])), __fmul_rn(sw, rx[c]));
                     }
                 }
+                __syncwarp();
             }
             // accumulator read out: hand it back to the MMA warp
             tc_fence_before();
