@@ -22,6 +22,20 @@ inline size_t ws_total_bytes(int64_t M, int64_t K) {
     return ws_q_bytes(M, K) + 2 * ws_scale_bytes(M);
 }
 
+// Optional split-K area after the base workspace: one int32 arrival counter and one int32
+// accumulation tile (128 weight rows x BN tokens) per split tile; the quantiser zeroes the
+// area on every call. Split-K runs only when the caller's workspace holds it.
+constexpr int kMaxSplitTiles = 80;
+int tc_pick_bn(int64_t M);
+inline size_t ws_split_cnt_bytes() { return align256(size_t(kMaxSplitTiles) * 4); }
+// Split-K runs only with token tiles of at most 128.
+inline size_t ws_split_tile_bytes(int64_t M) {
+    return size_t(128) * size_t(tc_pick_bn(M) < 128 ? tc_pick_bn(M) : 128) * 4;
+}
+inline size_t ws_split_bytes(int64_t M) {
+    return ws_split_cnt_bytes() + size_t(kMaxSplitTiles) * ws_split_tile_bytes(M);
+}
+
 // ----------------------------------------------------------------------------- GEMV
 struct GemvProj {
     const uint8_t* packed;
@@ -51,8 +65,11 @@ bool gemv_supported(int64_t M, int64_t K);
 // ----------------------------------------------------------------------------- quantisation
 // mode 0: natural-order q (public bitnet_quant_act); mode 1: permuted q + s_x + r_x for
 // the tensor-core path. q_in != nullptr: copy-permute given int8 q (no scales).
+// zero / zero_bytes: a 16-byte aligned region (multiple of 16 bytes) the launch clears, spread
+// over its CTAs (the split-K area of the GEMM that follows), or null.
 cudaError_t launch_quant(const uint16_t* x, const int8_t* q_in, int64_t M, int64_t K, int8_t* q,
-                         float* s_x, float* r_x, int permuted, cudaStream_t stream, bool pdl);
+                         float* s_x, float* r_x, int permuted, cudaStream_t stream, bool pdl,
+                         void* zero = nullptr, int64_t zero_bytes = 0);
 
 // ----------------------------------------------------------------------------- packing
 cudaError_t launch_pack_weights(const float* W, int64_t N, int64_t K, int per_row,
@@ -73,8 +90,12 @@ struct alignas(64) TcParams {
     CUtensorMap tmap_w[kMaxProj];  // packed weights (N, K/4) u8, box {32, 128}
     CUtensorMap tmap_q;            // workspace q (M, K) s8, box {128, BN}, 128-byte swizzle
     TcProj proj[kMaxProj];
-    const float* r_x;  // (M) 1 / s_x
-    int32_t* err;      // watchdog word
+    const float* r_x;     // (M) 1 / s_x
+    int32_t* err;         // watchdog word
+    int32_t* split_cnt;   // split-K: arrival counter per tile (zeroed by the quantiser)
+    int32_t* split_acc;   // split-K: int32 accumulation tile per tile, [tile][token][row]
+    int32_t splits;       // K splits per tile (1 = none)
+    int32_t pad2;
     int64_t K;
     int32_t M;
     int32_t nproj;
@@ -83,8 +104,8 @@ struct alignas(64) TcParams {
 };
 
 // Token-tile width chosen for M.
-int tc_pick_bn(int64_t M);
 cudaError_t launch_tc_gemm(const TcParams& p, int bn, cudaStream_t stream, bool pdl);
+int tc_num_sms();
 
 // Encodes the TMA descriptors (driver entry point fetched through the runtime).
 bool encode_tmap_2d_u8(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer,

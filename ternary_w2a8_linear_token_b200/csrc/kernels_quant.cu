@@ -73,7 +73,9 @@ __global__ void __launch_bounds__(kThreads) quant_rows_kernel(const uint16_t* __
                                                               int8_t* __restrict__ q,
                                                               float* __restrict__ s_x,
                                                               float* __restrict__ r_x,
-                                                              int permuted) {
+                                                              int permuted,
+                                                              uint4* __restrict__ zero,
+                                                              int64_t zero_words) {
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const int64_t m = int64_t(blockIdx.x) * kRowsPerCta + warp;
@@ -81,6 +83,10 @@ __global__ void __launch_bounds__(kThreads) quant_rows_kernel(const uint16_t* __
 
     pdl_wait();
     pdl_trigger();
+    // Clear the consumer GEMM's split-K area (counters and accumulation tiles) for this call.
+    for (int64_t i = int64_t(blockIdx.x) * kThreads + threadIdx.x; i < zero_words;
+         i += int64_t(gridDim.x) * kThreads)
+        zero[i] = make_uint4(0u, 0u, 0u, 0u);
     if (m >= M) return;  // whole warp leaves together
 
     float s = 0.0f;
@@ -164,7 +170,8 @@ __global__ void __launch_bounds__(kThreads) quant_rows_kernel(const uint16_t* __
 }  // namespace
 
 cudaError_t launch_quant(const uint16_t* x, const int8_t* q_in, int64_t M, int64_t K, int8_t* q,
-                         float* s_x, float* r_x, int permuted, cudaStream_t stream, bool pdl) {
+                         float* s_x, float* r_x, int permuted, cudaStream_t stream, bool pdl,
+                         void* zero, int64_t zero_bytes) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>((M + kRowsPerCta - 1) / kRowsPerCta));
     cfg.blockDim = dim3(kThreads);
@@ -175,7 +182,8 @@ cudaError_t launch_quant(const uint16_t* x, const int8_t* q_in, int64_t M, int64
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = pdl ? 1 : 0;
-    return cudaLaunchKernelEx(&cfg, quant_rows_kernel, x, q_in, M, K, q, s_x, r_x, permuted);
+    return cudaLaunchKernelEx(&cfg, quant_rows_kernel, x, q_in, M, K, q, s_x, r_x, permuted,
+                              static_cast<uint4*>(zero), zero_bytes / 16);
 }
 
 }  // namespace bitnet

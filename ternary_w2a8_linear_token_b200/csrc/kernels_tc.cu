@@ -108,6 +108,79 @@ __device__ __forceinline__ TileCoord tile_coord(const TcParams& p, int t, int bn
     return c;
 }
 
+// Barrier among the 8 epilogue warps only (named barrier 1).
+__device__ __forceinline__ void epilogue_bar_sync() {
+    asm volatile("bar.sync 1, %0;" ::"n"(kEpiThreads) : "memory");
+}
+
+// rx[c] = 1/s_x of column c of round r: lane l of rx_pre holds slot q*32 + l = r*kHC + c.
+template <int kHC, int kPre>
+__device__ __forceinline__ void spread_rx(const float (&rx_pre)[kPre], int r, float (&rx)[kHC]) {
+#pragma unroll
+    for (int c = 0; c < kHC; ++c) {
+        const int slot = r * kHC + c;
+        float mine = 0.0f;
+#pragma unroll
+        for (int q = 0; q < kPre; ++q)
+            if (q == slot / 32) mine = rx_pre[q];
+        rx[c] = __shfl_sync(0xFFFFFFFFu, mine, slot % 32);
+    }
+}
+
+// Dequantises kHC columns of accumulators (tokens m0 .. m0 + kHC - 1, weight row n) and
+// stores them: lanes hold adjacent rows n, so each store writes 32 adjacent outputs of one
+// token. Structured branch: the warp reconverges before the caller's next aligned TMEM load.
+template <int kHC>
+__device__ __forceinline__ void store_cols(const TcParams& p, const TcProj& pr, int m0, int64_t n,
+                                           bool nvalid, float sw, const float (&rx)[kHC],
+                                           const uint32_t (&v)[kHC]) {
+    if (nvalid) {
+        const int64_t mbase = m0;
+        if (p.out_kind == 2) {
+            int32_t* yp = static_cast<int32_t*>(pr.y) + mbase * pr.N + n;
+#pragma unroll
+            for (int c = 0; c < kHC; ++c)
+                if (mbase + c < p.M) yp[int64_t(c) * pr.N] = int32_t(v[c]);
+        } else if (p.out_kind == 0) {
+            __nv_bfloat16* yp = static_cast<__nv_bfloat16*>(pr.y) + mbase * pr.N + n;
+#pragma unroll
+            for (int c = 0; c < kHC; ++c)
+                if (mbase + c < p.M)
+                    yp[int64_t(c) * pr.N] = __float2bfloat16_rn(
+                        __fmul_rn(__int2float_rn(int32_t(v[c])), __fmul_rn(sw, rx[c])));
+        } else {
+            float* yp = static_cast<float*>(pr.y) + mbase * pr.N + n;
+#pragma unroll
+            for (int c = 0; c < kHC; ++c)
+                if (mbase + c < p.M)
+                    yp[int64_t(c) * pr.N] =
+                        __fmul_rn(__int2float_rn(int32_t(v[c])), __fmul_rn(sw, rx[c]));
+        }
+    }
+    __syncwarp();
+}
+
+// Work unit u = (tile t, K split sp): K stages [kb, kb + ns) of tile t.
+struct Unit {
+    int t, sp, kb, ns;
+};
+
+__device__ __forceinline__ Unit unit_of(int u, int splits, int num_k) {
+    Unit w;
+    w.t = u / splits;
+    w.sp = u - w.t * splits;
+    w.kb = (w.sp * num_k) / splits;
+    w.ns = ((w.sp + 1) * num_k) / splits - w.kb;
+    return w;
+}
+
+// K stage of the i-th stage of a unit: a whole tile rotates its start (see tile_coord); a
+// split unit walks its own K range.
+__device__ __forceinline__ int stage_k(const Unit& w, const TileCoord& tc, int i, int splits,
+                                       int num_k) {
+    return splits == 1 ? (tc.kt0 + i) % num_k : w.kb + i;
+}
+
 template <int BN>
 __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_constant__ TcParams p) {
     using L = TcLayout<BN>;
@@ -131,6 +204,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
     const int num_k = static_cast<int>((p.K + kBK - 1) / kBK);
     const int m_tiles = (p.M + BN - 1) / BN;
     const int num_tiles = m_tiles * p.n_tiles_total;
+    const int splits = p.splits;
+    const int num_units = num_tiles * splits;
 
     if (warp == kWarpB) {
         if (lane == 0) {
@@ -169,14 +244,15 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
             // ---------------- token tiles (written by the quantiser grid)
             pdl_wait();
             int kc = 0;
-            for (int t = blockIdx.x; t < num_tiles; t += gridDim.x) {
-                const TileCoord tc = tile_coord(p, t, BN);
-                for (int kt = 0; kt < num_k; ++kt, ++kc) {
+            for (int u = blockIdx.x; u < num_units; u += gridDim.x) {
+                const Unit w = unit_of(u, splits, num_k);
+                const TileCoord tc = tile_coord(p, w.t, BN);
+                for (int kt = 0; kt < w.ns; ++kt, ++kc) {
                     const int s = kc % L::kDB;
                     const uint32_t ph = (kc / L::kDB) & 1;
                     mbar_wait_bounded(&b_empty[s], ph ^ 1, p.err, kErrWaitEmpty, abort_flag);
                     mbar_arrive_expect_tx(&b_full[s], L::kB);
-                    const int kr = (tc.kt0 + kt) % num_k;
+                    const int kr = stage_k(w, tc, kt, splits, num_k);
                     tma_load_2d(smem + L::kOffB + s * L::kB, &p.tmap_q, &b_full[s], kr * kBK, tc.m0);
                 }
             }
@@ -189,14 +265,15 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
             // ---------------- packed weight tiles (independent of earlier grids)
             for (int j = 0; j < p.nproj; ++j) tma_prefetch_desc(&p.tmap_w[j]);
             int kc = 0;
-            for (int t = blockIdx.x; t < num_tiles; t += gridDim.x) {
-                const TileCoord tc = tile_coord(p, t, BN);
-                for (int kt = 0; kt < num_k; ++kt, ++kc) {
+            for (int u = blockIdx.x; u < num_units; u += gridDim.x) {
+                const Unit w = unit_of(u, splits, num_k);
+                const TileCoord tc = tile_coord(p, w.t, BN);
+                for (int kt = 0; kt < w.ns; ++kt, ++kc) {
                     const int s = kc % L::kDP;
                     const uint32_t ph = (kc / L::kDP) & 1;
                     mbar_wait_bounded(&p_empty[s], ph ^ 1, p.err, kErrWaitEmpty, abort_flag);
                     mbar_arrive_expect_tx(&p_full[s], L::kP);
-                    const int kr = (tc.kt0 + kt) % num_k;
+                    const int kr = stage_k(w, tc, kt, splits, num_k);
                     tma_load_2d(smem + L::kOffP + s * L::kP, &p.tmap_w[tc.proj], &p_full[s],
                                 kr * (kBK / 4), tc.n0);
                 }
@@ -210,13 +287,14 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
             // ---------------- MMA issuer
             constexpr uint32_t idesc = idesc_i8(kBM, BN);
             int kc = 0, i = 0;
-            for (int t = blockIdx.x; t < num_tiles; t += gridDim.x, ++i) {
+            for (int u = blockIdx.x; u < num_units; u += gridDim.x, ++i) {
+                const Unit w = unit_of(u, splits, num_k);
                 const int buf = i & 1;
                 mbar_wait_bounded(&acc_empty[buf], ((i >> 1) & 1) ^ 1, p.err, kErrWaitAccum,
                                   abort_flag);
                 tc_fence_after();
                 const uint32_t d = tmem_base + uint32_t(buf) * L::kAccCols;
-                for (int kt = 0; kt < num_k; ++kt, ++kc) {
+                for (int kt = 0; kt < w.ns; ++kt, ++kc) {
                     const int sa = kc % L::kDA, sb = kc % L::kDB;
                     mbar_wait_bounded(&a_full[sa], (kc / L::kDA) & 1, p.err, kErrWaitUnpack, abort_flag);
                     mbar_wait_bounded(&b_full[sb], (kc / L::kDB) & 1, p.err, kErrWaitTmaFull, abort_flag);
@@ -243,8 +321,9 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
         const int row = ut >> 1;                      // weight row of the tile
         const int half = ut & 1;                      // which 16 packed bytes (64 weights)
         int kc = 0;
-        for (int t = blockIdx.x; t < num_tiles; t += gridDim.x) {
-            for (int kt = 0; kt < num_k; ++kt, ++kc) {
+        for (int u = blockIdx.x; u < num_units; u += gridDim.x) {
+            const Unit w = unit_of(u, splits, num_k);
+            for (int kt = 0; kt < w.ns; ++kt, ++kc) {
                 const int sp = kc % L::kDP, sa = kc % L::kDA;
                 mbar_wait_bounded(&p_full[sp], (kc / L::kDP) & 1, p.err, kErrWaitTmaFull, abort_flag);
                 const uint4 pk = *reinterpret_cast<const uint4*>(smem + L::kOffP + sp * L::kP +
@@ -273,15 +352,19 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
         }
     } else {
         // ---------------- epilogue (warps 3-10: TMEM lane quarter warp % 4, column half)
-        pdl_wait();  // r_x comes from the quantiser grid; y may be read by earlier grids
+        pdl_wait();  // r_x and split counters come from the quantiser grid; y may be read earlier
         const int quarter = warp & 3;
         const int colhalf = (warp - kEpiWarp0) >> 2;
         const int n_local = quarter * 32 + lane;
+        const int et = threadIdx.x - kEpiWarp0 * 32;  // 0 .. 255
+        volatile int32_t* last_flag = reinterpret_cast<volatile int32_t*>(tmem_slot + 2);
         constexpr int kHC = BN / 2 < kHalfCols ? BN / 2 : kHalfCols;  // columns per warp per round
         constexpr int kRounds = BN / (2 * kHC);
+        constexpr int kPre = (kRounds * kHC + 31) / 32;
         int i = 0;
-        for (int t = blockIdx.x; t < num_tiles; t += gridDim.x, ++i) {
-            const TileCoord tc = tile_coord(p, t, BN);
+        for (int u = blockIdx.x; u < num_units; u += gridDim.x, ++i) {
+            const Unit w = unit_of(u, splits, num_k);
+            const TileCoord tc = tile_coord(p, w.t, BN);
             const TcProj& pr = p.proj[tc.proj];
             const int64_t n = int64_t(tc.n0) + n_local;
             const bool nvalid = n < pr.N;
@@ -292,66 +375,72 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
             const int buf = i & 1;
             // 1/s_x of this warp's columns, fetched before the accumulator is ready: lane l
             // holds token (round r, column l % kHC) for r = l / kHC (+ rounds of 32 / kHC).
-            constexpr int kPre = (kRounds * kHC + 31) / 32;
             float rx_pre[kPre];
 #pragma unroll
-            for (int u = 0; u < kPre; ++u) {
-                const int slot = u * 32 + lane;  // = round * kHC + column
+            for (int q = 0; q < kPre; ++q) {
+                const int slot = q * 32 + lane;  // = round * kHC + column
                 const int rr = slot / kHC, cc = slot % kHC;
                 const int64_t m = int64_t(tc.m0) + rr * 2 * kHC + colhalf * kHC + cc;
-                rx_pre[u] = (p.out_kind != 2 && rr < kRounds && m < p.M) ? p.r_x[m] : 0.0f;
+                rx_pre[q] = (p.out_kind != 2 && rr < kRounds && m < p.M) ? p.r_x[m] : 0.0f;
             }
             mbar_wait_bounded(&acc_full[buf], (i >> 1) & 1, p.err, kErrWaitAccum, abort_flag);
             tc_fence_after();
             const uint32_t d = tmem_base + uint32_t(buf) * L::kAccCols + (uint32_t(quarter * 32) << 16);
+            if (splits == 1) {
 #pragma unroll 1
-            for (int r = 0; r < kRounds; ++r) {
-                const int col0 = r * 2 * kHC + colhalf * kHC;  // this warp's first column
-                uint32_t v[kHC];
-                tmem_ld_cols<kHC>(d + uint32_t(col0), v);
-                float rx[kHC];
-#pragma unroll
-                for (int c = 0; c < kHC; ++c) {
-                    const int slot = r * kHC + c;
-                    float mine = 0.0f;
-#pragma unroll
-                    for (int u = 0; u < kPre; ++u)
-                        if (u == slot / 32) mine = rx_pre[u];
-                    rx[c] = __shfl_sync(0xFFFFFFFFu, mine, slot % 32);
+                for (int r = 0; r < kRounds; ++r) {
+                    const int col0 = r * 2 * kHC + colhalf * kHC;  // this warp's first column
+                    uint32_t v[kHC];
+                    tmem_ld_cols<kHC>(d + uint32_t(col0), v);
+                    float rx[kHC];
+                    spread_rx<kHC, kPre>(rx_pre, r, rx);
+                    tmem_ld_wait();
+                    store_cols<kHC>(p, pr, tc.m0 + col0, n, nvalid, sw, rx, v);
                 }
-                tmem_ld_wait();
-                // Lanes hold adjacent weight rows n, so each store of column c writes 32
-                // adjacent outputs of token m0 + col0 + c. (Structured branch: the warp
-                // reconverges before the next aligned TMEM load.)
-                if (nvalid) {
-                    const int64_t mbase = int64_t(tc.m0) + col0;
-                    if (p.out_kind == 2) {
-                        int32_t* yp = static_cast<int32_t*>(pr.y) + mbase * pr.N + n;
+                // accumulator read out: hand it back to the MMA warp
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&acc_empty[buf]);
+            } else {
+                // Split unit: this CTA adds its int32 partial tile into the tile's accumulation
+                // tile, [tile][token][row]; a warp adds 32 adjacent rows per reduction.
+                int32_t* acc = p.split_acc + size_t(w.t) * BN * kBM;
+#pragma unroll 1
+                for (int r = 0; r < kRounds; ++r) {
+                    const int col0 = r * 2 * kHC + colhalf * kHC;
+                    uint32_t v[kHC];
+                    tmem_ld_cols<kHC>(d + uint32_t(col0), v);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int c = 0; c < kHC; ++c)
+                        atomicAdd(acc + size_t(col0 + c) * kBM + n_local, int32_t(v[c]));
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&acc_empty[buf]);
+                // The last unit of the tile to arrive reads the summed tile (exact int32 adds,
+                // so the arrival order does not matter) and writes the outputs; no CTA waits
+                // for another.
+                __threadfence();
+                epilogue_bar_sync();
+                if (et == 0) *last_flag = atomicAdd(&p.split_cnt[w.t], 1) == splits - 1 ? 1 : 0;
+                epilogue_bar_sync();
+                if (*last_flag) {
+                    __threadfence();
+#pragma unroll 1
+                    for (int r = 0; r < kRounds; ++r) {
+                        const int col0 = r * 2 * kHC + colhalf * kHC;
+                        uint32_t v[kHC];
 #pragma unroll
                         for (int c = 0; c < kHC; ++c)
-                            if (mbase + c < p.M) yp[int64_t(c) * pr.N] = int32_t(v[c]);
-                    } else if (p.out_kind == 0) {
-                        __nv_bfloat16* yp = static_cast<__nv_bfloat16*>(pr.y) + mbase * pr.N + n;
-#pragma unroll
-                        for (int c = 0; c < kHC; ++c)
-                            if (mbase + c < p.M)
-                                yp[int64_t(c) * pr.N] = __float2bfloat16_rn(
-                                    __fmul_rn(__int2float_rn(int32_t(v[c])), __fmul_rn(sw, rx[c])));
-                    } else {
-                        float* yp = static_cast<float*>(pr.y) + mbase * pr.N + n;
-#pragma unroll
-                        for (int c = 0; c < kHC; ++c)
-                            if (mbase + c < p.M)
-                                yp[int64_t(c) * pr.N] =
-                                    __fmul_rn(__int2float_rn(int32_t(v[c])), __fmul_rn(sw, rx[c]));
+                            v[c] = uint32_t(__ldcg(acc + size_t(col0 + c) * kBM + n_local));
+                        float rx[kHC];
+                        spread_rx<kHC, kPre>(rx_pre, r, rx);
+                        store_cols<kHC>(p, pr, tc.m0 + col0, n, nvalid, sw, rx, v);
                     }
                 }
-                __syncwarp();
+                epilogue_bar_sync();  // last_flag is reused by the next unit
             }
-            // accumulator read out: hand it back to the MMA warp
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&acc_empty[buf]);
         }
     }
 
@@ -382,8 +471,8 @@ cudaError_t launch_bn(const TcParams& p, cudaStream_t stream, bool pdl) {
     auto kern = tc_gemm_kernel<BN>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kSmem);
     if (e != cudaSuccess) return e;
-    const int tiles = ((p.M + BN - 1) / BN) * p.n_tiles_total;
-    const int grid = tiles < num_sms_cached() ? tiles : num_sms_cached();
+    const int units = ((p.M + BN - 1) / BN) * p.n_tiles_total * p.splits;
+    const int grid = units < num_sms_cached() ? units : num_sms_cached();
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(grid));
     cfg.blockDim = dim3(kThreads);
@@ -398,6 +487,8 @@ cudaError_t launch_bn(const TcParams& p, cudaStream_t stream, bool pdl) {
 }
 
 }  // namespace
+
+int tc_num_sms() { return num_sms_cached(); }
 
 int tc_pick_bn(int64_t M) {
     if (M <= 16) return 16;
