@@ -139,6 +139,22 @@ bitnet_status run_batch(const uint16_t* x_bf16, const int8_t* q_in, int64_t M, i
     if (!encode_tmap_2d_u8(&p.tmap_q, q_ws, uint64_t(K), uint64_t(M), uint64_t(K), 128,
                            uint32_t(bn), /*swizzle128=*/true))
         return BITNET_ERR_CUDA;
+    // Outputs go out through TMA stores when the rows of y are 16-byte aligned; otherwise
+    // the epilogue stores from registers.
+    const uint64_t elem = out_kind == 0 ? 2 : 4;
+    const int y_type = out_kind == 0   ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                       : out_kind == 1 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
+                                       : CU_TENSOR_MAP_DATA_TYPE_INT32;
+    for (int i = 0; i < b.nproj; ++i) {
+        const uint64_t N = uint64_t(b.proj[i].N);
+        p.proj[i].tma_store = 0;
+        if ((reinterpret_cast<uintptr_t>(b.proj[i].y) & 15) == 0 && (N * elem) % 16 == 0) {
+            if (!encode_tmap_2d(&p.tmap_y[i], y_type, b.proj[i].y, N, uint64_t(M), N * elem, 32,
+                                uint32_t(tc_store_cols(bn)), /*swizzle128=*/false))
+                return BITNET_ERR_CUDA;
+            p.proj[i].tma_store = 1;
+        }
+    }
     p.r_x = r_x;
     p.err = device_error_word();
     if (!p.err) return BITNET_ERR_CUDA;
@@ -196,9 +212,9 @@ int32_t* device_error_word() {
     return g_err_ptr[dev];
 }
 
-bool encode_tmap_2d_u8(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer,
-                       uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer,
-                       bool swizzle128) {
+bool encode_tmap_2d(CUtensorMap* map, int dtype, const void* base, uint64_t inner, uint64_t outer,
+                    uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer,
+                    bool swizzle128) {
     std::call_once(g_encode_once, [] {
         void* fn = nullptr;
         cudaDriverEntryPointQueryResult q;
@@ -212,7 +228,7 @@ bool encode_tmap_2d_u8(CUtensorMap* map, const void* base, uint64_t inner, uint6
     const cuuint64_t strides[1] = {row_stride_bytes};
     const cuuint32_t box[2] = {box_inner, box_outer};
     const cuuint32_t estride[2] = {1, 1};
-    const CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base),
+    const CUresult r = g_encode(map, static_cast<CUtensorMapDataType>(dtype), 2, const_cast<void*>(base),
                                 dims, strides, box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE,
                                 swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
                                 CU_TENSOR_MAP_L2_PROMOTION_L2_256B,

@@ -84,11 +84,14 @@ struct TcProj {
     int64_t N;
     int32_t per_row;
     int32_t tile_begin;  // first n-tile index of this projection in the flattened grid
+    int32_t tma_store;   // 1: tmap_y is valid and the epilogue stores through it
+    int32_t pad;
 };
 
 struct alignas(64) TcParams {
     CUtensorMap tmap_w[kMaxProj];  // packed weights (N, K/4) u8, box {32, 128}
     CUtensorMap tmap_q;            // workspace q (M, K) s8, box {128, BN}, 128-byte swizzle
+    CUtensorMap tmap_y[kMaxProj];  // outputs (M, N), box {32 rows, tc_store_cols(BN) tokens}
     TcProj proj[kMaxProj];
     const float* r_x;     // (M) 1 / s_x
     int32_t* err;         // watchdog word
@@ -103,14 +106,22 @@ struct alignas(64) TcParams {
     int32_t out_kind;  // 0 bf16, 1 f32, 2 int32
 };
 
-// Token-tile width chosen for M.
 cudaError_t launch_tc_gemm(const TcParams& p, int bn, cudaStream_t stream, bool pdl);
 int tc_num_sms();
+// Tokens per epilogue store box for token-tile width bn.
+inline int tc_store_cols(int bn) { return bn / 2 < 16 ? bn / 2 : 16; }
 
 // Encodes the TMA descriptors (driver entry point fetched through the runtime).
-bool encode_tmap_2d_u8(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer,
-                       uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer,
-                       bool swizzle128);
+// dtype: a CUtensorMapDataType value.
+bool encode_tmap_2d(CUtensorMap* map, int dtype, const void* base, uint64_t inner, uint64_t outer,
+                    uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer,
+                    bool swizzle128);
+inline bool encode_tmap_2d_u8(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer,
+                              uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer,
+                              bool swizzle128) {
+    return encode_tmap_2d(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, base, inner, outer,
+                          row_stride_bytes, box_inner, box_outer, swizzle128);
+}
 
 // Device watchdog word of the current device.
 int32_t* device_error_word();

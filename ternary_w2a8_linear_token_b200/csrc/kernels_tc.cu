@@ -19,9 +19,11 @@
 //              commits them to the A/B slots they read and, per tile, to the accumulator;
 //  warp 2      lane 0 loads packed weight tiles (128 rows x 32 bytes) into ring P with TMA;
 //  warps 3-10  epilogue, two warps per TMEM lane quarter splitting the columns: TMEM ->
-//              registers -> y = acc * (s_w * 1/s_x) -> stores (a warp writes 32 adjacent
-//              outputs of one token per store); then the accumulator goes back to the MMA
-//              warp;
+//              registers -> y = acc * (s_w * 1/s_x) -> a per-warp staging tile in shared
+//              memory -> TMA store (the tensor map clips ragged edges); the dequantisation
+//              factors of the tile's tokens sit in a shared table filled before the
+//              accumulator is ready, and the accumulator goes back to the MMA warp as soon
+//              as its last columns are in registers;
 //  warps 11-18 unpack ring P into ring A: codes - 1 per byte, written as the 128-byte
 //              swizzled K-major operand tile.
 // The token tile arrives in the permuted in-group K order produced by the quantiser, which
@@ -54,15 +56,19 @@ struct TcLayout {
     static constexpr int kA = kBM * kBK;      // unpacked weights, 16 KB
     static constexpr int kB = BN * kBK;       // token tile
     static constexpr int kP = kBM * kBK / 4;  // packed weights, 4 KB
-    // Ring depths: the token ring is as deep as shared memory allows, since its TMA round
-    // trip (about 1 - 1.5 us measured on B200) sets the main-loop cadence.
+    // Ring depths: measured on B200, shallower rings than these (2 unpacked, 4 token and
+    // 2 packed stages at BN = 256) run the main loop at the same cadence, so the rest of
+    // shared memory goes to the epilogue staging tiles.
     static constexpr int kDA = BN >= 256 ? 3 : 4;
-    static constexpr int kDB = BN >= 256 ? 5 : BN >= 128 ? 8 : 8;
-    static constexpr int kDP = BN >= 256 ? 4 : 8;
+    static constexpr int kDB = BN >= 256 ? 4 : BN >= 128 ? 6 : 8;
+    static constexpr int kDP = BN >= 128 ? 4 : 8;
+    static constexpr int kStage = 2048;  // per epilogue warp: 32 rows x 16 tokens x 4 bytes
     static constexpr int kOffA = 0;
     static constexpr int kOffB = kOffA + kDA * kA;
     static constexpr int kOffP = kOffB + kDB * kB;
-    static constexpr int kOffBar = kOffP + kDP * kP;
+    static constexpr int kOffStage = kOffP + kDP * kP;
+    static constexpr int kOffTab = kOffStage + kEpiWarps * kStage;  // BN floats
+    static constexpr int kOffBar = kOffTab + (BN * 4 + 15) / 16 * 16;
     static constexpr int kNumBars = 2 * (kDA + kDB + kDP) + 4;
     static constexpr int kSmem = kOffBar + kNumBars * 8 + 16 + 1024;  // + slot, flag, align
     static constexpr uint32_t kAccCols = BN;  // columns per accumulator buffer
@@ -127,12 +133,13 @@ __device__ __forceinline__ void spread_rx(const float (&rx_pre)[kPre], int r, fl
     }
 }
 
-// Dequantises kHC columns of accumulators (tokens m0 .. m0 + kHC - 1, weight row n) and
-// stores them: lanes hold adjacent rows n, so each store writes 32 adjacent outputs of one
-// token. Structured branch: the warp reconverges before the caller's next aligned TMEM load.
+// Stores kHC columns of outputs (tokens m0 .. m0 + kHC - 1, weight row n) from registers:
+// y = acc * f[c], where f[c] is the column's dequantisation factor s_w * (1/s_x); lanes hold
+// adjacent rows n, so each store writes 32 adjacent outputs of one token. Structured
+// branch: the warp reconverges before the caller's next aligned TMEM load.
 template <int kHC>
 __device__ __forceinline__ void store_cols(const TcParams& p, const TcProj& pr, int m0, int64_t n,
-                                           bool nvalid, float sw, const float (&rx)[kHC],
+                                           bool nvalid, const float (&f)[kHC],
                                            const uint32_t (&v)[kHC]) {
     if (nvalid) {
         const int64_t mbase = m0;
@@ -146,19 +153,74 @@ __device__ __forceinline__ void store_cols(const TcParams& p, const TcProj& pr, 
 #pragma unroll
             for (int c = 0; c < kHC; ++c)
                 if (mbase + c < p.M)
-                    yp[int64_t(c) * pr.N] = __float2bfloat16_rn(
-                        __fmul_rn(__int2float_rn(int32_t(v[c])), __fmul_rn(sw, rx[c])));
+                    yp[int64_t(c) * pr.N] =
+                        __float2bfloat16_rn(__fmul_rn(__int2float_rn(int32_t(v[c])), f[c]));
         } else {
             float* yp = static_cast<float*>(pr.y) + mbase * pr.N + n;
 #pragma unroll
             for (int c = 0; c < kHC; ++c)
-                if (mbase + c < p.M)
-                    yp[int64_t(c) * pr.N] =
-                        __fmul_rn(__int2float_rn(int32_t(v[c])), __fmul_rn(sw, rx[c]));
+                if (mbase + c < p.M) yp[int64_t(c) * pr.N] = __fmul_rn(__int2float_rn(int32_t(v[c])), f[c]);
         }
     }
     __syncwarp();
 }
+
+// Writes this warp's kHC x 32 output block into its staging tile, laid out [token][row] as
+// the TMA store box expects (a row of 32 outputs per token; lanes write adjacent elements).
+template <int kHC>
+__device__ __forceinline__ void stage_cols(int out_kind, uint8_t* buf, int lane,
+                                           const float (&f)[kHC], const uint32_t (&v)[kHC]) {
+    if (out_kind == 0) {
+        __nv_bfloat16* b = reinterpret_cast<__nv_bfloat16*>(buf) + lane;
+#pragma unroll
+        for (int c = 0; c < kHC; ++c)
+            b[c * 32] = __float2bfloat16_rn(__fmul_rn(__int2float_rn(int32_t(v[c])), f[c]));
+    } else if (out_kind == 1) {
+        float* b = reinterpret_cast<float*>(buf) + lane;
+#pragma unroll
+        for (int c = 0; c < kHC; ++c) b[c * 32] = __fmul_rn(__int2float_rn(int32_t(v[c])), f[c]);
+    } else {
+        int32_t* b = reinterpret_cast<int32_t*>(buf) + lane;
+#pragma unroll
+        for (int c = 0; c < kHC; ++c) b[c * 32] = int32_t(v[c]);
+    }
+}
+
+// Dequantisation factors of kHC consecutive tokens from the tile's shared table (a
+// broadcast read: every lane reads the same addresses). The table holds s_w * (1/s_x) for
+// a per-tensor scale and 1/s_x for per-row scales, where this lane's row scale sw is
+// applied here: f = s_w * (1/s_x) rounded once either way.
+template <int kHC>
+__device__ __forceinline__ void table_factors(const float* tab, bool per_row, float sw,
+                                              float (&f)[kHC]) {
+    const float4* t4 = reinterpret_cast<const float4*>(tab);
+#pragma unroll
+    for (int q = 0; q < kHC / 4; ++q) {
+        const float4 t = t4[q];
+        f[4 * q + 0] = t.x;
+        f[4 * q + 1] = t.y;
+        f[4 * q + 2] = t.z;
+        f[4 * q + 3] = t.w;
+    }
+    if (per_row) {
+#pragma unroll
+        for (int c = 0; c < kHC; ++c) f[c] = __fmul_rn(sw, f[c]);
+    }
+}
+
+// Position in a ring of D slots: the slot and the parity of its current phase, advanced
+// without divisions.
+template <int D>
+struct Ring {
+    int slot = 0;
+    uint32_t phase = 0;
+    __device__ __forceinline__ void next() {
+        if (++slot == D) {
+            slot = 0;
+            phase ^= 1u;
+        }
+    }
+};
 
 // Work unit u = (tile t, K split sp): K stages [kb, kb + ns) of tile t.
 struct Unit {
@@ -243,17 +305,17 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
         if (lane == 0) {
             // ---------------- token tiles (written by the quantiser grid)
             pdl_wait();
+            Ring<L::kDB> rb;
             int kc = 0;
             for (int u = blockIdx.x; u < num_units; u += gridDim.x) {
                 const Unit w = unit_of(u, splits, num_k);
                 const TileCoord tc = tile_coord(p, w.t, BN);
-                for (int kt = 0; kt < w.ns; ++kt, ++kc) {
-                    const int s = kc % L::kDB;
-                    const uint32_t ph = (kc / L::kDB) & 1;
-                    mbar_wait_bounded(&b_empty[s], ph ^ 1, p.err, kErrWaitEmpty, abort_flag);
-                    mbar_arrive_expect_tx(&b_full[s], L::kB);
+                for (int kt = 0; kt < w.ns; ++kt, ++kc, rb.next()) {
+                    mbar_wait_bounded(&b_empty[rb.slot], rb.phase ^ 1, p.err, kErrWaitEmpty, abort_flag);
+                    mbar_arrive_expect_tx(&b_full[rb.slot], L::kB);
                     const int kr = stage_k(w, tc, kt, splits, num_k);
-                    tma_load_2d(smem + L::kOffB + s * L::kB, &p.tmap_q, &b_full[s], kr * kBK, tc.m0);
+                    tma_load_2d(smem + L::kOffB + rb.slot * L::kB, &p.tmap_q, &b_full[rb.slot],
+                                kr * kBK, tc.m0);
                 }
             }
             for (int k = kc > L::kDB ? kc - L::kDB : 0; k < kc; ++k)  // drain
@@ -264,18 +326,17 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
         if (lane == 0) {
             // ---------------- packed weight tiles (independent of earlier grids)
             for (int j = 0; j < p.nproj; ++j) tma_prefetch_desc(&p.tmap_w[j]);
+            Ring<L::kDP> rp;
             int kc = 0;
             for (int u = blockIdx.x; u < num_units; u += gridDim.x) {
                 const Unit w = unit_of(u, splits, num_k);
                 const TileCoord tc = tile_coord(p, w.t, BN);
-                for (int kt = 0; kt < w.ns; ++kt, ++kc) {
-                    const int s = kc % L::kDP;
-                    const uint32_t ph = (kc / L::kDP) & 1;
-                    mbar_wait_bounded(&p_empty[s], ph ^ 1, p.err, kErrWaitEmpty, abort_flag);
-                    mbar_arrive_expect_tx(&p_full[s], L::kP);
+                for (int kt = 0; kt < w.ns; ++kt, ++kc, rp.next()) {
+                    mbar_wait_bounded(&p_empty[rp.slot], rp.phase ^ 1, p.err, kErrWaitEmpty, abort_flag);
+                    mbar_arrive_expect_tx(&p_full[rp.slot], L::kP);
                     const int kr = stage_k(w, tc, kt, splits, num_k);
-                    tma_load_2d(smem + L::kOffP + s * L::kP, &p.tmap_w[tc.proj], &p_full[s],
-                                kr * (kBK / 4), tc.n0);
+                    tma_load_2d(smem + L::kOffP + rp.slot * L::kP, &p.tmap_w[tc.proj],
+                                &p_full[rp.slot], kr * (kBK / 4), tc.n0);
                 }
             }
             for (int k = kc > L::kDP ? kc - L::kDP : 0; k < kc; ++k)  // drain
@@ -284,9 +345,14 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
         __syncwarp();
     } else if (warp == kWarpMma) {
         if (lane == 0) {
-            // ---------------- MMA issuer
+            // ---------------- MMA issuer. Descriptors are advanced by adding the encoded
+            // start-address offsets (bytes / 16) of the ring slot and the 32-byte K step.
             constexpr uint32_t idesc = idesc_i8(kBM, BN);
-            int kc = 0, i = 0;
+            const uint64_t a_desc0 = smem_desc_k_sw128(smem_addr(smem + L::kOffA));
+            const uint64_t b_desc0 = smem_desc_k_sw128(smem_addr(smem + L::kOffB));
+            Ring<L::kDA> ra;
+            Ring<L::kDB> rb;
+            int i = 0;
             for (int u = blockIdx.x; u < num_units; u += gridDim.x, ++i) {
                 const Unit w = unit_of(u, splits, num_k);
                 const int buf = i & 1;
@@ -294,19 +360,18 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
                                   abort_flag);
                 tc_fence_after();
                 const uint32_t d = tmem_base + uint32_t(buf) * L::kAccCols;
-                for (int kt = 0; kt < w.ns; ++kt, ++kc) {
-                    const int sa = kc % L::kDA, sb = kc % L::kDB;
-                    mbar_wait_bounded(&a_full[sa], (kc / L::kDA) & 1, p.err, kErrWaitUnpack, abort_flag);
-                    mbar_wait_bounded(&b_full[sb], (kc / L::kDB) & 1, p.err, kErrWaitTmaFull, abort_flag);
+                for (int kt = 0; kt < w.ns; ++kt, ra.next(), rb.next()) {
+                    mbar_wait_bounded(&a_full[ra.slot], ra.phase, p.err, kErrWaitUnpack, abort_flag);
+                    mbar_wait_bounded(&b_full[rb.slot], rb.phase, p.err, kErrWaitTmaFull, abort_flag);
                     tc_fence_after();
-                    const uint32_t a_base = smem_addr(smem + L::kOffA + sa * L::kA);
-                    const uint32_t b_base = smem_addr(smem + L::kOffB + sb * L::kB);
+                    const uint64_t ad = a_desc0 + uint64_t(ra.slot * (L::kA >> 4));
+                    const uint64_t bd = b_desc0 + uint64_t(rb.slot * (L::kB >> 4));
 #pragma unroll
                     for (int kk = 0; kk < kBK / 32; ++kk)
-                        mma_i8(d, smem_desc_k_sw128(a_base + kk * 32),
-                               smem_desc_k_sw128(b_base + kk * 32), idesc, (kt | kk) != 0 ? 1u : 0u);
-                    mma_commit(&a_empty[sa]);
-                    mma_commit(&b_empty[sb]);
+                        mma_i8(d, ad + uint64_t(2 * kk), bd + uint64_t(2 * kk), idesc,
+                               (kt | kk) != 0 ? 1u : 0u);
+                    mma_commit(&a_empty[ra.slot]);
+                    mma_commit(&b_empty[rb.slot]);
                 }
                 mma_commit(&acc_full[buf]);
             }
@@ -320,19 +385,18 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
         const int ut = threadIdx.x - kUnpWarp0 * 32;  // 0 .. 255
         const int row = ut >> 1;                      // weight row of the tile
         const int half = ut & 1;                      // which 16 packed bytes (64 weights)
-        int kc = 0;
+        Ring<L::kDP> rp;
+        Ring<L::kDA> ra;
         for (int u = blockIdx.x; u < num_units; u += gridDim.x) {
             const Unit w = unit_of(u, splits, num_k);
-            for (int kt = 0; kt < w.ns; ++kt, ++kc) {
-                const int sp = kc % L::kDP, sa = kc % L::kDA;
-                mbar_wait_bounded(&p_full[sp], (kc / L::kDP) & 1, p.err, kErrWaitTmaFull, abort_flag);
-                const uint4 pk = *reinterpret_cast<const uint4*>(smem + L::kOffP + sp * L::kP +
+            for (int kt = 0; kt < w.ns; ++kt, rp.next(), ra.next()) {
+                mbar_wait_bounded(&p_full[rp.slot], rp.phase, p.err, kErrWaitTmaFull, abort_flag);
+                const uint4 pk = *reinterpret_cast<const uint4*>(smem + L::kOffP + rp.slot * L::kP +
                                                                  row * 32 + half * 16);
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&p_empty[sp]);
-                mbar_wait_bounded(&a_empty[sa], ((kc / L::kDA) & 1) ^ 1, p.err, kErrWaitEmpty,
-                                  abort_flag);
-                uint8_t* arow = smem + L::kOffA + sa * L::kA + row * kBK;
+                if (lane == 0) mbar_arrive(&p_empty[rp.slot]);
+                mbar_wait_bounded(&a_empty[ra.slot], ra.phase ^ 1, p.err, kErrWaitEmpty, abort_flag);
+                uint8_t* arow = smem + L::kOffA + ra.slot * L::kA + row * kBK;
                 const uint32_t words[4] = {pk.x, pk.y, pk.z, pk.w};
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
@@ -347,7 +411,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
                 }
                 fence_proxy_async_smem();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&a_full[sa]);
+                if (lane == 0) mbar_arrive(&a_full[ra.slot]);
             }
         }
     } else {
@@ -358,9 +422,13 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
         const int n_local = quarter * 32 + lane;
         const int et = threadIdx.x - kEpiWarp0 * 32;  // 0 .. 255
         volatile int32_t* last_flag = reinterpret_cast<volatile int32_t*>(tmem_slot + 2);
+        uint8_t* stage = smem + L::kOffStage + (warp - kEpiWarp0) * L::kStage;
+        float* tab = reinterpret_cast<float*>(smem + L::kOffTab);
         constexpr int kHC = BN / 2 < kHalfCols ? BN / 2 : kHalfCols;  // columns per warp per round
         constexpr int kRounds = BN / (2 * kHC);
         constexpr int kPre = (kRounds * kHC + 31) / 32;
+        static_assert(kHC == 8 || kHC == 16, "store box width");
+        uint32_t staged_stores = 0;  // selects the half of the staging tile (2-byte outputs)
         int i = 0;
         for (int u = blockIdx.x; u < num_units; u += gridDim.x, ++i) {
             const Unit w = unit_of(u, splits, num_k);
@@ -373,35 +441,78 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
                              : pr.per_row   ? (nvalid ? pr.s_w[n] : 0.0f)
                                             : pr.s_w[0];
             const int buf = i & 1;
-            // 1/s_x of this warp's columns, fetched before the accumulator is ready: lane l
-            // holds token (round r, column l % kHC) for r = l / kHC (+ rounds of 32 / kHC).
-            float rx_pre[kPre];
-#pragma unroll
-            for (int q = 0; q < kPre; ++q) {
-                const int slot = q * 32 + lane;  // = round * kHC + column
-                const int rr = slot / kHC, cc = slot % kHC;
-                const int64_t m = int64_t(tc.m0) + rr * 2 * kHC + colhalf * kHC + cc;
-                rx_pre[q] = (p.out_kind != 2 && rr < kRounds && m < p.M) ? p.r_x[m] : 0.0f;
-            }
-            mbar_wait_bounded(&acc_full[buf], (i >> 1) & 1, p.err, kErrWaitAccum, abort_flag);
-            tc_fence_after();
-            const uint32_t d = tmem_base + uint32_t(buf) * L::kAccCols + (uint32_t(quarter * 32) << 16);
             if (splits == 1) {
+                // Dequantisation factors of the tile's tokens, filled while the main loop runs.
+                epilogue_bar_sync();  // every warp is done with the previous tile's table
+                if (et < BN) {
+                    const int64_t m = int64_t(tc.m0) + et;
+                    float fv = 0.0f;
+                    if (p.out_kind != 2 && m < p.M) {
+                        fv = p.r_x[m];
+                        if (!pr.per_row) fv = __fmul_rn(sw, fv);
+                    }
+                    tab[et] = fv;
+                }
+                epilogue_bar_sync();
+                mbar_wait_bounded(&acc_full[buf], (i >> 1) & 1, p.err, kErrWaitAccum, abort_flag);
+                tc_fence_after();
+                const uint32_t d =
+                    tmem_base + uint32_t(buf) * L::kAccCols + (uint32_t(quarter * 32) << 16);
+                const bool staged = pr.tma_store != 0;
 #pragma unroll 1
                 for (int r = 0; r < kRounds; ++r) {
                     const int col0 = r * 2 * kHC + colhalf * kHC;  // this warp's first column
                     uint32_t v[kHC];
                     tmem_ld_cols<kHC>(d + uint32_t(col0), v);
-                    float rx[kHC];
-                    spread_rx<kHC, kPre>(rx_pre, r, rx);
                     tmem_ld_wait();
-                    store_cols<kHC>(p, pr, tc.m0 + col0, n, nvalid, sw, rx, v);
+                    if (r == kRounds - 1) {
+                        // accumulator read out: hand it back to the MMA warp
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(&acc_empty[buf]);
+                    }
+                    float f[kHC];
+                    table_factors<kHC>(tab + col0, pr.per_row != 0, sw, f);
+                    if (staged) {
+                        // 2-byte outputs alternate between the two 1 KB halves of the staging
+                        // tile; 4-byte outputs use all 2 KB, so the previous store must have
+                        // read it out first.
+                        uint8_t* sb = stage + (p.out_kind == 0 ? (staged_stores & 1u) * 1024u : 0u);
+                        if (lane == 0) {
+                            if (p.out_kind == 0)
+                                bulk_wait_group_read<1>();
+                            else
+                                bulk_wait_group_read<0>();
+                        }
+                        __syncwarp();
+                        stage_cols<kHC>(p.out_kind, sb, lane, f, v);
+                        fence_proxy_async_smem();
+                        __syncwarp();
+                        const int x = tc.n0 + quarter * 32, y = tc.m0 + col0;
+                        if (lane == 0 && x < pr.N && y < p.M) {
+                            tma_store_2d(&p.tmap_y[tc.proj], sb, x, y);
+                            bulk_commit_group();
+                        }
+                        ++staged_stores;
+                    } else {
+                        store_cols<kHC>(p, pr, tc.m0 + col0, n, nvalid, f, v);
+                    }
                 }
-                // accumulator read out: hand it back to the MMA warp
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&acc_empty[buf]);
             } else {
+                // 1/s_x of this warp's columns, fetched before the accumulator is ready: lane l
+                // holds token (round r, column l % kHC) for r = l / kHC (+ rounds of 32 / kHC).
+                float rx_pre[kPre];
+#pragma unroll
+                for (int q = 0; q < kPre; ++q) {
+                    const int slot = q * 32 + lane;  // = round * kHC + column
+                    const int rr = slot / kHC, cc = slot % kHC;
+                    const int64_t m = int64_t(tc.m0) + rr * 2 * kHC + colhalf * kHC + cc;
+                    rx_pre[q] = (p.out_kind != 2 && rr < kRounds && m < p.M) ? p.r_x[m] : 0.0f;
+                }
+                mbar_wait_bounded(&acc_full[buf], (i >> 1) & 1, p.err, kErrWaitAccum, abort_flag);
+                tc_fence_after();
+                const uint32_t d =
+                    tmem_base + uint32_t(buf) * L::kAccCols + (uint32_t(quarter * 32) << 16);
                 // Split unit: this CTA adds its int32 partial tile into the tile's accumulation
                 // tile, [tile][token][row]; a warp adds 32 adjacent rows per reduction.
                 int32_t* acc = p.split_acc + size_t(w.t) * BN * kBM;
@@ -436,12 +547,19 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
                             v[c] = uint32_t(__ldcg(acc + size_t(col0 + c) * kBM + n_local));
                         float rx[kHC];
                         spread_rx<kHC, kPre>(rx_pre, r, rx);
-                        store_cols<kHC>(p, pr, tc.m0 + col0, n, nvalid, sw, rx, v);
+                        float f[kHC];
+#pragma unroll
+                        for (int c = 0; c < kHC; ++c) f[c] = __fmul_rn(sw, rx[c]);
+                        store_cols<kHC>(p, pr, tc.m0 + col0, n, nvalid, f, v);
                     }
                 }
                 epilogue_bar_sync();  // last_flag is reused by the next unit
             }
         }
+        // Staged stores must be complete before the CTA exits (their source is this CTA's
+        // shared memory, and the next grid reads y).
+        if (lane == 0) bulk_wait_group<0>();
+        __syncwarp();
     }
 
     tc_fence_before();
