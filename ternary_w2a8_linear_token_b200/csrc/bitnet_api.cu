@@ -121,7 +121,7 @@ bitnet_status run_batch(const uint16_t* x_bf16, const int8_t* q_in, int64_t M, i
     for (int i = 0; i < b.nproj; ++i) {
         const int64_t N = b.proj[i].N;
         if (!encode_tmap_2d_u8(&p.tmap_w[i], b.proj[i].packed, uint64_t(K / 4), uint64_t(N),
-                               uint64_t(K / 4), 32, 128, /*swizzle128=*/false))
+                               uint64_t(K / 4), 64, 128, /*swizzle128=*/false))
             return BITNET_ERR_CUDA;
         p.proj[i].s_w = b.proj[i].s_w;
         p.proj[i].y = b.proj[i].y;
@@ -130,12 +130,18 @@ bitnet_status run_batch(const uint16_t* x_bf16, const int8_t* q_in, int64_t M, i
         p.proj[i].tile_begin = tiles;
         tiles += static_cast<int>((N + 127) / 128);
     }
-    // Token tile width: the widest that M needs, narrowed from 256 to 128 when the 256-wide
-    // tiling would leave more than half of the SMs idle (twice the tiles, each half as long;
-    // measured on B200: M = 512, N = 2560 goes from 22.9 to 17.7 us per call).
+    // Token tile width: the widest that M needs; past 128 tokens, 192 or 128, whichever
+    // gives the shorter run of tile waves, a K stage of a BN-token tile costing about
+    // BN + 264 units (fitted to per-call times measured on B200 at M = 512 ... 4096).
     const int sms = tc_num_sms();
     int bn = tc_pick_bn(M);
-    if (bn == 256 && int64_t(tiles) * ((M + 255) / 256) * 2 <= sms) bn = 128;
+    if (bn > 128) {
+        auto waves_cost = [&](int64_t w) {
+            const int64_t t = int64_t(tiles) * ((M + w - 1) / w);
+            return ((t + sms - 1) / sms) * (w + 264);
+        };
+        if (waves_cost(128) <= waves_cost(bn)) bn = 128;
+    }
     if (!encode_tmap_2d_u8(&p.tmap_q, q_ws, uint64_t(K), uint64_t(M), uint64_t(K), 128,
                            uint32_t(bn), /*swizzle128=*/true))
         return BITNET_ERR_CUDA;
@@ -165,21 +171,22 @@ bitnet_status run_batch(const uint16_t* x_bf16, const int8_t* q_in, int64_t M, i
     p.out_kind = out_kind;
 
     // Split-K when the tiles leave most SMs idle and the workspace holds the split area:
-    // each tile's K range is cut into `splits` units (at least 4 K stages each) so that about
+    // each tile's K range is cut into `splits` units (at least 512 K bytes each) so that about
     // one unit runs per SM; units add their int32 partial tiles into a zeroed accumulation tile.
     p.splits = 1;
-    const int64_t num_k = (K + 127) / 128;
+    const int64_t num_k = (K + 255) / 256;  // 256-byte K stages
     const int64_t m_tiles = (M + bn - 1) / bn;
     const int64_t tiles_all = m_tiles * tiles;
     void* zero = nullptr;
     int64_t zero_bytes = 0;
-    // Measured on B200: splitting pays for token tiles of up to 128 with at most a quarter
-    // of the SMs busy; with 256-token tiles the reduction of the 128 KB partial tiles costs
-    // more than the shorter main loop saves.
-    if (bn <= 128 && tiles_all * 4 <= sms && tiles_all <= kMaxSplitTiles && num_k >= 8 &&
+    // Measured on B200: splitting pays for token tiles of up to 32, and of 64 with long K
+    // loops; for wider tiles the atomic reduction of the partial tiles costs more than the
+    // shorter main loop saves.
+    const bool split_pays = bn <= 32 || (bn == 64 && num_k >= 16);
+    if (split_pays && tiles_all * 4 <= sms && tiles_all <= kMaxSplitTiles && num_k >= 4 &&
         workspace_bytes >= ws_total_bytes(M, K) + ws_split_bytes(M)) {
         int64_t sp = sms / tiles_all;
-        if (sp > num_k / 4) sp = num_k / 4;
+        if (sp > num_k / 2) sp = num_k / 2;
         if (sp > 8) sp = 8;
         if (sp >= 2) {
             p.splits = static_cast<int32_t>(sp);

@@ -28,9 +28,9 @@ inline size_t ws_total_bytes(int64_t M, int64_t K) {
 constexpr int kMaxSplitTiles = 80;
 int tc_pick_bn(int64_t M);
 inline size_t ws_split_cnt_bytes() { return align256(size_t(kMaxSplitTiles) * 4); }
-// Split-K runs only with token tiles of at most 128.
+// Split-K runs only with token tiles of at most 64.
 inline size_t ws_split_tile_bytes(int64_t M) {
-    return size_t(128) * size_t(tc_pick_bn(M) < 128 ? tc_pick_bn(M) : 128) * 4;
+    return size_t(128) * size_t(tc_pick_bn(M) < 64 ? tc_pick_bn(M) : 64) * 4;
 }
 inline size_t ws_split_bytes(int64_t M) {
     return ws_split_cnt_bytes() + size_t(kMaxSplitTiles) * ws_split_tile_bytes(M);
@@ -89,7 +89,7 @@ struct TcProj {
 };
 
 struct alignas(64) TcParams {
-    CUtensorMap tmap_w[kMaxProj];  // packed weights (N, K/4) u8, box {32, 128}
+    CUtensorMap tmap_w[kMaxProj];  // packed weights (N, K/4) u8, box {64, 128}
     CUtensorMap tmap_q;            // workspace q (M, K) s8, box {128, BN}, 128-byte swizzle
     CUtensorMap tmap_y[kMaxProj];  // outputs (M, N), box {32 rows, tc_store_cols(BN) tokens}
     TcProj proj[kMaxProj];

@@ -6,26 +6,34 @@
 // (page "BitNet-Triton", section "技术架构：融合内核的三重优化", item 2 "INT8张量核心加速").
 //
 // Operand roles are swapped so that the weight rows fill the 128-row MMA dimension and
-// the tokens are the MMA N dimension (16 ... 256): D[n, m] in TMEM = T[n, :] . Q[m, :].
+// the tokens are the MMA N dimension (16 ... 192): D[n, m] in TMEM = T[n, :] . Q[m, :].
 // That keeps small token counts efficient and re-unpacks each weight tile once per
-// token tile of up to 256 tokens.
+// token tile of up to 192 tokens.
 //
-// One CTA per SM walks a static list of 128 x BN output tiles. Three shared-memory rings
-// decouple the stages of the main loop, and two TMEM accumulators let the epilogue of one
-// tile overlap the main loop of the next:
-//  warp 0      TMEM allocation; lane 0 loads token tiles (BN rows x 128 bytes, 128-byte
-//              swizzle) into ring B with TMA;
-//  warp 1      lane 0 issues 4 tcgen05.mma.kind::i8 (K = 32 each) per 128-byte K stage and
-//              commits them to the A/B slots they read and, per tile, to the accumulator;
-//  warp 2      lane 0 loads packed weight tiles (128 rows x 32 bytes) into ring P with TMA;
+// The unpacked weights go from registers straight into TMEM and feed the MMA as its A
+// operand from there. The main loop is bound by shared-memory traffic (TMA writes plus the
+// tensor core's operand reads, measured on B200), and this keeps the weight operand out
+// of shared memory altogether; TMEM then holds two accumulators and a 4-stage weight ring,
+// which caps the token tile at 192.
+//
+// One CTA per SM walks a static list of 128 x BN output tiles. Two shared-memory rings and
+// the TMEM weight ring decouple the stages of the main loop, and two TMEM accumulators let
+// the epilogue of one tile overlap the main loop of the next:
+//  warp 0      TMEM allocation; lane 0 loads token tiles (two BN-row x 128-byte boxes per
+//              256-byte K stage, 128-byte swizzle) into ring B with TMA;
+//  warp 1      lane 0 issues 8 tcgen05.mma.kind::i8 (K = 32 each) per 256-byte K stage and
+//              commits them to the A/B slots they read and, per tile, to the accumulator
+//              (the single issuing thread's barrier round trips, not the tensor core, set
+//              the cadence of 128-byte stages on B200, hence the wider stage);
+//  warp 2      lane 0 loads packed weight tiles (128 rows x 64 bytes) into ring P with TMA;
 //  warps 3-10  epilogue, two warps per TMEM lane quarter splitting the columns: TMEM ->
 //              registers -> y = acc * (s_w * 1/s_x) -> a per-warp staging tile in shared
 //              memory -> TMA store (the tensor map clips ragged edges); the dequantisation
 //              factors of the tile's tokens sit in a shared table filled before the
 //              accumulator is ready, and the accumulator goes back to the MMA warp as soon
 //              as its last columns are in registers;
-//  warps 11-18 unpack ring P into ring A: codes - 1 per byte, written as the 128-byte
-//              swizzled K-major operand tile.
+//  warps 11-18 unpack ring P into the TMEM weight ring: codes - 1 per byte, one row per
+//              TMEM lane, four K bytes per column.
 // The token tile arrives in the permuted in-group K order produced by the quantiser, which
 // is the order a packed word unpacks into with shifts and masks alone.
 //
@@ -44,7 +52,8 @@ namespace bitnet {
 namespace {
 
 constexpr int kBM = 128;  // weight rows per tile (MMA M)
-constexpr int kBK = 128;  // K bytes per stage
+constexpr int kBK = 256;   // K bytes per stage: 8 MMAs between barrier round trips
+constexpr int kSub = 128;  // K bytes per token sub-tile (TMA box width, 128-byte swizzle atom)
 constexpr int kWarpB = 0, kWarpMma = 1, kWarpP = 2, kEpiWarp0 = 3, kEpiWarps = 8,
               kUnpWarp0 = 11, kUnpWarps = 8;
 constexpr int kThreads = (kUnpWarp0 + kUnpWarps) * 32;  // 608
@@ -53,27 +62,33 @@ constexpr int kHalfCols = 16;                           // columns per epilogue 
 
 template <int BN>
 struct TcLayout {
-    static constexpr int kA = kBM * kBK;      // unpacked weights, 16 KB
-    static constexpr int kB = BN * kBK;       // token tile
-    static constexpr int kP = kBM * kBK / 4;  // packed weights, 4 KB
-    // Ring depths: measured on B200, shallower rings than these (2 unpacked, 4 token and
-    // 2 packed stages at BN = 256) run the main loop at the same cadence, so the rest of
-    // shared memory goes to the epilogue staging tiles.
-    static constexpr int kDA = BN >= 256 ? 3 : 4;
-    static constexpr int kDB = BN >= 256 ? 4 : BN >= 128 ? 6 : 8;
-    static constexpr int kDP = BN >= 128 ? 4 : 8;
+    static constexpr int kB = BN * kBK;       // token tile: kBK / kSub sub-tiles of BN x kSub
+    static constexpr int kP = kBM * kBK / 4;  // packed weights, 8 KB
+    // Ring depths. The unpacked weights live in TMEM (kDA stages of 64 columns), so shared
+    // memory carries only the token and packed-weight rings and the epilogue staging.
+    static constexpr int kDA = BN >= 192 ? 2 : 4;
+    static constexpr int kDB = BN >= 192 ? 3 : BN >= 128 ? 4 : 6;
+    static constexpr int kDP = 4;
     static constexpr int kStage = 2048;  // per epilogue warp: 32 rows x 16 tokens x 4 bytes
-    static constexpr int kOffA = 0;
-    static constexpr int kOffB = kOffA + kDA * kA;
+    static constexpr int kOffB = 0;
     static constexpr int kOffP = kOffB + kDB * kB;
     static constexpr int kOffStage = kOffP + kDP * kP;
     static constexpr int kOffTab = kOffStage + kEpiWarps * kStage;  // BN floats
     static constexpr int kOffBar = kOffTab + (BN * 4 + 15) / 16 * 16;
     static constexpr int kNumBars = 2 * (kDA + kDB + kDP) + 4;
     static constexpr int kSmem = kOffBar + kNumBars * 8 + 16 + 1024;  // + slot, flag, align
-    static constexpr uint32_t kAccCols = BN;  // columns per accumulator buffer
-    static constexpr uint32_t kTmemCols = 2 * BN < 32 ? 32 : 2 * BN;
-    static_assert(kA % 1024 == 0 && kB % 1024 == 0, "swizzled tiles need 1024-byte alignment");
+    // TMEM: two accumulators of BN columns, then the unpacked-weight ring.
+    static constexpr uint32_t kAccCols = BN;
+    static constexpr uint32_t kACol0 = 2 * BN;
+    static constexpr uint32_t kAStageCols = kBK / 4;
+    static constexpr uint32_t kTmemNeed = 2 * BN + kDA * kAStageCols;
+    static constexpr uint32_t kTmemCols = kTmemNeed <= 32    ? 32
+                                          : kTmemNeed <= 64  ? 64
+                                          : kTmemNeed <= 128 ? 128
+                                          : kTmemNeed <= 256 ? 256
+                                                             : 512;
+    static_assert(kTmemNeed <= 512, "TMEM budget");
+    static_assert(kB % 1024 == 0, "swizzled tiles need 1024-byte alignment");
     static_assert(kSmem <= 232448, "shared memory budget");
 };
 
@@ -314,8 +329,10 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
                     mbar_wait_bounded(&b_empty[rb.slot], rb.phase ^ 1, p.err, kErrWaitEmpty, abort_flag);
                     mbar_arrive_expect_tx(&b_full[rb.slot], L::kB);
                     const int kr = stage_k(w, tc, kt, splits, num_k);
-                    tma_load_2d(smem + L::kOffB + rb.slot * L::kB, &p.tmap_q, &b_full[rb.slot],
-                                kr * kBK, tc.m0);
+#pragma unroll
+                    for (int h = 0; h < kBK / kSub; ++h)
+                        tma_load_2d(smem + L::kOffB + rb.slot * L::kB + h * BN * kSub, &p.tmap_q,
+                                    &b_full[rb.slot], kr * kBK + h * kSub, tc.m0);
                 }
             }
             for (int k = kc > L::kDB ? kc - L::kDB : 0; k < kc; ++k)  // drain
@@ -345,10 +362,11 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
         __syncwarp();
     } else if (warp == kWarpMma) {
         if (lane == 0) {
-            // ---------------- MMA issuer. Descriptors are advanced by adding the encoded
-            // start-address offsets (bytes / 16) of the ring slot and the 32-byte K step.
+            // ---------------- MMA issuer. The token descriptor is advanced by adding the
+            // encoded start-address offsets (bytes / 16) of the ring slot and the 32-byte K
+            // step; the weight operand is read from its TMEM ring slot, 8 columns per K step.
             constexpr uint32_t idesc = idesc_i8(kBM, BN);
-            const uint64_t a_desc0 = smem_desc_k_sw128(smem_addr(smem + L::kOffA));
+            const uint32_t a_tmem0 = tmem_base + L::kACol0;
             const uint64_t b_desc0 = smem_desc_k_sw128(smem_addr(smem + L::kOffB));
             Ring<L::kDA> ra;
             Ring<L::kDB> rb;
@@ -364,12 +382,15 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
                     mbar_wait_bounded(&a_full[ra.slot], ra.phase, p.err, kErrWaitUnpack, abort_flag);
                     mbar_wait_bounded(&b_full[rb.slot], rb.phase, p.err, kErrWaitTmaFull, abort_flag);
                     tc_fence_after();
-                    const uint64_t ad = a_desc0 + uint64_t(ra.slot * (L::kA >> 4));
+                    const uint32_t at = a_tmem0 + uint32_t(ra.slot) * L::kAStageCols;
                     const uint64_t bd = b_desc0 + uint64_t(rb.slot * (L::kB >> 4));
 #pragma unroll
-                    for (int kk = 0; kk < kBK / 32; ++kk)
-                        mma_i8(d, ad + uint64_t(2 * kk), bd + uint64_t(2 * kk), idesc,
-                               (kt | kk) != 0 ? 1u : 0u);
+                    for (int kk = 0; kk < kBK / 32; ++kk) {
+                        const int h = kk / (kSub / 32), k32 = kk % (kSub / 32);
+                        mma_i8_tmem_a(d, at + uint32_t(8 * kk),
+                                      bd + uint64_t((h * BN * kSub) >> 4) + uint64_t(2 * k32), idesc,
+                                      (kt | kk) != 0 ? 1u : 0u);
+                    }
                     mma_commit(&a_empty[ra.slot]);
                     mma_commit(&b_empty[rb.slot]);
                 }
@@ -381,35 +402,42 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
         }
         __syncwarp();
     } else if (warp >= kUnpWarp0) {
-        // ---------------- unpack: ring P -> ring A
-        const int ut = threadIdx.x - kUnpWarp0 * 32;  // 0 .. 255
-        const int row = ut >> 1;                      // weight row of the tile
-        const int half = ut & 1;                      // which 16 packed bytes (64 weights)
+        // ---------------- unpack: ring P (shared memory) -> ring A (TMEM). A warp may only
+        // reach its own TMEM lane quarter (warp % 4); the two warps of a quarter take the two
+        // 128-weight halves of each row's 256-weight stage.
+        const int quarter = warp & 3;
+        const int half = (warp - kUnpWarp0) >> 2;
+        const int row = quarter * 32 + lane;  // weight row of the tile = TMEM lane
+        const uint32_t a_lane = tmem_base + (uint32_t(quarter * 32) << 16) + L::kACol0 +
+                                uint32_t(half * (L::kAStageCols / 2));
         Ring<L::kDP> rp;
         Ring<L::kDA> ra;
         for (int u = blockIdx.x; u < num_units; u += gridDim.x) {
             const Unit w = unit_of(u, splits, num_k);
             for (int kt = 0; kt < w.ns; ++kt, rp.next(), ra.next()) {
                 mbar_wait_bounded(&p_full[rp.slot], rp.phase, p.err, kErrWaitTmaFull, abort_flag);
-                const uint4 pk = *reinterpret_cast<const uint4*>(smem + L::kOffP + rp.slot * L::kP +
-                                                                 row * 32 + half * 16);
+                const uint8_t* prow = smem + L::kOffP + rp.slot * L::kP + row * (kBK / 4) + half * (kBK / 8);
+                const uint4 pk0 = *reinterpret_cast<const uint4*>(prow);
+                const uint4 pk1 = *reinterpret_cast<const uint4*>(prow + 16);
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&p_empty[rp.slot]);
-                mbar_wait_bounded(&a_empty[ra.slot], ra.phase ^ 1, p.err, kErrWaitEmpty, abort_flag);
-                uint8_t* arow = smem + L::kOffA + ra.slot * L::kA + row * kBK;
-                const uint32_t words[4] = {pk.x, pk.y, pk.z, pk.w};
+                // Codes c in {0, 1, 2} -> int8 t = c - 1. Packed word c holds 16 weights; its
+                // shifts by 0, 2, 4, 6 give the four 32-bit columns in the permuted in-group
+                // K order of the token operand.
+                const uint32_t words[8] = {pk0.x, pk0.y, pk0.z, pk0.w, pk1.x, pk1.y, pk1.z, pk1.w};
+                uint32_t t[32];
 #pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    const uint32_t wv = words[c];
-                    uint4 tv;
-                    tv.x = codes_to_ternary_s8x4(wv & 0x03030303u);
-                    tv.y = codes_to_ternary_s8x4((wv >> 2) & 0x03030303u);
-                    tv.z = codes_to_ternary_s8x4((wv >> 4) & 0x03030303u);
-                    tv.w = codes_to_ternary_s8x4((wv >> 6) & 0x03030303u);
-                    const int chunk = half * 4 + c;  // 16-byte chunk of the 128-byte row
-                    *reinterpret_cast<uint4*>(arow + ((chunk ^ (row & 7)) << 4)) = tv;
+                for (int c = 0; c < 8; ++c) {
+                    t[4 * c + 0] = codes_to_ternary_s8x4(words[c] & 0x03030303u);
+                    t[4 * c + 1] = codes_to_ternary_s8x4((words[c] >> 2) & 0x03030303u);
+                    t[4 * c + 2] = codes_to_ternary_s8x4((words[c] >> 4) & 0x03030303u);
+                    t[4 * c + 3] = codes_to_ternary_s8x4((words[c] >> 6) & 0x03030303u);
                 }
-                fence_proxy_async_smem();
+                mbar_wait_bounded(&a_empty[ra.slot], ra.phase ^ 1, p.err, kErrWaitEmpty, abort_flag);
+                tc_fence_after();
+                tmem_st_32x32b_x32(a_lane + uint32_t(ra.slot) * L::kAStageCols, t);
+                tmem_st_wait();
+                tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&a_full[ra.slot]);
             }
@@ -613,7 +641,7 @@ int tc_pick_bn(int64_t M) {
     if (M <= 32) return 32;
     if (M <= 64) return 64;
     if (M <= 128) return 128;
-    return 256;
+    return 192;
 }
 
 cudaError_t launch_tc_gemm(const TcParams& p, int bn, cudaStream_t stream, bool pdl) {
@@ -622,7 +650,7 @@ cudaError_t launch_tc_gemm(const TcParams& p, int bn, cudaStream_t stream, bool 
         case 32: return launch_bn<32>(p, stream, pdl);
         case 64: return launch_bn<64>(p, stream, pdl);
         case 128: return launch_bn<128>(p, stream, pdl);
-        default: return launch_bn<256>(p, stream, pdl);
+        default: return launch_bn<192>(p, stream, pdl);
     }
 }
 

@@ -125,7 +125,8 @@ I32_CASES = [  # (M, N, K): tile multiples, ragged tails and the minimum K
     (9, 130, 512), (16, 128, 256), (17, 257, 512), (63, 384, 640), (64, 128, 2560),
     (65, 129, 1024), (127, 256, 512), (128, 128, 128), (129, 300, 384), (255, 128, 512),
     (256, 256, 2560), (257, 129, 512), (600, 200, 448),
-    (300, 384, 2560), (1000, 640, 2560),  # 128-token tiles past M = 128, split-K with a tail
+    (300, 384, 2560), (1000, 640, 2560),  # 128-token tiles past M = 128
+    (48, 256, 4160), (20, 200, 1088),  # split-K with 64- and 32-token tiles, K not a stage multiple
 ]
 
 
@@ -176,6 +177,7 @@ LINEAR_CASES = [  # (M, N, K, per_row)
     (4, 6912, 2560, False), (6, 200, 1024, True), (8, 257, 512, False), (9, 129, 512, True),
     (31, 640, 2560, False), (64, 300, 512, True), (100, 256, 1024, False),
     (129, 131, 640, True), (300, 256, 512, False), (200, 640, 1024, True),
+    (40, 300, 4096, True),  # split-K, ragged tokens and rows
 ]
 
 
