@@ -130,8 +130,8 @@ bitnet_status run_batch(const uint16_t* x_bf16, const int8_t* q_in, int64_t M, i
         p.proj[i].tile_begin = tiles;
         tiles += static_cast<int>((N + 127) / 128);
     }
-    // Token tile width: the widest that M needs; past 128 tokens, 192 or 128, whichever
-    // gives the shorter run of tile waves, a K stage of a BN-token tile costing about
+    // Token tile width: the widest that M needs; past 128 tokens, 192, 160 or 128, whichever
+    // gives the shortest run of tile waves, a K stage of a BN-token tile costing about
     // BN + 264 units (fitted to per-call times measured on B200 at M = 512 ... 4096).
     const int sms = tc_num_sms();
     int bn = tc_pick_bn(M);
@@ -140,7 +140,14 @@ bitnet_status run_batch(const uint16_t* x_bf16, const int8_t* q_in, int64_t M, i
             const int64_t t = int64_t(tiles) * ((M + w - 1) / w);
             return ((t + sms - 1) / sms) * (w + 264);
         };
-        if (waves_cost(128) <= waves_cost(bn)) bn = 128;
+        int64_t best = waves_cost(bn);
+        for (int w : {160, 128}) {
+            const int64_t c = waves_cost(w);
+            if (c <= best) {
+                best = c;
+                bn = w;
+            }
+        }
     }
     if (!encode_tmap_2d_u8(&p.tmap_q, q_ws, uint64_t(K), uint64_t(M), uint64_t(K), 128,
                            uint32_t(bn), /*swizzle128=*/true))

@@ -66,8 +66,8 @@ struct TcLayout {
     static constexpr int kP = kBM * kBK / 4;  // packed weights, 8 KB
     // Ring depths. The unpacked weights live in TMEM (kDA stages of 64 columns), so shared
     // memory carries only the token and packed-weight rings and the epilogue staging.
-    static constexpr int kDA = BN >= 192 ? 2 : 4;
-    static constexpr int kDB = BN >= 192 ? 3 : BN >= 128 ? 4 : 6;
+    static constexpr int kDA = BN > 128 ? 2 : 4;
+    static constexpr int kDB = BN > 128 ? 3 : BN >= 128 ? 4 : 6;
     static constexpr int kDP = 4;
     static constexpr int kStage = 2048;  // per epilogue warp: 32 rows x 16 tokens x 4 bytes
     static constexpr int kOffB = 0;
@@ -456,6 +456,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
         constexpr int kRounds = BN / (2 * kHC);
         constexpr int kPre = (kRounds * kHC + 31) / 32;
         static_assert(kHC == 8 || kHC == 16, "store box width");
+        static_assert(BN % (2 * kHC) == 0, "whole epilogue rounds");
         uint32_t staged_stores = 0;  // selects the half of the staging tile (2-byte outputs)
         int i = 0;
         for (int u = blockIdx.x; u < num_units; u += gridDim.x, ++i) {
@@ -650,6 +651,7 @@ cudaError_t launch_tc_gemm(const TcParams& p, int bn, cudaStream_t stream, bool 
         case 32: return launch_bn<32>(p, stream, pdl);
         case 64: return launch_bn<64>(p, stream, pdl);
         case 128: return launch_bn<128>(p, stream, pdl);
+        case 160: return launch_bn<160>(p, stream, pdl);
         default: return launch_bn<192>(p, stream, pdl);
     }
 }
