@@ -307,15 +307,29 @@ cudaError_t launch_one(const GemvParams& p, cudaStream_t stream, bool pdl) {
     return cudaLaunchKernelEx(&cfg, kern, q);
 }
 
-// Rows per warp: two for short rows when the grid would exceed one CTA per SM, which
-// keeps more of this grid and the next one (started early by programmatic dependent
-// launch) resident together; more rows per warp lengthen the work left after the wait
-// for the previous grid, which costs more than it saves (measured on B200).
+// Rows per warp. One or two tokens run two CTAs per SM (so the next grid, started early by
+// programmatic dependent launch, loads its weights while this one finishes) and take two
+// rows per warp for short rows once the grid would exceed one CTA per SM; more rows per
+// warp lengthen the work left after the wait for the previous grid, which costs more than
+// it saves (measured on B200). Four or eight tokens run one CTA per SM and take as many
+// rows per warp as let one wave cover every row: a second wave would repeat each CTA's
+// quantisation of the tokens and its whole dependent chain. Register-resident weights cap
+// the rows per warp.
 template <int MT, int CPL>
 cudaError_t launch_cpl(const GemvParams& p, cudaStream_t stream, bool pdl) {
     const int64_t slots = int64_t(num_sms()) * kWarps;  // warps of one CTA per SM
-    if constexpr (CPL <= 2 && MT <= 2) {
-        if (p.total_rows > slots) return launch_one<MT, CPL, 2>(p, stream, pdl);
+    if constexpr (MT <= 2) {
+        if constexpr (CPL <= 2) {
+            if (p.total_rows > slots) return launch_one<MT, CPL, 2>(p, stream, pdl);
+        }
+    } else {
+        const int64_t need = (p.total_rows + slots - 1) / slots;
+        if constexpr (CPL <= 2 && MT <= 4) {
+            if (need >= 3) return launch_one<MT, CPL, 3>(p, stream, pdl);
+        }
+        if constexpr (CPL <= 2 || (MT <= 4 && CPL <= 4)) {
+            if (need >= 2) return launch_one<MT, CPL, 2>(p, stream, pdl);
+        }
     }
     return launch_one<MT, CPL, 1>(p, stream, pdl);
 }
