@@ -30,19 +30,20 @@ constexpr int kThreads = kWarps * 32;
 __device__ __forceinline__ float bf16_lo(uint32_t v) { return __uint_as_float(v << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }
 
-__device__ __forceinline__ int q8(float xv, float s) {
-    return min(max(__float2int_rn(__fmul_rn(xv, s)), -128), 127);
-}
+// q = rint(x * s_x). The definition's clamp to [-128, 127] never acts here: s_x = RN(127 / a)
+// with a = max(amax, 1e-5) >= |x|, so |x * s_x| <= 127 (1 + 2^-24)^2 < 127.5 and the rounded
+// value lies in [-127, 127].
+__device__ __forceinline__ int q8(float xv, float s) { return __float2int_rn(__fmul_rn(xv, s)); }
 
+// Low bytes of a, b, c, d -> one word (byte 0 = a).
 __device__ __forceinline__ uint32_t pack4(int a, int b, int c, int d) {
-    return (uint32_t(a) & 0xFFu) | ((uint32_t(b) & 0xFFu) << 8) | ((uint32_t(c) & 0xFFu) << 16) |
-           (uint32_t(d) << 24);
+    const uint32_t lo = __byte_perm(uint32_t(a), uint32_t(b), 0x0040);
+    const uint32_t hi = __byte_perm(uint32_t(c), uint32_t(d), 0x0040);
+    return __byte_perm(lo, hi, 0x5410);
 }
 
-__device__ __forceinline__ int bytesum(uint32_t w) {
-    return int(int8_t(w & 0xFF)) + int(int8_t((w >> 8) & 0xFF)) + int(int8_t((w >> 16) & 0xFF)) +
-           int(int8_t(w >> 24));
-}
+// Sum of the four signed bytes of w.
+__device__ __forceinline__ int bytesum(uint32_t w) { return __dp4a(int(w), 0x01010101, 0); }
 
 // See kernels_quant.cu: lane pair (h = 0, 1) of one 16-group -> this lane's 8 permuted bytes.
 __device__ __forceinline__ uint2 permute_group_half(uint2 nat, int h) {
