@@ -21,12 +21,14 @@
 // the epilogue of one tile overlap the main loop of the next:
 //  warp 0      TMEM allocation; lane 0 loads token tiles (two BN-row x 128-byte boxes per
 //              256-byte K stage, 128-byte swizzle) into ring B with TMA;
-//  warp 1      lane 0 issues 8 tcgen05.mma.kind::i8 (K = 32 each) per 256-byte K stage and
-//              commits them to the A/B slots they read and, per tile, to the accumulator
-//              (the single issuing thread's barrier round trips, not the tensor core, set
-//              the cadence of 128-byte stages on B200, hence the wider stage);
+//  warps 1, 19 lane 0 of each issues 8 tcgen05.mma.kind::i8 (K = 32 each) per 256-byte K
+//              stage, the two threads taking alternate stages, and commits them to the A/B
+//              slots they read and, per tile, to the accumulator (barrier round trips of a
+//              single issuing thread, not the tensor core, set the main-loop cadence on B200,
+//              hence the wide stage and the second issuer);
 //  warp 2      lane 0 loads packed weight tiles (128 rows x 64 bytes) into ring P with TMA;
-//  warps 3-10  epilogue, two warps per TMEM lane quarter splitting the columns: TMEM ->
+//  warps 3-10  epilogue, two warps per TMEM lane quarter splitting the columns; they zero
+//              each accumulator as they read it (every MMA accumulates): TMEM ->
 //              registers -> y = acc * (s_w * 1/s_x) -> a per-warp staging tile in shared
 //              memory -> TMA store (the tensor map clips ragged edges); the dequantisation
 //              factors of the tile's tokens sit in a shared table filled before the
@@ -55,8 +57,9 @@ constexpr int kBM = 128;  // weight rows per tile (MMA M)
 constexpr int kBK = 256;   // K bytes per stage: 8 MMAs between barrier round trips
 constexpr int kSub = 128;  // K bytes per token sub-tile (TMA box width, 128-byte swizzle atom)
 constexpr int kWarpB = 0, kWarpMma = 1, kWarpP = 2, kEpiWarp0 = 3, kEpiWarps = 8,
-              kUnpWarp0 = 11, kUnpWarps = 8;
-constexpr int kThreads = (kUnpWarp0 + kUnpWarps) * 32;  // 608
+              kUnpWarp0 = 11, kUnpWarps = 8, kWarpMma2 = 19;
+constexpr int kMmaIssuers = 2;                  // warps kWarpMma and kWarpMma2
+constexpr int kThreads = (kWarpMma2 + 1) * 32;  // 640
 constexpr int kEpiThreads = kEpiWarps * 32;
 constexpr int kHalfCols = 16;                           // columns per epilogue warp per round
 
@@ -66,9 +69,13 @@ struct TcLayout {
     static constexpr int kP = kBM * kBK / 4;  // packed weights, 8 KB
     // Ring depths. The unpacked weights live in TMEM (kDA stages of 64 columns), so shared
     // memory carries only the token and packed-weight rings and the epilogue staging.
+    // The two MMA issuers take the global K stages by parity, so the weight and token rings
+    // have even depths: each slot is then always consumed by the same issuer, in order, and
+    // no issuer can wait two phases ahead on one slot's barrier.
     static constexpr int kDA = BN > 128 ? 2 : 4;
-    static constexpr int kDB = BN > 128 ? 3 : BN >= 128 ? 4 : 6;
-    static constexpr int kDP = 4;
+    static constexpr int kDB = BN > 64 ? 4 : 6;
+    static constexpr int kDP = BN > 160 ? 2 : 4;
+    static_assert(kDA % 2 == 0 && kDB % 2 == 0, "one issuer per ring slot");
     static constexpr int kStage = 2048;  // per epilogue warp: 32 rows x 16 tokens x 4 bytes
     static constexpr int kOffB = 0;
     static constexpr int kOffP = kOffB + kDB * kB;
@@ -100,6 +107,14 @@ __device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, uint32_t (&v)[N]) {
         uint32_t(&r)[8] = *reinterpret_cast<uint32_t(*)[8]>(&v[8 * i]);
         tmem_ld_32x32b_x8(taddr + uint32_t(8 * i), r);
     }
+}
+
+template <int N>
+__device__ __forceinline__ void tmem_st_cols(uint32_t taddr, const uint32_t (&v)[N]) {
+    static_assert(N % 8 == 0, "columns in multiples of 8");
+#pragma unroll
+    for (int i = 0; i < N / 8; ++i)
+        tmem_st_32x32b_x8(taddr + uint32_t(8 * i), *reinterpret_cast<const uint32_t(*)[8]>(&v[8 * i]));
 }
 
 struct TileCoord {
@@ -244,6 +259,13 @@ struct Unit {
 
 __device__ __forceinline__ Unit unit_of(int u, int splits, int num_k) {
     Unit w;
+    if (splits == 1) {  // whole tiles: no divisions
+        w.t = u;
+        w.sp = 0;
+        w.kb = 0;
+        w.ns = num_k;
+        return w;
+    }
     w.t = u / splits;
     w.sp = u - w.t * splits;
     w.kb = (w.sp * num_k) / splits;
@@ -299,7 +321,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
                 mbar_init(&b_empty[s], 1);
             }
             for (int b = 0; b < 2; ++b) {
-                mbar_init(&acc_full[b], 1);
+                mbar_init(&acc_full[b], kMmaIssuers);
                 mbar_init(&acc_empty[b], kEpiWarps);
             }
             *abort_flag = 0;
@@ -360,25 +382,32 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
                 mbar_wait_bounded(&p_full[k % L::kDP], (k / L::kDP) & 1, p.err, kErrWaitDrain, nullptr);
         }
         __syncwarp();
-    } else if (warp == kWarpMma) {
+    } else if (warp == kWarpMma || warp == kWarpMma2) {
         if (lane == 0) {
-            // ---------------- MMA issuer. The token descriptor is advanced by adding the
-            // encoded start-address offsets (bytes / 16) of the ring slot and the 32-byte K
-            // step; the weight operand is read from its TMEM ring slot, 8 columns per K step.
+            // ---------------- MMA issuers: two threads take alternate K stages of each tile,
+            // so one thread's barrier waits and commits overlap the other's MMAs (one issuing
+            // thread left the tensor pipe idle between stages, measured on B200). Every MMA
+            // accumulates into an accumulator the epilogue zeroed; the int32 sums are exact in
+            // any order. The token descriptor is advanced by adding the encoded start-address
+            // offsets (bytes / 16) of the ring slot and the 32-byte K step; the weight operand
+            // is read from its TMEM ring slot, 8 columns per K step.
+            const int issuer = warp == kWarpMma ? 0 : 1;
             constexpr uint32_t idesc = idesc_i8(kBM, BN);
             const uint32_t a_tmem0 = tmem_base + L::kACol0;
             const uint64_t b_desc0 = smem_desc_k_sw128(smem_addr(smem + L::kOffB));
             Ring<L::kDA> ra;
             Ring<L::kDB> rb;
             int i = 0;
+            uint32_t g = 0;  // K stages of this CTA so far, over all its units
             for (int u = blockIdx.x; u < num_units; u += gridDim.x, ++i) {
                 const Unit w = unit_of(u, splits, num_k);
                 const int buf = i & 1;
-                mbar_wait_bounded(&acc_empty[buf], ((i >> 1) & 1) ^ 1, p.err, kErrWaitAccum,
-                                  abort_flag);
+                // The epilogue released both accumulators once after zeroing them at start.
+                mbar_wait_bounded(&acc_empty[buf], (i >> 1) & 1, p.err, kErrWaitAccum, abort_flag);
                 tc_fence_after();
                 const uint32_t d = tmem_base + uint32_t(buf) * L::kAccCols;
-                for (int kt = 0; kt < w.ns; ++kt, ra.next(), rb.next()) {
+                for (int kt = 0; kt < w.ns; ++kt, ++g, ra.next(), rb.next()) {
+                    if (int(g & 1u) != issuer) continue;  // the other issuer's stage
                     mbar_wait_bounded(&a_full[ra.slot], ra.phase, p.err, kErrWaitUnpack, abort_flag);
                     mbar_wait_bounded(&b_full[rb.slot], rb.phase, p.err, kErrWaitTmaFull, abort_flag);
                     tc_fence_after();
@@ -389,7 +418,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
                         const int h = kk / (kSub / 32), k32 = kk % (kSub / 32);
                         mma_i8_tmem_a(d, at + uint32_t(8 * kk),
                                       bd + uint64_t((h * BN * kSub) >> 4) + uint64_t(2 * k32), idesc,
-                                      (kt | kk) != 0 ? 1u : 0u);
+                                      1u);
                     }
                     mma_commit(&a_empty[ra.slot]);
                     mma_commit(&b_empty[rb.slot]);
@@ -458,6 +487,28 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
         static_assert(kHC == 8 || kHC == 16, "store box width");
         static_assert(BN % (2 * kHC) == 0, "whole epilogue rounds");
         uint32_t staged_stores = 0;  // selects the half of the staging tile (2-byte outputs)
+        // Every MMA accumulates, so an accumulator starts at zero: zero both now, and each
+        // one again as its columns are read out, before it goes back to the MMA warps.
+        uint32_t zeros[kHC];
+#pragma unroll
+        for (int c = 0; c < kHC; ++c) zeros[c] = 0u;
+        {
+            const uint32_t lane_base = tmem_base + (uint32_t(quarter * 32) << 16);
+#pragma unroll 1
+            for (int b = 0; b < 2; ++b)
+#pragma unroll 1
+                for (int r = 0; r < kRounds; ++r)
+                    tmem_st_cols<kHC>(lane_base + uint32_t(b) * L::kAccCols +
+                                          uint32_t(r * 2 * kHC + colhalf * kHC),
+                                      zeros);
+            tmem_st_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(&acc_empty[0]);
+                mbar_arrive(&acc_empty[1]);
+            }
+        }
         int i = 0;
         for (int u = blockIdx.x; u < num_units; u += gridDim.x, ++i) {
             const Unit w = unit_of(u, splits, num_k);
@@ -494,8 +545,10 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
                     uint32_t v[kHC];
                     tmem_ld_cols<kHC>(d + uint32_t(col0), v);
                     tmem_ld_wait();
+                    tmem_st_cols<kHC>(d + uint32_t(col0), zeros);
                     if (r == kRounds - 1) {
-                        // accumulator read out: hand it back to the MMA warp
+                        // accumulator read out and zeroed: hand it back to the MMA warps
+                        tmem_st_wait();
                         tc_fence_before();
                         __syncwarp();
                         if (lane == 0) mbar_arrive(&acc_empty[buf]);
@@ -551,10 +604,12 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
                     uint32_t v[kHC];
                     tmem_ld_cols<kHC>(d + uint32_t(col0), v);
                     tmem_ld_wait();
+                    tmem_st_cols<kHC>(d + uint32_t(col0), zeros);
 #pragma unroll
                     for (int c = 0; c < kHC; ++c)
                         atomicAdd(acc + size_t(col0 + c) * kBM + n_local, int32_t(v[c]));
                 }
+                tmem_st_wait();
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&acc_empty[buf]);
