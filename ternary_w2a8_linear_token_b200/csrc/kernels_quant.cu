@@ -167,6 +167,64 @@ __global__ void __launch_bounds__(kThreads) quant_rows_kernel(const uint16_t* __
     }
 }
 
+// Rows of 4096 < K <= 14336: four warps per row, each thread holding up to 14 pieces of 8
+// values in registers, so x is read once (the one-warp kernel above takes two passes there).
+constexpr int kLongThreads = 256;
+constexpr int kLongRowThreads = 128;
+constexpr int kLongRows = kLongThreads / kLongRowThreads;
+constexpr int kLongPieces = 14;
+constexpr int64_t kLongMaxK = int64_t(kLongRowThreads) * kLongPieces * 8;
+
+__global__ void __launch_bounds__(kLongThreads) quant_long_rows_kernel(
+    const uint16_t* __restrict__ x, int64_t M, int64_t K, int8_t* __restrict__ q,
+    float* __restrict__ s_x, float* __restrict__ r_x, int permuted, uint4* __restrict__ zero,
+    int64_t zero_words) {
+    __shared__ uint32_t s_mx[kLongRows][kLongRowThreads / 32];
+    const int row = threadIdx.x / kLongRowThreads;
+    const int t = threadIdx.x % kLongRowThreads;
+    const int lane = threadIdx.x & 31;
+    const int64_t m = int64_t(blockIdx.x) * kLongRows + row;
+    const bool active = m < M;
+    const int64_t pieces = K / 8;
+
+    pdl_wait();
+    pdl_trigger();
+    for (int64_t i = int64_t(blockIdx.x) * kLongThreads + threadIdx.x; i < zero_words;
+         i += int64_t(gridDim.x) * kLongThreads)
+        zero[i] = make_uint4(0u, 0u, 0u, 0u);
+
+    const uint4* xr = reinterpret_cast<const uint4*>(x + (active ? m : 0) * K);
+    uint4 v[kLongPieces];
+#pragma unroll
+    for (int u = 0; u < kLongPieces; ++u) {
+        const int64_t c = int64_t(u) * kLongRowThreads + t;
+        v[u] = (active && c < pieces) ? xr[c] : make_uint4(0u, 0u, 0u, 0u);
+    }
+    uint32_t mx = 0;
+#pragma unroll
+    for (int u = 0; u < kLongPieces; ++u) mx = max(mx, absmax8_bits(v[u]));
+    mx = __reduce_max_sync(0xFFFFFFFFu, mx);
+    if (lane == 0) s_mx[row][t >> 5] = mx;
+    __syncthreads();
+    uint32_t all = 0;
+#pragma unroll
+    for (int w = 0; w < kLongRowThreads / 32; ++w) all = max(all, s_mx[row][w]);
+    const float s = __fdiv_rn(127.0f, fmaxf(bf16_bits_to_float(all), kEps));
+    if (active && t == 0) {
+        if (s_x) s_x[m] = s;
+        if (r_x) r_x[m] = __frcp_rn(s);
+    }
+    int8_t* qr = q + (active ? m : 0) * K;
+#pragma unroll
+    for (int u = 0; u < kLongPieces; ++u) {
+        if (int64_t(u) * kLongRowThreads >= pieces) break;  // uniform over the row's warps
+        const int64_t c = int64_t(u) * kLongRowThreads + t;  // lane pairs share a 16-group
+        const uint2 nat = quant8(v[u], s);
+        const uint2 out = permuted ? permute_group_half(nat, lane & 1) : nat;
+        if (active && c < pieces) reinterpret_cast<uint2*>(qr)[c] = out;
+    }
+}
+
 }  // namespace
 
 cudaError_t launch_quant(const uint16_t* x, const int8_t* q_in, int64_t M, int64_t K, int8_t* q,
@@ -182,6 +240,12 @@ cudaError_t launch_quant(const uint16_t* x, const int8_t* q_in, int64_t M, int64
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = pdl ? 1 : 0;
+    if (q_in == nullptr && K > int64_t(32) * kRegPieces * 8 && K <= kLongMaxK) {
+        cfg.gridDim = dim3(static_cast<unsigned>((M + kLongRows - 1) / kLongRows));
+        cfg.blockDim = dim3(kLongThreads);
+        return cudaLaunchKernelEx(&cfg, quant_long_rows_kernel, x, M, K, q, s_x, r_x, permuted,
+                                  static_cast<uint4*>(zero), zero_bytes / 16);
+    }
     return cudaLaunchKernelEx(&cfg, quant_rows_kernel, x, q_in, M, K, q, s_x, r_x, permuted,
                               static_cast<uint4*>(zero), zero_bytes / 16);
 }
