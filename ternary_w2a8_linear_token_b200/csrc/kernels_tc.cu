@@ -69,13 +69,16 @@ struct TcLayout {
     static constexpr int kP = kBM * kBK / 4;  // packed weights, 8 KB
     // Ring depths. The unpacked weights live in TMEM (kDA stages of 64 columns), so shared
     // memory carries only the token and packed-weight rings and the epilogue staging.
-    // The two MMA issuers take the global K stages by parity, so the weight and token rings
-    // have even depths: each slot is then always consumed by the same issuer, in order, and
-    // no issuer can wait two phases ahead on one slot's barrier.
-    static constexpr int kDA = BN > 128 ? 2 : 4;
+    // The two MMA issuers take the global K stages by parity. The token ring has an even
+    // depth, so each of its slots is always consumed by the same issuer, in order: its TMA
+    // fills may land out of order, and an issuer must never wait on a slot whose previous
+    // fill has not landed (a parity wait cannot tell the two phases apart). The weight ring
+    // needs no such rule: the unpack warps arrive in stage order, so when an issuer has
+    // consumed its previous stage g - 2, every stage up to g - 2 >= g - kDA has completed.
+    static constexpr int kDA = BN > 160 ? 2 : BN > 128 ? 3 : 4;
     static constexpr int kDB = BN > 64 ? 4 : 6;
     static constexpr int kDP = BN > 160 ? 2 : 4;
-    static_assert(kDA % 2 == 0 && kDB % 2 == 0, "one issuer per ring slot");
+    static_assert(kDB % 2 == 0, "one issuer per token-ring slot");
     static constexpr int kStage = 2048;  // per epilogue warp: 32 rows x 16 tokens x 4 bytes
     static constexpr int kOffB = 0;
     static constexpr int kOffP = kOffB + kDB * kB;
