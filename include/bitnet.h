@@ -207,9 +207,28 @@ bitnet_status bitnet_linear_noalloc(const uint16_t* x, int64_t M, int64_t K,
 /*
  * bitnet_check_device_errors — synchronises the current device, returns the library's
  * watchdog word in *flags (0 = no kernel gave up a bounded wait since the last check)
- * and clears it. Returns BITNET_ERR_TIMEOUT when the word was non-zero.
+ * and clears it. Returns BITNET_ERR_TIMEOUT when the word was non-zero. The word is an OR
+ * of the BITNET_WATCHDOG_* bits of the waits that expired.
  */
+#define BITNET_WATCHDOG_TMA_FULL (1 << 0)   /* a stage's TMA load never completed */
+#define BITNET_WATCHDOG_UNPACK (1 << 1)     /* unpacked weights never arrived */
+#define BITNET_WATCHDOG_EMPTY (1 << 2)      /* a ring slot was never released */
+#define BITNET_WATCHDOG_ACCUM (1 << 3)      /* an accumulator handoff never happened */
+#define BITNET_WATCHDOG_DRAIN (1 << 4)      /* copies or MMAs in flight at exit never completed */
+#define BITNET_WATCHDOG_SELFTEST (1 << 6)   /* bitnet_selftest_wait_timeout's wait */
 bitnet_status bitnet_check_device_errors(int32_t* flags);
+
+/*
+ * bitnet_selftest_wait_timeout — test hook for the failure detection, not on the hot path
+ * (the pages have no counterpart). Launches one thread that waits on an mbarrier nothing
+ * completes, through the same bounded wait every tensor-core kernel wait uses, with a limit
+ * of limit_ns nanoseconds of %globaltimer. On expiry the kernel ORs
+ * BITNET_WATCHDOG_SELFTEST into the watchdog word and returns (no trap, the context stays
+ * usable), so a following bitnet_check_device_errors returns BITNET_ERR_TIMEOUT.
+ * limit_ns must lie in [1e6, 2e9] (BITNET_ERR_UNSUPPORTED otherwise). Asynchronous on
+ * `stream`.
+ */
+bitnet_status bitnet_selftest_wait_timeout(int64_t limit_ns, void* stream);
 
 /* Human-readable name of a status code (static storage). */
 const char* bitnet_status_string(bitnet_status status);

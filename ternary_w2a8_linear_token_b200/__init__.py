@@ -40,6 +40,9 @@ SCALE_PER_TENSOR, SCALE_PER_ROW = 0, 1
 OUT_BF16, OUT_F32 = 0, 1
 PATH_AUTO, PATH_GEMV, PATH_TC = 0, 1, 2
 GEMV_MAX_M = 8
+WATCHDOG_TMA_FULL, WATCHDOG_UNPACK, WATCHDOG_EMPTY, WATCHDOG_ACCUM, WATCHDOG_DRAIN = (
+    1 << 0, 1 << 1, 1 << 2, 1 << 3, 1 << 4)
+WATCHDOG_SELFTEST = 1 << 6
 MAX_PROJ = 8
 
 _P, _I64, _I32, _SZ = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_size_t
@@ -67,6 +70,7 @@ _SIGS = {
     "bitnet_linear_noalloc": ([_P, _I64, _I64, _P, _P, ctypes.c_int, _I64, _P, ctypes.c_int, _P],
                               ctypes.c_int),
     "bitnet_check_device_errors": ([ctypes.POINTER(_I32)], ctypes.c_int),
+    "bitnet_selftest_wait_timeout": ([_I64, _P], ctypes.c_int),
     "bitnet_status_string": ([ctypes.c_int], ctypes.c_char_p),
     "bitnet_version": ([], _I32),
 }
@@ -238,6 +242,13 @@ def bitnet_check_device_errors() -> int:
     if st not in (OK, ERR_TIMEOUT):
         raise BitnetError(st, "bitnet_check_device_errors")
     return int(flags.value)
+
+
+def bitnet_selftest_wait_timeout(limit_ns: int, stream=None) -> None:
+    """Launches the watchdog self-test: one bounded wait on a barrier nothing completes."""
+    st = lib.bitnet_selftest_wait_timeout(int(limit_ns), _stream(stream))
+    if st != OK:
+        raise BitnetError(st, "bitnet_selftest_wait_timeout")
 
 
 def bitnet_version() -> int:

@@ -6,6 +6,8 @@
 #include <cstdint>
 #include <cuda_runtime.h>
 
+#include "bitnet.h"
+
 namespace bitnet {
 
 // Watchdog codes OR-ed into the library's device error word.
@@ -15,7 +17,12 @@ enum : int32_t {
     kErrWaitEmpty = 1 << 2,
     kErrWaitAccum = 1 << 3,
     kErrWaitDrain = 1 << 4,
+    kErrSelfTest = 1 << 6,
 };
+static_assert(kErrWaitTmaFull == BITNET_WATCHDOG_TMA_FULL && kErrWaitUnpack == BITNET_WATCHDOG_UNPACK &&
+                  kErrWaitEmpty == BITNET_WATCHDOG_EMPTY && kErrWaitAccum == BITNET_WATCHDOG_ACCUM &&
+                  kErrWaitDrain == BITNET_WATCHDOG_DRAIN && kErrSelfTest == BITNET_WATCHDOG_SELFTEST,
+              "watchdog bits match the public header");
 
 // A bounded wait gives up after this many nanoseconds of %globaltimer.
 constexpr uint64_t kWaitLimitNs = 1000ull * 1000ull * 1000ull;  // 1 s
@@ -67,7 +74,8 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 // kernel still ends). Once the abort flag is up, later waits return false at once. A
 // drain wait (abort == nullptr) ignores the flag and always runs to its own limit.
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, int32_t* err,
-                                                  int32_t code, volatile int32_t* abort) {
+                                                  int32_t code, volatile int32_t* abort,
+                                                  uint64_t limit_ns = kWaitLimitNs) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = global_timer_ns();
     uint32_t spins = 0;
@@ -77,7 +85,7 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
         if (spins > 256u) __nanosleep(spins > 4096u ? 256u : 64u);
         if ((++spins & 63u) == 0u) {
             if (abort && *abort) return false;
-            if (global_timer_ns() - t0 > kWaitLimitNs) {
+            if (global_timer_ns() - t0 > limit_ns) {
                 if (err) atomicOr(err, code);
                 if (abort) *abort = 1;
                 return false;

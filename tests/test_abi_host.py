@@ -106,6 +106,13 @@ def test_batch_argument_errors(bn):
     assert f(FAKE, 256, 512, arr, 2, 0, None, 0, None) == bn.ERR_WORKSPACE
 
 
+def test_watchdog_selftest_rejects_limits_before_launch(bn):
+    # Out-of-range limits are refused on the host; nothing is launched (no GPU here).
+    assert bn.lib.bitnet_selftest_wait_timeout(999_999, None) == bn.ERR_UNSUPPORTED
+    assert bn.lib.bitnet_selftest_wait_timeout(2_000_000_001, None) == bn.ERR_UNSUPPORTED
+    assert bn.lib.bitnet_selftest_wait_timeout(-1, None) == bn.ERR_UNSUPPORTED
+
+
 def test_other_calls_argument_errors(bn):
     L = bn.lib
     assert L.bitnet_pack_weights(None, 4, 64, 0, FAKE, FAKE, None) == bn.ERR_NULL
