@@ -158,6 +158,79 @@ def build_prefill(bn, torch, dev, M):
     return calls
 
 
+STACK_SPECS = {
+    # name: (layers, hidden, ffn, token counts M, per_row scales)
+    "2B-4T stack": (30, 2560, 6912, (1, 8, 32, 64), False),
+    "8B-class stack": (32, 4096, 14336, (1, 16, 128, 4096), True),
+}
+BATCHED = ("q", "k", "v", "gate", "up")  # share the layer input x_h
+
+
+def build_stack(bn, torch, dev, name):
+    """Device weights of one stack. Layer 0 follows the recipe (2B-4T: ternary P(0)=0.4 drawn
+    directly, per-tensor s_w ~ U(0.5, 2); 8B-class: latent W ~ N(0, 0.02^2) quantised per row by
+    bitnet_pack_weights) and is copied into every other layer's own buffers, so each layer
+    streams distinct memory; kernel time does not depend on the values, and parity of every
+    projection shape is covered by the tests."""
+    layers = STACK_SPECS[name][0]
+    base = {}
+    if name.startswith("2B"):
+        for proj, d in synth.stack2b_layer(0).items():
+            base[proj] = (bn.bitnet_pack_ternary(torch.from_numpy(d["t"]).to(dev)),
+                          torch.from_numpy(d["s_w"]).to(dev), False)
+    else:
+        for proj in synth.SHAPES_8B:
+            W = torch.from_numpy(synth.stack8b_latent(0, proj)).to(dev)
+            packed, s_w = bn.bitnet_pack_weights(W, True)
+            del W
+            base[proj] = (packed, s_w, True)
+    torch.cuda.synchronize()
+    return [base] + [{k: (p.clone(), s_.clone(), r) for k, (p, s_, r) in base.items()}
+                     for _ in range(layers - 1)]
+
+
+def run_stack(bn, torch, dev, name, stack, M, steps, warmup, flush, world, peaks):
+    """One pass = every layer back to back: bitnet_linear_batch(x_h -> q, k, v, gate, up),
+    bitnet_linear(x_h -> o), bitnet_linear(x_f -> down), on fixed synthetic inputs."""
+    layers, hidden, ffn, _, _ = STACK_SPECS[name]
+    gen = synth.stack2b_x if name.startswith("2B") else synth.stack8b_x
+    x_h = torch.from_numpy(gen(M, hidden, which=0).view(np.int16).copy()).to(dev).view(torch.bfloat16)
+    x_f = torch.from_numpy(gen(M, ffn, which=1).view(np.int16).copy()).to(dev).view(torch.bfloat16)
+    L0 = stack[0]
+    ys = [torch.empty((M, L0[p][0].shape[0]), dtype=torch.bfloat16, device=dev) for p in BATCHED]
+    y_o = torch.empty((M, hidden), dtype=torch.bfloat16, device=dev)
+    y_d = torch.empty((M, hidden), dtype=torch.bfloat16, device=dev)
+    tc = M > bn.GEMV_MAX_M
+    ws_h = bn.make_workspace(M, hidden, dev) if tc else None
+    ws_f = bn.make_workspace(M, ffn, dev) if tc else None
+
+    def one_pass():
+        for L in stack:
+            bn.bitnet_linear_batch(x_h, [L[p] for p in BATCHED], ys=ys, workspace=ws_h)
+            bn.bitnet_linear(x_h, *L["o"], y=y_o, workspace=ws_h)
+            bn.bitnet_linear(x_f, *L["down"], y=y_d, workspace=ws_f)
+
+    g = capture(torch, one_pass)
+    ms = timed_steps(torch, g.replay, steps, warmup, flush, world)
+    assert bn.bitnet_check_device_errors() == 0
+    ms_max, _ = reduce_over_ranks(ms, 0.0, world)
+    t = ms_max * 1e-3 / steps
+    shapes = [(L0[p][0].shape[0], L0[p][0].shape[1] * 4) for p in L0]
+    w_bytes = layers * sum(N * K // 4 + 4 * (N if L0[p][2] else 1)
+                           for p, (N, K) in zip(L0, shapes))
+    act_bytes = layers * sum(2 * M * K + 2 * M * N for N, K in shapes)
+    ops = layers * sum(2.0 * M * N * K for N, K in shapes)
+    int8_peak = peaks["bf16_tflops"] * INT8_PER_BF16
+    roof = max((w_bytes + act_bytes) / (peaks["hbm_gbs"] * 1e9), ops / (int8_peak * 1e12))
+    launches = layers * 3 * (2 if tc else 1)
+    del g
+    return {"stack": name, "M": M, "us_per_pass": t * 1e6, "tokens_per_s": M / t,
+            "GB_per_s": (w_bytes + act_bytes) / t / 1e9, "TOPS": ops / t / 1e12,
+            "roofline_us": roof * 1e6, "frac": roof / t,
+            "bound": "hbm" if (w_bytes + act_bytes) / (peaks["hbm_gbs"] * 1e9) >= ops / (int8_peak * 1e12)
+            else "tensor", "launches_per_pass": launches}, launches
+
+
 def run_calls(bn, calls):
     for c in calls:
         bn.bitnet_linear(c["x"], c["packed"], c["s_w"], False, y=c["y"], workspace=c.get("ws"))
@@ -348,6 +421,20 @@ def run_ours(args):
                                          "(nominal int8:bf16)",
                              "note": "per-call time includes the quantiser launch"}}
 
+    # ---------------- layer stacks (2B-4T and 8B-class, every layer back to back)
+    stacks = []
+    stack_launches = 0
+    if args.stacks == "all" and args.only == "all":
+        for name, spec in STACK_SPECS.items():
+            st = build_stack(bn, torch, dev, name)
+            for M in spec[3]:
+                r, nl = run_stack(bn, torch, dev, name, st, M, min(args.steps, 5), args.warmup,
+                                  flush, world, peaks)
+                stacks.append(r)
+                stack_launches += nl * min(args.steps, 5)
+            del st
+            torch.cuda.empty_cache()
+
     cpu = oracle_sample(args.cpu_seconds) if (rank == 0 and world == 1 and args.cpu_seconds > 0) \
         else None
 
@@ -375,9 +462,11 @@ def run_ours(args):
             "e2e": {"value": e2e_gbs, "unit": "GB/s",
                     "h2d_bytes_per_step": int(h_x.numel() * 2),
                     "d2h_bytes_per_step": int(h_y.numel() * 2)},
-            "gpu_launches": args.steps * launches_per_step * 2 + args.steps * 2 * len(pcalls),
+            "gpu_launches": args.steps * launches_per_step * 2 + args.steps * 2 * len(pcalls)
+                            + stack_launches,
             "clocks": clk.summary(),
             "gemm": gemm,
+            "stacks": stacks,
             "cpu_baseline": cpu,
         }
         print(json.dumps(line), flush=True)
@@ -401,6 +490,8 @@ def main():
                     help="weight replicas per decode step (0: enough to exceed 2x L2)")
     ap.add_argument("--prefill-m", type=int, default=PREFILL_M,
                     help="tokens of the prefill GEMM part")
+    ap.add_argument("--stacks", choices=["all", "none"], default="all",
+                    help="time the 2B-4T and 8B-class layer stacks (extra objects on the line)")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)  # at least 3 untimed warm-up steps
     if args.impl == "reference":
