@@ -200,7 +200,7 @@ def run_stack(bn, torch, dev, name, stack, M, steps, warmup, flush, world, peaks
     ys = [torch.empty((M, L0[p][0].shape[0]), dtype=torch.bfloat16, device=dev) for p in BATCHED]
     y_o = torch.empty((M, hidden), dtype=torch.bfloat16, device=dev)
     y_d = torch.empty((M, hidden), dtype=torch.bfloat16, device=dev)
-    tc = M > bn.GEMV_MAX_M
+    tc = M > bn.GEMV_AUTO_M
     ws_h = bn.make_workspace(M, hidden, dev) if tc else None
     ws_f = bn.make_workspace(M, ffn, dev) if tc else None
 

@@ -64,12 +64,15 @@ typedef enum {
 } bitnet_out_dtype;
 
 typedef enum {
-    BITNET_PATH_AUTO = 0, /* GEMV for M <= BITNET_GEMV_MAX_M, tensor-core GEMM above      */
+    BITNET_PATH_AUTO = 0, /* GEMV for M <= BITNET_GEMV_AUTO_M; for M up to                */
+                          /* BITNET_GEMV_MAX_M the tensor-core GEMM when the workspace    */
+                          /* holds it, else the GEMV; tensor-core GEMM above              */
     BITNET_PATH_GEMV = 1, /* force the dp4a GEMV with fused activation quantisation      */
     BITNET_PATH_TC = 2    /* force the tcgen05 GEMM (needs the workspace)                 */
 } bitnet_path;
 
 #define BITNET_GEMV_MAX_M 8
+#define BITNET_GEMV_AUTO_M 4
 #define BITNET_MAX_PROJ 8
 
 /*
@@ -110,9 +113,10 @@ bitnet_status bitnet_quant_act(const uint16_t* x, int64_t M, int64_t K, int8_t* 
 
 /*
  * Workspace bytes the tensor-core path of bitnet_linear / bitnet_linear_batch needs for
- * M tokens of width K (quantised activations and per-token scales). The GEMV path
- * (M <= BITNET_GEMV_MAX_M under BITNET_PATH_AUTO) uses none: callers that only run such
- * M may pass workspace = NULL.
+ * M tokens of width K (quantised activations and per-token scales). The GEMV path uses
+ * none: under BITNET_PATH_AUTO, calls with M <= BITNET_GEMV_MAX_M may pass workspace =
+ * NULL and then run the GEMV (for 5 <= M <= 8 a sufficient workspace selects the faster
+ * tensor-core path instead).
  */
 size_t bitnet_linear_workspace_size(int64_t M, int64_t K);
 
@@ -124,7 +128,7 @@ size_t bitnet_linear_workspace_size(int64_t M, int64_t K);
  *   s_w      [in]  fp32, 1 or N elements by `mode`.
  *   y        [out] (M, N) bf16 or fp32 by `out_dtype`.
  *   workspace, workspace_bytes: device scratch of at least bitnet_linear_workspace_size(M, K)
- *            bytes when the tensor-core path runs (M > BITNET_GEMV_MAX_M); its contents
+ *            bytes when the tensor-core path runs (M > BITNET_GEMV_AUTO_M); its contents
  *            on entry are ignored, and it must not be shared by calls that may overlap.
  * Epilogue arithmetic: acc = exact int32 sum; r = 1/s_x[m] (binary32, rounded);
  * y = (float)acc * (s_w[n or 0] * r), each product rounded; bf16 is RNE of that fp32

@@ -40,6 +40,7 @@ SCALE_PER_TENSOR, SCALE_PER_ROW = 0, 1
 OUT_BF16, OUT_F32 = 0, 1
 PATH_AUTO, PATH_GEMV, PATH_TC = 0, 1, 2
 GEMV_MAX_M = 8
+GEMV_AUTO_M = 4  # PATH_AUTO: GEMV up to here; 5..8 tokens take the tensor-core path given a workspace
 WATCHDOG_TMA_FULL, WATCHDOG_UNPACK, WATCHDOG_EMPTY, WATCHDOG_ACCUM, WATCHDOG_DRAIN = (
     1 << 0, 1 << 1, 1 << 2, 1 << 3, 1 << 4)
 WATCHDOG_SELFTEST = 1 << 6
@@ -151,7 +152,7 @@ def bitnet_quant_act(x: torch.Tensor, stream=None):
 
 
 def _ws_args(workspace: Optional[torch.Tensor], M: int, K: int, path: int, device):
-    need_tc = path == PATH_TC or (path == PATH_AUTO and M > GEMV_MAX_M)
+    need_tc = path == PATH_TC or (path == PATH_AUTO and M > GEMV_AUTO_M)
     if workspace is None:
         if not need_tc:
             return None, 0, None

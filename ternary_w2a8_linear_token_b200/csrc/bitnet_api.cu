@@ -74,17 +74,23 @@ bitnet_status check_workspace(void* ws, size_t bytes, int64_t M, int64_t K) {
     return BITNET_OK;
 }
 
-bool use_gemv(int64_t M, int64_t K, bitnet_path path) {
+// Five to eight tokens take the tensor-core path when the caller's workspace holds it: the
+// GEMV's per-CTA quantisation and dp4a work grow with the token count, and on B200 the
+// tensor-core path with 16-token tiles is as fast or faster there (2B-4T shapes, 8 tokens:
+// 10.7 / 8.7 / 20.9 / 27.2 us per GEMV call against about 10 / 9 / 11 / 15 us).
+bool use_gemv(int64_t M, int64_t K, bitnet_path path, const void* ws, size_t ws_bytes) {
     if (path == BITNET_PATH_GEMV) return true;
     if (path == BITNET_PATH_TC) return false;
-    return M <= BITNET_GEMV_MAX_M && gemv_supported(M, K);
+    if (M > BITNET_GEMV_MAX_M || !gemv_supported(M, K)) return false;
+    if (M <= BITNET_GEMV_AUTO_M) return true;
+    return !(ws && ws_bytes >= ws_total_bytes(M, K) && aligned(ws, 256));
 }
 
 // Runs a validated batch. x_bf16 or q_in (int8, contraction-only) is the input.
 bitnet_status run_batch(const uint16_t* x_bf16, const int8_t* q_in, int64_t M, int64_t K,
                         const Batch& b, int out_kind, void* workspace, size_t workspace_bytes,
                         bitnet_path path, cudaStream_t stream) {
-    if (use_gemv(M, K, path)) {
+    if (use_gemv(M, K, path, workspace, workspace_bytes)) {
         if (!gemv_supported(M, K)) return BITNET_ERR_UNSUPPORTED;
         GemvParams p;
         std::memset(&p, 0, sizeof(p));
