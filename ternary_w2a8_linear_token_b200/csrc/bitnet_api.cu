@@ -127,7 +127,7 @@ bitnet_status run_batch(const uint16_t* x_bf16, const int8_t* q_in, int64_t M, i
     for (int i = 0; i < b.nproj; ++i) {
         const int64_t N = b.proj[i].N;
         if (!encode_tmap_2d_u8(&p.tmap_w[i], b.proj[i].packed, uint64_t(K / 4), uint64_t(N),
-                               uint64_t(K / 4), 64, 128, /*swizzle128=*/false))
+                               uint64_t(K / 4), 64, 128, /*swizzle_bytes=*/64))
             return BITNET_ERR_CUDA;
         p.proj[i].s_w = b.proj[i].s_w;
         p.proj[i].y = b.proj[i].y;
@@ -156,7 +156,7 @@ bitnet_status run_batch(const uint16_t* x_bf16, const int8_t* q_in, int64_t M, i
         }
     }
     if (!encode_tmap_2d_u8(&p.tmap_q, q_ws, uint64_t(K), uint64_t(M), uint64_t(K), 128,
-                           uint32_t(bn), /*swizzle128=*/true))
+                           uint32_t(bn), /*swizzle_bytes=*/128))
         return BITNET_ERR_CUDA;
     // Outputs go out through TMA stores when the rows of y are 16-byte aligned; otherwise
     // the epilogue stores from registers.
@@ -169,7 +169,7 @@ bitnet_status run_batch(const uint16_t* x_bf16, const int8_t* q_in, int64_t M, i
         p.proj[i].tma_store = 0;
         if ((reinterpret_cast<uintptr_t>(b.proj[i].y) & 15) == 0 && (N * elem) % 16 == 0) {
             if (!encode_tmap_2d(&p.tmap_y[i], y_type, b.proj[i].y, N, uint64_t(M), N * elem, 32,
-                                uint32_t(tc_store_cols(bn)), /*swizzle128=*/false))
+                                uint32_t(tc_store_cols(bn)), /*swizzle_bytes=*/0))
                 return BITNET_ERR_CUDA;
             p.proj[i].tma_store = 1;
         }
@@ -234,7 +234,7 @@ int32_t* device_error_word() {
 
 bool encode_tmap_2d(CUtensorMap* map, int dtype, const void* base, uint64_t inner, uint64_t outer,
                     uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer,
-                    bool swizzle128) {
+                    int swizzle_bytes) {
     std::call_once(g_encode_once, [] {
         void* fn = nullptr;
         cudaDriverEntryPointQueryResult q;
@@ -250,7 +250,9 @@ bool encode_tmap_2d(CUtensorMap* map, int dtype, const void* base, uint64_t inne
     const cuuint32_t estride[2] = {1, 1};
     const CUresult r = g_encode(map, static_cast<CUtensorMapDataType>(dtype), 2, const_cast<void*>(base),
                                 dims, strides, box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                                swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                                swizzle_bytes == 128  ? CU_TENSOR_MAP_SWIZZLE_128B
+                                : swizzle_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                                      : CU_TENSOR_MAP_SWIZZLE_NONE,
                                 CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;

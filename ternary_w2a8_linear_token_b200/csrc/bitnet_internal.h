@@ -112,15 +112,16 @@ int tc_num_sms();
 inline int tc_store_cols(int bn) { return bn / 2 < 16 ? bn / 2 : 16; }
 
 // Encodes the TMA descriptors (driver entry point fetched through the runtime).
-// dtype: a CUtensorMapDataType value.
+// dtype: a CUtensorMapDataType value. swizzle_bytes: 0 (none), 64 or 128: the 16-byte chunks
+// of each box row are permuted in shared memory as the hardware swizzle of that span.
 bool encode_tmap_2d(CUtensorMap* map, int dtype, const void* base, uint64_t inner, uint64_t outer,
                     uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer,
-                    bool swizzle128);
+                    int swizzle_bytes);
 inline bool encode_tmap_2d_u8(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer,
                               uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer,
-                              bool swizzle128) {
+                              int swizzle_bytes) {
     return encode_tmap_2d(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, base, inner, outer,
-                          row_stride_bytes, box_inner, box_outer, swizzle128);
+                          row_stride_bytes, box_inner, box_outer, swizzle_bytes);
 }
 
 // Device watchdog word of the current device.

@@ -26,7 +26,8 @@
 //              slots they read and, per tile, to the accumulator (barrier round trips of a
 //              single issuing thread, not the tensor core, set the main-loop cadence on B200,
 //              hence the wide stage and the second issuer);
-//  warp 2      lane 0 loads packed weight tiles (128 rows x 64 bytes) into ring P with TMA;
+//  warp 2      lane 0 loads packed weight tiles (128 rows x 64 bytes, 64-byte swizzle) into
+//              ring P with TMA;
 //  warps 3-10  epilogue, two warps per TMEM lane quarter splitting the columns; they zero
 //              each accumulator as they read it (every MMA accumulates): TMEM ->
 //              registers -> y = acc * (s_w * 1/s_x) -> a per-warp staging tile in shared
@@ -448,9 +449,13 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
             const Unit w = unit_of(u, splits, num_k);
             for (int kt = 0; kt < w.ns; ++kt, rp.next(), ra.next()) {
                 mbar_wait_bounded(&p_full[rp.slot], rp.phase, p.err, kErrWaitTmaFull, abort_flag);
-                const uint8_t* prow = smem + L::kOffP + rp.slot * L::kP + row * (kBK / 4) + half * (kBK / 8);
-                const uint4 pk0 = *reinterpret_cast<const uint4*>(prow);
-                const uint4 pk1 = *reinterpret_cast<const uint4*>(prow + 16);
+                // The packed tile arrives with the 64-byte TMA swizzle: 16-byte chunk c of row r
+                // sits at chunk c ^ ((r >> 1) & 3), so the 32 lanes' reads (one row each) spread
+                // over all banks instead of four rows sharing each bank.
+                const uint8_t* prow = smem + L::kOffP + rp.slot * L::kP + row * (kBK / 4);
+                const int sw = (row >> 1) & 3;
+                const uint4 pk0 = *reinterpret_cast<const uint4*>(prow + (((2 * half) ^ sw) << 4));
+                const uint4 pk1 = *reinterpret_cast<const uint4*>(prow + (((2 * half + 1) ^ sw) << 4));
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&p_empty[rp.slot]);
                 // Codes c in {0, 1, 2} -> int8 t = c - 1. Packed word c holds 16 weights; its
