@@ -30,10 +30,14 @@ constexpr int kThreads = kWarps * 32;
 __device__ __forceinline__ float bf16_lo(uint32_t v) { return __uint_as_float(v << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }
 
-// q = rint(x * s_x). The definition's clamp to [-128, 127] never acts here: s_x = RN(127 / a)
-// with a = max(amax, 1e-5) >= |x|, so |x * s_x| <= 127 (1 + 2^-24)^2 < 127.5 and the rounded
-// value lies in [-127, 127].
-__device__ __forceinline__ int q8(float xv, float s) { return __float2int_rn(__fmul_rn(xv, s)); }
+// q = rint(x * s_x) as the low byte of a binary32. The definition's clamp to [-128, 127]
+// never acts here: s_x = RN(127 / a) with a = max(amax, 1e-5) >= |x|, so |x * s_x| <=
+// 127 (1 + 2^-24)^2 < 127.5. Adding 1.5 * 2^23 to the rounded product lands where the binary32
+// spacing is 1, so the sum is rint(x * s_x) + 1.5 * 2^23 (ties to even) and its low mantissa
+// byte is q in two's complement; both steps are separately rounded (no FMA contraction).
+__device__ __forceinline__ int q8(float xv, float s) {
+    return int(__float_as_uint(__fadd_rn(__fmul_rn(xv, s), 12582912.0f)));
+}
 
 // Low bytes of a, b, c, d -> one word (byte 0 = a).
 __device__ __forceinline__ uint32_t pack4(int a, int b, int c, int d) {

@@ -26,19 +26,29 @@ __device__ __forceinline__ float bf16_bits_to_float(uint32_t b) {
     return __uint_as_float(b << 16);
 }
 
-__device__ __forceinline__ uint32_t quant_pair(uint32_t two_bf16, float s) {
-    const int a = __float2int_rn(__fmul_rn(bf16_bits_to_float(two_bf16 & 0xFFFFu), s));
-    const int b = __float2int_rn(__fmul_rn(bf16_bits_to_float(two_bf16 >> 16), s));
-    const int qa = min(max(a, -128), 127);
-    const int qb = min(max(b, -128), 127);
-    return (static_cast<uint32_t>(qa) & 0xFFu) | ((static_cast<uint32_t>(qb) & 0xFFu) << 8);
+// q = clamp(rint(x * s_x), -128, 127) for one value, as the bits of a binary32 whose low byte
+// is q. The clamp never acts: s_x = RN(127 / a) with a = max(amax, 1e-5) >= |x|, so
+// |x * s_x| <= 127 (1 + 2^-24)^2 < 127.5. Adding 1.5 * 2^23 to the rounded product lands in
+// [2^23, 2^24), where the binary32 spacing is 1, so that sum is rint(x * s_x) + 1.5 * 2^23
+// (round half to even, as cvt.rni) and its low mantissa byte is q in two's complement.
+// Both steps are separately rounded intrinsics, so nothing is contracted into an FMA.
+__device__ __forceinline__ uint32_t qbits(float xv, float s) {
+    return __float_as_uint(__fadd_rn(__fmul_rn(xv, s), 12582912.0f));
 }
 
 // 8 bf16 (one uint4) -> 8 int8 as two 32-bit words (values k..k+3, k+4..k+7).
 __device__ __forceinline__ uint2 quant8(const uint4 v, float s) {
+    const uint32_t b0 = qbits(bf16_bits_to_float(v.x & 0xFFFFu), s);
+    const uint32_t b1 = qbits(__uint_as_float(v.x & 0xFFFF0000u), s);
+    const uint32_t b2 = qbits(bf16_bits_to_float(v.y & 0xFFFFu), s);
+    const uint32_t b3 = qbits(__uint_as_float(v.y & 0xFFFF0000u), s);
+    const uint32_t b4 = qbits(bf16_bits_to_float(v.z & 0xFFFFu), s);
+    const uint32_t b5 = qbits(__uint_as_float(v.z & 0xFFFF0000u), s);
+    const uint32_t b6 = qbits(bf16_bits_to_float(v.w & 0xFFFFu), s);
+    const uint32_t b7 = qbits(__uint_as_float(v.w & 0xFFFF0000u), s);
     uint2 r;
-    r.x = quant_pair(v.x, s) | (quant_pair(v.y, s) << 16);
-    r.y = quant_pair(v.z, s) | (quant_pair(v.w, s) << 16);
+    r.x = __byte_perm(__byte_perm(b0, b1, 0x0040), __byte_perm(b2, b3, 0x0040), 0x5410);
+    r.y = __byte_perm(__byte_perm(b4, b5, 0x0040), __byte_perm(b6, b7, 0x0040), 0x5410);
     return r;
 }
 
