@@ -120,6 +120,7 @@ bitnet_status run_batch(const uint16_t* x_bf16, const int8_t* q_in, int64_t M, i
     int8_t* q_ws = reinterpret_cast<int8_t*>(ws);
     float* s_x = reinterpret_cast<float*>(ws + ws_q_bytes(M, K));
     float* r_x = reinterpret_cast<float*>(ws + ws_q_bytes(M, K) + ws_scale_bytes(M));
+    int32_t* qsum = reinterpret_cast<int32_t*>(ws + ws_q_bytes(M, K) + 2 * ws_scale_bytes(M));
 
     TcParams p;
     std::memset(&p, 0, sizeof(p));
@@ -175,6 +176,7 @@ bitnet_status run_batch(const uint16_t* x_bf16, const int8_t* q_in, int64_t M, i
         }
     }
     p.r_x = r_x;
+    p.qsum = qsum;
     p.err = device_error_word();
     if (!p.err) return BITNET_ERR_CUDA;
     p.K = K;
@@ -213,7 +215,7 @@ bitnet_status run_batch(const uint16_t* x_bf16, const int8_t* q_in, int64_t M, i
 
     cudaError_t e = launch_quant(x_bf16, q_in, M, K, q_ws, q_in ? nullptr : s_x,
                                  q_in ? nullptr : r_x, /*permuted=*/1, stream, /*pdl=*/true, zero,
-                                 zero_bytes);
+                                 zero_bytes, qsum);
     if (e != cudaSuccess) return BITNET_ERR_CUDA;
     return from_cuda(launch_tc_gemm(p, bn, stream, /*pdl=*/true));
 }

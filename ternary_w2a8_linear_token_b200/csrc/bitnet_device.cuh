@@ -259,10 +259,11 @@ __device__ __forceinline__ uint64_t smem_desc_k_sw128(uint32_t saddr) {
     return d;
 }
 
-// Instruction descriptor: kind::i8, A and B signed int8, D int32, both K-major.
-__host__ __device__ constexpr uint32_t idesc_i8(int m, int n) {
+// Instruction descriptor: kind::i8, D int32, both operands K-major; B signed int8, A signed
+// or (a_unsigned) unsigned int8.
+__host__ __device__ constexpr uint32_t idesc_i8(int m, int n, bool a_unsigned = false) {
     return (2u << 4)                                  // D format: s32
-           | (1u << 7)                                // A format: s8
+           | ((a_unsigned ? 0u : 1u) << 7)            // A format: u8 or s8
            | (1u << 10)                               // B format: s8
            | (static_cast<uint32_t>(n >> 3) << 17)    // N / 8
            | (static_cast<uint32_t>(m >> 4) << 24);   // M / 16
@@ -284,9 +285,5 @@ __device__ __forceinline__ uint4 ldg_stream_v4(const void* p) {
     return v;
 }
 
-// Per byte t = code - 1 for four codes in {0, 1, 2} (no borrow between bytes).
-__device__ __forceinline__ uint32_t codes_to_ternary_s8x4(uint32_t codes) {
-    return ((codes | 0x80808080u) - 0x01010101u) ^ 0x80808080u;
-}
 
 }  // namespace bitnet

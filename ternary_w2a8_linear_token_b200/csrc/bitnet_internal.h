@@ -13,13 +13,14 @@ namespace bitnet {
 constexpr int kMaxProj = BITNET_MAX_PROJ;
 
 // ----------------------------------------------------------------------------- workspace
-// Tensor-core path scratch: q (M, K) int8 in the in-group permuted K order, s_x (M) and
-// r_x = 1/s_x (M), each region 256-byte aligned.
+// Tensor-core path scratch: q (M, K) int8 in the in-group permuted K order, s_x (M),
+// r_x = 1/s_x (M) and qsum (M, int32: the sum of each token's q), each region 256-byte
+// aligned.
 inline size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 inline size_t ws_q_bytes(int64_t M, int64_t K) { return align256(size_t(M) * size_t(K)); }
 inline size_t ws_scale_bytes(int64_t M) { return align256(size_t(M) * 4); }
 inline size_t ws_total_bytes(int64_t M, int64_t K) {
-    return ws_q_bytes(M, K) + 2 * ws_scale_bytes(M);
+    return ws_q_bytes(M, K) + 3 * ws_scale_bytes(M);
 }
 
 // Optional split-K area after the base workspace: one int32 arrival counter and one int32
@@ -69,7 +70,7 @@ bool gemv_supported(int64_t M, int64_t K);
 // over its CTAs (the split-K area of the GEMM that follows), or null.
 cudaError_t launch_quant(const uint16_t* x, const int8_t* q_in, int64_t M, int64_t K, int8_t* q,
                          float* s_x, float* r_x, int permuted, cudaStream_t stream, bool pdl,
-                         void* zero = nullptr, int64_t zero_bytes = 0);
+                         void* zero = nullptr, int64_t zero_bytes = 0, int32_t* qsum = nullptr);
 
 // ----------------------------------------------------------------------------- packing
 cudaError_t launch_pack_weights(const float* W, int64_t N, int64_t K, int per_row,
@@ -94,6 +95,7 @@ struct alignas(64) TcParams {
     CUtensorMap tmap_y[kMaxProj];  // outputs (M, N), box {32 rows, tc_store_cols(BN) tokens}
     TcProj proj[kMaxProj];
     const float* r_x;     // (M) 1 / s_x
+    const int32_t* qsum;  // (M) sum over k of q[m, k] (the MMA multiplies codes t + 1)
     int32_t* err;         // watchdog word
     int32_t* split_cnt;   // split-K: arrival counter per tile (zeroed by the quantiser)
     int32_t* split_acc;   // split-K: int32 accumulation tile per tile, [tile][token][row]

@@ -85,7 +85,8 @@ __global__ void __launch_bounds__(kThreads) quant_rows_kernel(const uint16_t* __
                                                               float* __restrict__ r_x,
                                                               int permuted,
                                                               uint4* __restrict__ zero,
-                                                              int64_t zero_words) {
+                                                              int64_t zero_words,
+                                                              int32_t* __restrict__ qsum) {
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const int64_t m = int64_t(blockIdx.x) * kRowsPerCta + warp;
@@ -119,13 +120,19 @@ __global__ void __launch_bounds__(kThreads) quant_rows_kernel(const uint16_t* __
             if (s_x) s_x[m] = s;
             if (r_x) r_x[m] = __frcp_rn(s);
         }
+        int qs = 0;  // this lane's share of sum_k q (padding pieces quantise to 0)
 #pragma unroll
         for (int u = 0; u < kRegPieces; ++u) {
             if (u * 32 >= pieces) break;  // warp-uniform
             const int64_t c = u * 32 + lane;
             const uint2 nat = quant8(v[u], s);
+            qs = __dp4a(int(nat.x), 0x01010101, __dp4a(int(nat.y), 0x01010101, qs));
             const uint2 out = permuted ? permute_group_half(nat, lane & 1) : nat;
             if (c < pieces) reinterpret_cast<uint2*>(qr)[c] = out;
+        }
+        if (qsum) {
+            qs = __reduce_add_sync(0xFFFFFFFFu, qs);
+            if (lane == 0) qsum[m] = qs;
         }
         return;
     }
@@ -149,6 +156,7 @@ __global__ void __launch_bounds__(kThreads) quant_rows_kernel(const uint16_t* __
         }
     }
 
+    int qs = 0;
     for (int64_t c0 = 0; c0 < pieces; c0 += 32 * kUnroll) {
         uint2 nat[kUnroll];
         if (q_in == nullptr) {
@@ -171,9 +179,14 @@ __global__ void __launch_bounds__(kThreads) quant_rows_kernel(const uint16_t* __
 #pragma unroll
         for (int u = 0; u < kUnroll; ++u) {
             const int64_t c = c0 + u * 32 + lane;  // c0 + u*32 is even: lane pairs share a group
+            qs = __dp4a(int(nat[u].x), 0x01010101, __dp4a(int(nat[u].y), 0x01010101, qs));
             const uint2 out = permuted ? permute_group_half(nat[u], lane & 1) : nat[u];
             if (c < pieces) reinterpret_cast<uint2*>(qr)[c] = out;
         }
+    }
+    if (qsum) {
+        qs = __reduce_add_sync(0xFFFFFFFFu, qs);
+        if (lane == 0) qsum[m] = qs;
     }
 }
 
@@ -188,8 +201,9 @@ constexpr int64_t kLongMaxK = int64_t(kLongRowThreads) * kLongPieces * 8;
 __global__ void __launch_bounds__(kLongThreads) quant_long_rows_kernel(
     const uint16_t* __restrict__ x, int64_t M, int64_t K, int8_t* __restrict__ q,
     float* __restrict__ s_x, float* __restrict__ r_x, int permuted, uint4* __restrict__ zero,
-    int64_t zero_words) {
+    int64_t zero_words, int32_t* __restrict__ qsum) {
     __shared__ uint32_t s_mx[kLongRows][kLongRowThreads / 32];
+    __shared__ int32_t s_qs[kLongRows][kLongRowThreads / 32];
     const int row = threadIdx.x / kLongRowThreads;
     const int t = threadIdx.x % kLongRowThreads;
     const int lane = threadIdx.x & 31;
@@ -225,13 +239,26 @@ __global__ void __launch_bounds__(kLongThreads) quant_long_rows_kernel(
         if (r_x) r_x[m] = __frcp_rn(s);
     }
     int8_t* qr = q + (active ? m : 0) * K;
+    int qs = 0;  // padding pieces quantise to 0
 #pragma unroll
     for (int u = 0; u < kLongPieces; ++u) {
         if (int64_t(u) * kLongRowThreads >= pieces) break;  // uniform over the row's warps
         const int64_t c = int64_t(u) * kLongRowThreads + t;  // lane pairs share a 16-group
         const uint2 nat = quant8(v[u], s);
+        qs = __dp4a(int(nat.x), 0x01010101, __dp4a(int(nat.y), 0x01010101, qs));
         const uint2 out = permuted ? permute_group_half(nat, lane & 1) : nat;
         if (active && c < pieces) reinterpret_cast<uint2*>(qr)[c] = out;
+    }
+    if (qsum) {  // uniform over the CTA
+        qs = __reduce_add_sync(0xFFFFFFFFu, qs);
+        if (lane == 0) s_qs[row][t >> 5] = qs;
+        __syncthreads();
+        if (active && t == 0) {
+            int32_t tot = 0;
+#pragma unroll
+            for (int w = 0; w < kLongRowThreads / 32; ++w) tot += s_qs[row][w];
+            qsum[m] = tot;
+        }
     }
 }
 
@@ -239,7 +266,7 @@ __global__ void __launch_bounds__(kLongThreads) quant_long_rows_kernel(
 
 cudaError_t launch_quant(const uint16_t* x, const int8_t* q_in, int64_t M, int64_t K, int8_t* q,
                          float* s_x, float* r_x, int permuted, cudaStream_t stream, bool pdl,
-                         void* zero, int64_t zero_bytes) {
+                         void* zero, int64_t zero_bytes, int32_t* qsum) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>((M + kRowsPerCta - 1) / kRowsPerCta));
     cfg.blockDim = dim3(kThreads);
@@ -254,10 +281,10 @@ cudaError_t launch_quant(const uint16_t* x, const int8_t* q_in, int64_t M, int64
         cfg.gridDim = dim3(static_cast<unsigned>((M + kLongRows - 1) / kLongRows));
         cfg.blockDim = dim3(kLongThreads);
         return cudaLaunchKernelEx(&cfg, quant_long_rows_kernel, x, M, K, q, s_x, r_x, permuted,
-                                  static_cast<uint4*>(zero), zero_bytes / 16);
+                                  static_cast<uint4*>(zero), zero_bytes / 16, qsum);
     }
     return cudaLaunchKernelEx(&cfg, quant_rows_kernel, x, q_in, M, K, q, s_x, r_x, permuted,
-                              static_cast<uint4*>(zero), zero_bytes / 16);
+                              static_cast<uint4*>(zero), zero_bytes / 16, qsum);
 }
 
 }  // namespace bitnet

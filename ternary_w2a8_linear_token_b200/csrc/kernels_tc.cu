@@ -84,8 +84,8 @@ struct TcLayout {
     static constexpr int kOffB = 0;
     static constexpr int kOffP = kOffB + kDB * kB;
     static constexpr int kOffStage = kOffP + kDP * kP;
-    static constexpr int kOffTab = kOffStage + kEpiWarps * kStage;  // BN floats
-    static constexpr int kOffBar = kOffTab + (BN * 4 + 15) / 16 * 16;
+    static constexpr int kOffTab = kOffStage + kEpiWarps * kStage;  // BN floats, then BN int32
+    static constexpr int kOffBar = kOffTab + (2 * BN * 4 + 15) / 16 * 16;
     static constexpr int kNumBars = 2 * (kDA + kDB + kDP) + 4;
     static constexpr int kSmem = kOffBar + kNumBars * 8 + 16 + 1024;  // + slot, flag, align
     // TMEM: two accumulators of BN columns, then the unpacked-weight ring.
@@ -396,7 +396,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
             // offsets (bytes / 16) of the ring slot and the 32-byte K step; the weight operand
             // is read from its TMEM ring slot, 8 columns per K step.
             const int issuer = warp == kWarpMma ? 0 : 1;
-            constexpr uint32_t idesc = idesc_i8(kBM, BN);
+            constexpr uint32_t idesc = idesc_i8(kBM, BN, /*a_unsigned=*/true);
             const uint32_t a_tmem0 = tmem_base + L::kACol0;
             const uint64_t b_desc0 = smem_desc_k_sw128(smem_addr(smem + L::kOffB));
             Ring<L::kDA> ra;
@@ -458,17 +458,18 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
                 const uint4 pk1 = *reinterpret_cast<const uint4*>(prow + (((2 * half + 1) ^ sw) << 4));
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&p_empty[rp.slot]);
-                // Codes c in {0, 1, 2} -> int8 t = c - 1. Packed word c holds 16 weights; its
-                // shifts by 0, 2, 4, 6 give the four 32-bit columns in the permuted in-group
-                // K order of the token operand.
+                // The MMA multiplies the codes c = t + 1 in {0, 1, 2} themselves (unsigned A
+                // operand); the epilogue removes sum_k q once per token (sum q t = sum q c -
+                // sum q). Packed word c holds 16 weights; its shifts by 0, 2, 4, 6 give the
+                // four 32-bit columns in the permuted in-group K order of the token operand.
                 const uint32_t words[8] = {pk0.x, pk0.y, pk0.z, pk0.w, pk1.x, pk1.y, pk1.z, pk1.w};
                 uint32_t t[32];
 #pragma unroll
                 for (int c = 0; c < 8; ++c) {
-                    t[4 * c + 0] = codes_to_ternary_s8x4(words[c] & 0x03030303u);
-                    t[4 * c + 1] = codes_to_ternary_s8x4((words[c] >> 2) & 0x03030303u);
-                    t[4 * c + 2] = codes_to_ternary_s8x4((words[c] >> 4) & 0x03030303u);
-                    t[4 * c + 3] = codes_to_ternary_s8x4((words[c] >> 6) & 0x03030303u);
+                    t[4 * c + 0] = words[c] & 0x03030303u;
+                    t[4 * c + 1] = (words[c] >> 2) & 0x03030303u;
+                    t[4 * c + 2] = (words[c] >> 4) & 0x03030303u;
+                    t[4 * c + 3] = (words[c] >> 6) & 0x03030303u;
                 }
                 mbar_wait_bounded(&a_empty[ra.slot], ra.phase ^ 1, p.err, kErrWaitEmpty, abort_flag);
                 tc_fence_after();
@@ -489,6 +490,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
         volatile int32_t* last_flag = reinterpret_cast<volatile int32_t*>(tmem_slot + 2);
         uint8_t* stage = smem + L::kOffStage + (warp - kEpiWarp0) * L::kStage;
         float* tab = reinterpret_cast<float*>(smem + L::kOffTab);
+        int32_t* qtab = reinterpret_cast<int32_t*>(tab + BN);  // sum_k q of the tile's tokens
         constexpr int kHC = BN / 2 < kHalfCols ? BN / 2 : kHalfCols;  // columns per warp per round
         constexpr int kRounds = BN / (2 * kHC);
         constexpr int kPre = (kRounds * kHC + 31) / 32;
@@ -540,6 +542,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
                         if (!pr.per_row) fv = __fmul_rn(sw, fv);
                     }
                     tab[et] = fv;
+                    qtab[et] = m < p.M ? p.qsum[m] : 0;
                 }
                 epilogue_bar_sync();
                 mbar_wait_bounded(&acc_full[buf], (i >> 1) & 1, p.err, kErrWaitAccum, abort_flag);
@@ -560,6 +563,17 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
                         tc_fence_before();
                         __syncwarp();
                         if (lane == 0) mbar_arrive(&acc_empty[buf]);
+                    }
+                    {  // acc = sum q c - sum q (exact int32)
+                        const int4* q4 = reinterpret_cast<const int4*>(qtab + col0);
+#pragma unroll
+                        for (int c4 = 0; c4 < kHC / 4; ++c4) {
+                            const int4 qq = q4[c4];
+                            v[4 * c4 + 0] = uint32_t(int32_t(v[4 * c4 + 0]) - qq.x);
+                            v[4 * c4 + 1] = uint32_t(int32_t(v[4 * c4 + 1]) - qq.y);
+                            v[4 * c4 + 2] = uint32_t(int32_t(v[4 * c4 + 2]) - qq.z);
+                            v[4 * c4 + 3] = uint32_t(int32_t(v[4 * c4 + 3]) - qq.w);
+                        }
                     }
                     float f[kHC];
                     table_factors<kHC>(tab + col0, pr.per_row != 0, sw, f);
@@ -635,8 +649,11 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
                         const int col0 = r * 2 * kHC + colhalf * kHC;
                         uint32_t v[kHC];
 #pragma unroll
-                        for (int c = 0; c < kHC; ++c)
-                            v[c] = uint32_t(__ldcg(acc + size_t(col0 + c) * kBM + n_local));
+                        for (int c = 0; c < kHC; ++c) {
+                            const int64_t m = int64_t(tc.m0) + col0 + c;
+                            v[c] = uint32_t(__ldcg(acc + size_t(col0 + c) * kBM + n_local) -
+                                            (m < p.M ? p.qsum[m] : 0));
+                        }
                         float rx[kHC];
                         spread_rx<kHC, kPre>(rx_pre, r, rx);
                         float f[kHC];
