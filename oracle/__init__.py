@@ -64,9 +64,10 @@ def _load():
             lib.oracle_round_bf16.restype = None
             lib.oracle_bitlinear_sampled.argtypes = [P, I64, I64, P, P, I, I64, P, I64, P, I64,
                                                      P, P, P, P, P, P, P]
+            lib.oracle_swiglu.argtypes = [P, P, I64, P, P]
             for name in ("oracle_absmean_scale", "oracle_ternarize", "oracle_pack",
                          "oracle_unpack", "oracle_quant_act", "oracle_ternary_matmul",
-                         "oracle_dequant", "oracle_bitlinear_sampled"):
+                         "oracle_dequant", "oracle_bitlinear_sampled", "oracle_swiglu"):
                 getattr(lib, name).restype = ctypes.c_int
             _lib = lib
     return _lib
@@ -205,3 +206,40 @@ def bitlinear_sampled(x_bf16_bits: np.ndarray, packed: np.ndarray, s_w: np.ndarr
                                           _ptr(q), _ptr(sx), _ptr(st), _ptr(sq), _ptr(ssx))
     _check(rc, "bitlinear_sampled")
     return {"y": y, "acc": acc, "q": q, "s_x": sx}
+
+
+def swiglu(g_bits: np.ndarray, u_bits: np.ndarray):
+    """SwiGLU on bf16 g, u ("BitNet 深度实战", §3.2 BitLlamaMLP): s = bf16(silu(g)),
+    h = bf16(s * u). Returns (s_bits, h_bits), uint16 bf16 patterns of g's shape."""
+    g = np.ascontiguousarray(g_bits, dtype=np.uint16)
+    u = np.ascontiguousarray(u_bits, dtype=np.uint16)
+    assert g.shape == u.shape
+    s = np.empty(g.shape, dtype=np.uint16)
+    h = np.empty(g.shape, dtype=np.uint16)
+    _check(_load().oracle_swiglu(_ptr(g), _ptr(u), g.size, _ptr(s), _ptr(h)), "swiglu")
+    return s, h
+
+
+def swiglu_gate_up(x_bf16_bits: np.ndarray, packed_gate: np.ndarray, s_w_gate: np.ndarray,
+                   packed_up: np.ndarray, s_w_up: np.ndarray, per_row: bool, K: int):
+    """The MLP's gate and up BitLinears followed by SwiGLU ("BitNet 深度实战", §3.2):
+    g = bf16(gate(x)), u = bf16(up(x)), h = bf16(bf16(silu(g)) * u). Returns a dict with the
+    exact fp64 g and u, their bf16 bits, and s (silu) and h bits, all (M, I)."""
+    yg = bitlinear(x_bf16_bits, packed_gate, s_w_gate, per_row, K)["y"]
+    yu = bitlinear(x_bf16_bits, packed_up, s_w_up, per_row, K)["y"]
+    g_bits, u_bits = round_bf16(yg), round_bf16(yu)
+    s_bits, h_bits = swiglu(g_bits, u_bits)
+    return {"g": yg, "u": yu, "g_bits": g_bits, "u_bits": u_bits, "s_bits": s_bits,
+            "h_bits": h_bits}
+
+
+def swiglu_gate_up_sampled(x_bf16_bits: np.ndarray, packed_gate: np.ndarray,
+                           s_w_gate: np.ndarray, packed_up: np.ndarray, s_w_up: np.ndarray,
+                           per_row: bool, K: int, m_idx, n_idx):
+    """swiglu_gate_up restricted to tokens m_idx and outputs n_idx (full-size parity)."""
+    yg = bitlinear_sampled(x_bf16_bits, packed_gate, s_w_gate, per_row, K, m_idx, n_idx)["y"]
+    yu = bitlinear_sampled(x_bf16_bits, packed_up, s_w_up, per_row, K, m_idx, n_idx)["y"]
+    g_bits, u_bits = round_bf16(yg), round_bf16(yu)
+    s_bits, h_bits = swiglu(g_bits, u_bits)
+    return {"g": yg, "u": yu, "g_bits": g_bits, "u_bits": u_bits, "s_bits": s_bits,
+            "h_bits": h_bits}

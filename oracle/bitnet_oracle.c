@@ -17,7 +17,8 @@
  *           quantiser (scale = mean |W| along the row, clamped at eps = 1e-5;
  *           t = clamp(round(W / scale), -1, 1)) and its worked example.
  *  [P5-3.2] same page, section 3.2: BitLinear uses the same quantiser and the
- *           float product linear(x, t * scale).
+ *           float product linear(x, t * scale); its BitLlamaMLP feeds the down
+ *           projection silu(gate(x)) * up(x) (SwiGLU).
  *  [P5-4.3] same page, section 4.3 "位打包（Bit Packing）存储": four 2-bit codes
  *           per byte, the first weight in bits 0-1 up to the fourth in bits 6-7.
  *  [P5-4.4] same page, section 4.4 "查找表加速": the int8 x ternary product with
@@ -43,6 +44,9 @@
  *  - Output: y[m,n] = acc[m,n] * s_w / s_x[m], the exact real value, evaluated
  *    in binary64 (error < 2^-52 relative); rounding to bf16 is round-to-nearest-
  *    even of that value.
+ *  - SwiGLU: g and u are the bf16 outputs of the gate and up projections;
+ *    silu(g) is rounded to bf16, then the product with u is rounded to bf16, the
+ *    rounding points of the page's module run in bf16 (each op returns bf16).
  *
  * Return codes: 0 = ok, 1 = bad argument, 2 = invalid data (a weight outside
  * {-1,0,+1}, or a packed code 3).
@@ -285,5 +289,29 @@ int oracle_bitlinear_sampled(const uint16_t* x, int64_t M, int64_t K, const uint
     }
     if (q_out) memcpy(q_out, scratch_q, (size_t)(Ms * K));
     if (sx_out) memcpy(sx_out, scratch_sx, (size_t)Ms * sizeof(float));
+    return ORACLE_OK;
+}
+
+/* ---------------------------------------------------------------------------
+ * SwiGLU of the MLP, [P5-3.2] BitLlamaMLP: the down projection's input is
+ * silu(gate(x)) * up(x), silu(z) = z * sigmoid(z) = z / (1 + e^-z). g and u are
+ * the bf16 outputs of the gate and up BitLinears. As in the page's module, where
+ * each op returns a bf16 tensor, every op rounds its result to bf16:
+ *   s = bf16(silu(g))   evaluated in binary64 with libm exp, rounded once to bf16;
+ *   h = bf16(s * u)     the product of two bf16 values is exact in binary64.
+ * s_out (optional) receives s. All arrays hold bf16 bit patterns.
+ * ------------------------------------------------------------------------- */
+int oracle_swiglu(const uint16_t* g, const uint16_t* u, int64_t count, uint16_t* s_out,
+                  uint16_t* h) {
+    if (!g || !u || !h || count < 0) return ORACLE_BAD_ARG;
+    for (int64_t i = 0; i < count; ++i) {
+        double gv = (double)bf16_to_float(g[i]);
+        double silu = gv / (1.0 + exp(-gv));
+        uint16_t s;
+        oracle_round_bf16(&silu, 1, &s);
+        double prod = (double)bf16_to_float(s) * (double)bf16_to_float(u[i]);
+        oracle_round_bf16(&prod, 1, &h[i]);
+        if (s_out) s_out[i] = s;
+    }
     return ORACLE_OK;
 }

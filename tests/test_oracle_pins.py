@@ -285,3 +285,143 @@ def test_bitlinear_composite_and_sampled(oracle):
     xf = synth.bf16_bits_to_f32(cfg["x"]).astype(np.float64)
     dense = xf @ cfg["W"].astype(np.float64).T
     assert np.corrcoef(dense.ravel(), full["y"].ravel())[0, 1] > 0.8
+
+
+# ---------------------------------------------------------------- SwiGLU (MLP gate/up)
+# Independent exact arithmetic for the pins below: Fractions for rational steps, Decimal
+# at 50 digits for e^-z, and RNE to bf16 by integer scaling (not the oracle's frexp route).
+from decimal import Decimal, getcontext
+from fractions import Fraction
+
+
+def _bf16_value(bits: int) -> Fraction:
+    sign = -1 if bits & 0x8000 else 1
+    e = (bits >> 7) & 0xFF
+    m = bits & 0x7F
+    if e == 0:
+        return sign * Fraction(m, 1 << 133)  # subnormal: m * 2^-133
+    return sign * Fraction(128 + m, 128) * Fraction(2) ** (e - 127)
+
+
+def _rne_bf16(v: Fraction) -> int:
+    """Exact round-half-even of a rational to bf16 bits (finite range only)."""
+    if v == 0:
+        return 0x0000
+    sign = 0x8000 if v < 0 else 0
+    a = abs(v)
+    e = a.numerator.bit_length() - a.denominator.bit_length()  # 2^e <= a < 2^(e+2)
+    while Fraction(2) ** e > a:
+        e -= 1
+    while Fraction(2) ** (e + 1) <= a:
+        e += 1
+    q_exp = max(e, -126) - 7  # quantum: 8 significant bits, or 2^-133 below the normals
+    scaled = a / Fraction(2) ** q_exp
+    n = scaled.numerator // scaled.denominator
+    rem = scaled - n
+    if rem > Fraction(1, 2) or (rem == Fraction(1, 2) and n % 2 == 1):
+        n += 1
+    r = n * Fraction(2) ** q_exp
+    if r == 0:
+        return sign
+    if r >= Fraction(2) ** -126:
+        e2 = r.numerator.bit_length() - r.denominator.bit_length()
+        while Fraction(2) ** e2 > r:
+            e2 -= 1
+        while Fraction(2) ** (e2 + 1) <= r:
+            e2 += 1
+        mant = int(r / Fraction(2) ** (e2 - 7)) - 128
+        assert e2 + 127 < 255, "overflow is outside these pins"
+        return sign | ((e2 + 127) << 7) | mant
+    return sign | int(r * (1 << 133))
+
+
+def _silu_exact_bf16(g_bits: int) -> int:
+    getcontext().prec = 50
+    z = _bf16_value(g_bits)
+    ez = (-Decimal(z.numerator) / Decimal(z.denominator)).exp()
+    silu = z / (1 + Fraction(ez))
+    return _rne_bf16(silu)
+
+
+def test_rne_bf16_helper_matches_torch():
+    """The pins' own rounding helper agrees with torch's fp32 -> bf16 RNE on fp32 values."""
+    vals = np.array([1.0, 1.00390625, 1.005859375, 1.001953125, -3.0e-39, 2.5e-40, 0.1,
+                     -123.456, 65504.0, 1e-30], dtype=np.float32)
+    got = [_rne_bf16(Fraction(float(v))) for v in vals]
+    ref = torch.from_numpy(vals).to(torch.bfloat16).view(torch.int16).numpy().astype(np.uint16)
+    assert got == ref.tolist()
+
+
+def test_swiglu_silu_exact_over_bf16_grid(oracle):
+    """silu rounded to bf16 equals the exactly rounded value (50-digit exp) on a spread of
+    bf16 inputs: every exponent from 2^-20 to 2^7, both signs, several mantissas."""
+    bits = []
+    for e in range(127 - 20, 127 + 7):
+        for m in (0, 1, 37, 64, 100, 127):
+            for sign in (0, 0x8000):
+                bits.append(sign | (e << 7) | m)
+    g = np.array(bits, dtype=np.uint16)
+    u = np.full(g.shape, 0x3F80, dtype=np.uint16)  # u = 1: h = s
+    s, h = oracle.swiglu(g, u)
+    expect = [_silu_exact_bf16(int(b)) for b in bits]
+    assert s.tolist() == expect
+    assert h.tolist() == expect
+
+
+def test_swiglu_closed_forms(oracle):
+    """silu(0) = 0; silu(1) = 1/(1 + 1/e) = 0.7310585786 -> bf16 0.73046875; for z >= 16
+    the relative deficit z e^-z is far below half a bf16 step, so silu(z) rounds to z; for
+    z <= -100 |silu(z)| < 2^-134 (half the least bf16 subnormal) and rounds to -0."""
+    g = np.array([0x0000, 0x3F80, 0x4180, 0x4300, 0x4780, 0xC2C8, 0xC47A], dtype=np.uint16)
+    u = np.full(g.shape, 0x3F80, dtype=np.uint16)
+    s, _ = oracle.swiglu(g, u)
+    assert s[0] == 0x0000
+    assert _bf16_value(int(s[1])) == Fraction(187, 256)  # 0.73046875
+    assert s[2] == 0x4180 and s[3] == 0x4300 and s[4] == 0x4780  # 16, 128, 65536
+    assert s[5] == 0x8000 and s[6] == 0x8000  # -100, -1000
+
+
+def test_swiglu_product_rounding_and_operand_order(oracle):
+    """h = bf16(s * u) with the exact product: u scales h; swapping g and u changes h
+    (silu applies to the gate only); a tie in the product rounds to even."""
+    rng = np.random.default_rng(5)
+    g = synth.to_bf16_bits(rng.normal(0, 3, 400).astype(np.float32))
+    u = synth.to_bf16_bits(rng.normal(0, 3, 400).astype(np.float32))
+    s, h = oracle.swiglu(g, u)
+    for i in range(400):
+        assert int(h[i]) == _rne_bf16(_bf16_value(int(s[i])) * _bf16_value(int(u[i])))
+    _, h_swapped = oracle.swiglu(u, g)
+    assert np.count_nonzero(h_swapped != h) > 300
+    # silu(3.125) = 2.9935 rounds to s = 3 exactly; s * u with u = 1 + 2^-7 is 3.0234375,
+    # nine significant bits with a trailing 1: a tie between 3.015625 (odd last bit) and
+    # 3.03125 (even), so h = 3.03125.
+    _, h1 = oracle.swiglu(np.array([0x4048], dtype=np.uint16), np.array([0x3F81], dtype=np.uint16))
+    assert _bf16_value(int(h1[0])) == Fraction(97, 32)
+
+
+def test_swiglu_gate_up_end_to_end_exact(oracle):
+    """Tiny MLP gate/up: the oracle's h equals an exact rational evaluation of the whole
+    definition (quantiser, integer contraction, y = acc s_w / s_x, bf16 of g and u, silu,
+    product), written here without the oracle's C code."""
+    rng = np.random.default_rng(11)
+    M, I, K = 3, 16, 64
+    x = synth.to_bf16_bits(rng.normal(0, 1, (M, K)).astype(np.float32))
+    tg = rng.integers(-1, 2, (I, K)).astype(np.int8)
+    tu = rng.integers(-1, 2, (I, K)).astype(np.int8)
+    sg = np.array([0.75], dtype=np.float32)
+    su = np.array([1.25], dtype=np.float32)
+    r = oracle.swiglu_gate_up(x, oracle.pack(tg), sg, oracle.pack(tu), su, False, K)
+    xf = synth.bf16_bits_to_f32(x)
+    for m in range(M):
+        amax = float(np.max(np.abs(xf[m])))
+        s_x = np.float32(127.0) / np.float32(max(amax, 1e-5))
+        q = np.rint((xf[m] * s_x).astype(np.float32)).astype(np.int64)
+        for n in range(I):
+            ag = int(np.dot(q, tg[n].astype(np.int64)))
+            au = int(np.dot(q, tu[n].astype(np.int64)))
+            gb = _rne_bf16(Fraction(ag) * Fraction(float(sg[0])) / Fraction(float(s_x)))
+            ub = _rne_bf16(Fraction(au) * Fraction(float(su[0])) / Fraction(float(s_x)))
+            assert int(r["g_bits"][m, n]) == gb and int(r["u_bits"][m, n]) == ub
+            sb = _silu_exact_bf16(gb)
+            assert int(r["s_bits"][m, n]) == sb
+            assert int(r["h_bits"][m, n]) == _rne_bf16(_bf16_value(sb) * _bf16_value(ub))
