@@ -184,6 +184,45 @@ bitnet_status bitnet_linear_i32(const int8_t* q, int64_t M, int64_t K, const uin
                                 bitnet_path path, void* stream);
 
 /*
+ * Fused MLP gate/up projections with SwiGLU ("BitNet 深度实战" section 3.2, BitLlamaMLP:
+ * the down projection's input is silu(gate_proj(x)) * up_proj(x)). Two calls:
+ *
+ * bitnet_interleave_gate_up — offline layout step, like packing. It writes the gate and
+ * up projections of one MLP (each packed (I, K/4) with its scale) as one matrix of 2I rows
+ * in blocks of 16: rows 32b .. 32b+15 are gate rows 16b .. 16b+15 and rows 32b+16 ..
+ * 32b+31 are up rows 16b .. 16b+15. Per-row scales are interleaved the same way (2I
+ * floats); per-tensor scales become {s_gate, s_up} (2 floats). Both projections use `mode`.
+ *   I: intermediate width, a multiple of 16.  K: as for packing (a multiple of 64).
+ *   packed_gu [out] (2I, K/4) uint8, 16-byte aligned.  s_w_gu [out] 2 or 2I floats.
+ *   All pointers device; outputs must not overlap inputs. Asynchronous on `stream`.
+ */
+bitnet_status bitnet_interleave_gate_up(const uint8_t* packed_gate, const float* s_w_gate,
+                                        const uint8_t* packed_up, const float* s_w_up,
+                                        bitnet_scale_mode mode, int64_t I, int64_t K,
+                                        uint8_t* packed_gu, float* s_w_gu, void* stream);
+
+/*
+ * bitnet_linear_swiglu — h = SwiGLU of the gate and up projections of x, with no (M, 2I)
+ * intermediate in memory. Per token m and output j:
+ *   g = bf16 output of gate row j for x (the arithmetic of bitnet_linear, bit for bit);
+ *   u = the same for up row j;
+ *   s = bf16(silu(g)), silu evaluated in binary32: g / (1 + e^-g) for g >= 0 and
+ *       g e^g / (1 + e^g) for g < 0 (expf, IEEE multiply, add and divide);
+ *   h = bf16(s * u) (the product of two bf16 values, exact in binary32 above 2^-126).
+ *   x [in] (M, K) bf16 bits.  packed_gu, s_w_gu [in] from bitnet_interleave_gate_up.
+ *   h [out] (M, I) bf16 bits, 16-byte aligned.
+ *   workspace, workspace_bytes, path: as bitnet_linear_ex (the GEMV path for M <=
+ *   BITNET_GEMV_AUTO_M under BITNET_PATH_AUTO, needing no workspace).
+ * s differs from the exactly rounded silu(g) by at most one bf16 step, and only where the
+ * binary32 value falls within a few binary32 steps of a bf16 rounding boundary.
+ */
+bitnet_status bitnet_linear_swiglu(const uint16_t* x, int64_t M, int64_t K,
+                                   const uint8_t* packed_gu, const float* s_w_gu,
+                                   bitnet_scale_mode mode, int64_t I, uint16_t* h,
+                                   void* workspace, size_t workspace_bytes, bitnet_path path,
+                                   void* stream);
+
+/*
  * bitnet_linear_noalloc — bitnet_linear for callers that cannot allocate device memory.
  * The pages have no counterpart to this call; it exists for callers such as a serving
  * loop in which cudaMalloc could synchronise the device and stall other streams, a plug-in

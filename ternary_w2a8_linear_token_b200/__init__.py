@@ -14,6 +14,8 @@ Functions keep the C names:
     bitnet_linear(x, packed, s_w, per_row, ...) -> y
     bitnet_linear_batch(x, projs, ...)         -> [y, ...]
     bitnet_linear_i32(q, packed, ...)          -> acc (int32)
+    bitnet_interleave_gate_up(pg, sg, pu, su, per_row) -> (packed_gu, s_w_gu)
+    bitnet_linear_swiglu(x, packed_gu, s_w_gu, per_row, ...) -> h (bf16)
     bitnet_check_device_errors()               -> watchdog word (0 = clean)
 """
 from __future__ import annotations
@@ -45,6 +47,7 @@ WATCHDOG_TMA_FULL, WATCHDOG_UNPACK, WATCHDOG_EMPTY, WATCHDOG_ACCUM, WATCHDOG_DRA
     1 << 0, 1 << 1, 1 << 2, 1 << 3, 1 << 4)
 WATCHDOG_SELFTEST = 1 << 6
 MAX_PROJ = 8
+SWIGLU_BLOCK = 16  # interleaved gate/up rows come in blocks of this many
 
 _P, _I64, _I32, _SZ = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_size_t
 
@@ -70,6 +73,10 @@ _SIGS = {
     "bitnet_linear_i32": ([_P, _I64, _I64, _P, _I64, _P, _P, _SZ, ctypes.c_int, _P], ctypes.c_int),
     "bitnet_linear_noalloc": ([_P, _I64, _I64, _P, _P, ctypes.c_int, _I64, _P, ctypes.c_int, _P],
                               ctypes.c_int),
+    "bitnet_interleave_gate_up": ([_P, _P, _P, _P, ctypes.c_int, _I64, _I64, _P, _P, _P],
+                                  ctypes.c_int),
+    "bitnet_linear_swiglu": ([_P, _I64, _I64, _P, _P, ctypes.c_int, _I64, _P, _P, _SZ,
+                             ctypes.c_int, _P], ctypes.c_int),
     "bitnet_check_device_errors": ([ctypes.POINTER(_I32)], ctypes.c_int),
     "bitnet_selftest_wait_timeout": ([_I64, _P], ctypes.c_int),
     "bitnet_status_string": ([ctypes.c_int], ctypes.c_char_p),
@@ -214,6 +221,46 @@ def bitnet_linear_i32(q: torch.Tensor, packed: torch.Tensor, path: int = PATH_AU
                                  _dev(packed, torch.uint8, "packed"), N, acc.data_ptr(), wp, wb,
                                  path, _stream(stream)), "bitnet_linear_i32")
     return acc
+
+
+def bitnet_interleave_gate_up(packed_gate: torch.Tensor, s_w_gate: torch.Tensor,
+                              packed_up: torch.Tensor, s_w_up: torch.Tensor, per_row: bool,
+                              stream=None):
+    """Gate and up projections (each (I, K/4) packed) -> the interleaved (2I, K/4) matrix
+    and its scales (2I per row, or {s_gate, s_up}) that bitnet_linear_swiglu reads."""
+    I, K4 = packed_gate.shape
+    if tuple(packed_up.shape) != (I, K4):
+        raise ValueError("gate and up must have the same shape")
+    dev = packed_gate.device
+    packed_gu = torch.empty((2 * I, K4), dtype=torch.uint8, device=dev)
+    s_w_gu = torch.empty(2 * I if per_row else 2, dtype=torch.float32, device=dev)
+    _check(lib.bitnet_interleave_gate_up(_dev(packed_gate, torch.uint8, "packed_gate"),
+                                         _dev(s_w_gate, torch.float32, "s_w_gate"),
+                                         _dev(packed_up, torch.uint8, "packed_up"),
+                                         _dev(s_w_up, torch.float32, "s_w_up"),
+                                         int(bool(per_row)), I, 4 * K4, packed_gu.data_ptr(),
+                                         s_w_gu.data_ptr(), _stream(stream)),
+           "bitnet_interleave_gate_up")
+    return packed_gu, s_w_gu
+
+
+def bitnet_linear_swiglu(x: torch.Tensor, packed_gu: torch.Tensor, s_w_gu: torch.Tensor,
+                         per_row: bool, h: Optional[torch.Tensor] = None,
+                         workspace: Optional[torch.Tensor] = None, path: int = PATH_AUTO,
+                         stream=None) -> torch.Tensor:
+    """h = bf16(bf16(silu(gate(x))) * up(x)), (M, I), from the interleaved gate/up matrix."""
+    M, K = x.shape
+    I = packed_gu.shape[0] // 2
+    if packed_gu.shape[1] * 4 != K:
+        raise ValueError("packed_gu must be (2I, K/4)")
+    if h is None:
+        h = torch.empty((M, I), dtype=torch.bfloat16, device=x.device)
+    wp, wb, _keep = _ws_args(workspace, M, K, path, x.device)
+    _check(lib.bitnet_linear_swiglu(_x_ptr(x), M, K, _dev(packed_gu, torch.uint8, "packed_gu"),
+                                    _dev(s_w_gu, torch.float32, "s_w_gu"), int(bool(per_row)), I,
+                                    _dev(h, torch.bfloat16, "h"), wp, wb, path, _stream(stream)),
+           "bitnet_linear_swiglu")
+    return h
 
 
 NOALLOC_SCRATCH_BYTES = 16 * 1024 * 1024

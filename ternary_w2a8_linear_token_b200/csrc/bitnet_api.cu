@@ -86,10 +86,11 @@ bool use_gemv(int64_t M, int64_t K, bitnet_path path, const void* ws, size_t ws_
     return !(ws && ws_bytes >= ws_total_bytes(M, K) && aligned(ws, 256));
 }
 
-// Runs a validated batch. x_bf16 or q_in (int8, contraction-only) is the input.
+// Runs a validated batch. x_bf16 or q_in (int8, contraction-only) is the input. swiglu: the
+// batch is one interleaved gate/up matrix of N = 2I rows whose output is h (M, I) bf16.
 bitnet_status run_batch(const uint16_t* x_bf16, const int8_t* q_in, int64_t M, int64_t K,
                         const Batch& b, int out_kind, void* workspace, size_t workspace_bytes,
-                        bitnet_path path, cudaStream_t stream) {
+                        bitnet_path path, cudaStream_t stream, bool swiglu = false) {
     if (use_gemv(M, K, path, workspace, workspace_bytes)) {
         if (!gemv_supported(M, K)) return BITNET_ERR_UNSUPPORTED;
         GemvParams p;
@@ -111,6 +112,11 @@ bitnet_status run_batch(const uint16_t* x_bf16, const int8_t* q_in, int64_t M, i
             rows += b.proj[i].N;
         }
         p.total_rows = rows;
+        if (swiglu) {  // one warp per output pair: I pairs, output width I
+            p.swiglu = 1;
+            p.total_rows = rows / 2;
+            p.proj[0].N = rows / 2;
+        }
         return from_cuda(launch_gemv(p, stream, /*pdl=*/true));
     }
 
@@ -134,6 +140,10 @@ bitnet_status run_batch(const uint16_t* x_bf16, const int8_t* q_in, int64_t M, i
         p.proj[i].y = b.proj[i].y;
         p.proj[i].N = N;
         p.proj[i].per_row = b.proj[i].mode == BITNET_SCALE_PER_ROW;
+        if (swiglu) {  // the factor table holds 1/s_x; each lane applies its row's scale
+            p.proj[i].sw_pair = b.proj[i].mode == BITNET_SCALE_PER_TENSOR;
+            p.proj[i].per_row = 1;
+        }
         p.proj[i].tile_begin = tiles;
         tiles += static_cast<int>((N + 127) / 128);
     }
@@ -165,7 +175,16 @@ bitnet_status run_batch(const uint16_t* x_bf16, const int8_t* q_in, int64_t M, i
     const int y_type = out_kind == 0   ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
                        : out_kind == 1 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
                                        : CU_TENSOR_MAP_DATA_TYPE_INT32;
-    for (int i = 0; i < b.nproj; ++i) {
+    if (swiglu) {  // h (M, I) bf16 through TMA stores of 16 outputs x tc_store_cols tokens
+        const uint64_t I = uint64_t(b.proj[0].N) / 2;
+        if (!encode_tmap_2d(&p.tmap_y[0], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, b.proj[0].y, I,
+                            uint64_t(M), I * 2, kSwigluBlock, uint32_t(tc_store_cols(bn)),
+                            /*swizzle_bytes=*/0))
+            return BITNET_ERR_CUDA;
+        p.proj[0].tma_store = 1;
+        p.swiglu = 1;
+    }
+    for (int i = 0; i < b.nproj && !swiglu; ++i) {
         const uint64_t N = uint64_t(b.proj[i].N);
         p.proj[i].tma_store = 0;
         if ((reinterpret_cast<uintptr_t>(b.proj[i].y) & 15) == 0 && (N * elem) % 16 == 0) {
@@ -197,7 +216,7 @@ bitnet_status run_batch(const uint16_t* x_bf16, const int8_t* q_in, int64_t M, i
     // Measured on B200: splitting pays for token tiles of up to 32, and of 64 with long K
     // loops; for wider tiles the atomic reduction of the partial tiles costs more than the
     // shorter main loop saves.
-    const bool split_pays = bn <= 32 || (bn == 64 && num_k >= 16);
+    const bool split_pays = !swiglu && (bn <= 32 || (bn == 64 && num_k >= 16));
     if (split_pays && tiles_all * 4 <= sms && tiles_all <= kMaxSplitTiles && num_k >= 4 &&
         workspace_bytes >= ws_total_bytes(M, K) + ws_split_bytes(M)) {
         int64_t sp = sms / tiles_all;
@@ -365,6 +384,72 @@ bitnet_status bitnet_linear_i32(const int8_t* q, int64_t M, int64_t K, const uin
     if (st != BITNET_OK) return st;
     return run_batch(nullptr, q, M, K, b, 2, workspace, workspace_bytes, path,
                      static_cast<cudaStream_t>(stream));
+}
+
+bitnet_status bitnet_interleave_gate_up(const uint8_t* packed_gate, const float* s_w_gate,
+                                        const uint8_t* packed_up, const float* s_w_up,
+                                        bitnet_scale_mode mode, int64_t I, int64_t K,
+                                        uint8_t* packed_gu, float* s_w_gu, void* stream) {
+    if (!packed_gate || !s_w_gate || !packed_up || !s_w_up || !packed_gu || !s_w_gu)
+        return BITNET_ERR_NULL;
+    bitnet_status st = check_mk(1, K);
+    if (st != BITNET_OK) return st;
+    if ((st = check_n(I)) != BITNET_OK) return st;
+    if (I % kSwigluBlock != 0) return BITNET_ERR_SHAPE;
+    if (mode != BITNET_SCALE_PER_TENSOR && mode != BITNET_SCALE_PER_ROW) return BITNET_ERR_UNSUPPORTED;
+    if (!aligned(packed_gate, 16) || !aligned(packed_up, 16) || !aligned(packed_gu, 16) ||
+        !aligned(s_w_gate, 4) || !aligned(s_w_up, 4) || !aligned(s_w_gu, 4))
+        return BITNET_ERR_ALIGN;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    // Blocks of 16 rows: gate block b -> rows 32b.., up block b -> rows 32b + 16.. (one 2D
+    // copy per matrix, a "row" of the copy being one block).
+    const size_t row = size_t(K / 4);
+    const size_t blk = row * kSwigluBlock;
+    const size_t nblk = size_t(I / kSwigluBlock);
+    cudaError_t e = cudaMemcpy2DAsync(packed_gu, 2 * blk, packed_gate, blk, blk, nblk,
+                                      cudaMemcpyDeviceToDevice, s);
+    if (e == cudaSuccess)
+        e = cudaMemcpy2DAsync(packed_gu + blk, 2 * blk, packed_up, blk, blk, nblk,
+                              cudaMemcpyDeviceToDevice, s);
+    if (e == cudaSuccess) {
+        if (mode == BITNET_SCALE_PER_ROW) {
+            const size_t sblk = sizeof(float) * kSwigluBlock;
+            e = cudaMemcpy2DAsync(s_w_gu, 2 * sblk, s_w_gate, sblk, sblk, nblk,
+                                  cudaMemcpyDeviceToDevice, s);
+            if (e == cudaSuccess)
+                e = cudaMemcpy2DAsync(s_w_gu + kSwigluBlock, 2 * sblk, s_w_up, sblk, sblk, nblk,
+                                      cudaMemcpyDeviceToDevice, s);
+        } else {
+            e = cudaMemcpyAsync(s_w_gu, s_w_gate, sizeof(float), cudaMemcpyDeviceToDevice, s);
+            if (e == cudaSuccess)
+                e = cudaMemcpyAsync(s_w_gu + 1, s_w_up, sizeof(float), cudaMemcpyDeviceToDevice, s);
+        }
+    }
+    return from_cuda(e);
+}
+
+bitnet_status bitnet_linear_swiglu(const uint16_t* x, int64_t M, int64_t K,
+                                   const uint8_t* packed_gu, const float* s_w_gu,
+                                   bitnet_scale_mode mode, int64_t I, uint16_t* h,
+                                   void* workspace, size_t workspace_bytes, bitnet_path path,
+                                   void* stream) {
+    if (path != BITNET_PATH_AUTO && path != BITNET_PATH_GEMV && path != BITNET_PATH_TC)
+        return BITNET_ERR_UNSUPPORTED;
+    if (!h) return BITNET_ERR_NULL;
+    bitnet_status st = check_n(I);
+    if (st != BITNET_OK) return st;
+    if (I % kSwigluBlock != 0 || 2 * I >= (int64_t(1) << 31)) return BITNET_ERR_SHAPE;
+    bitnet_proj pr;
+    pr.packed = packed_gu;
+    pr.s_w = s_w_gu;
+    pr.mode = int32_t(mode);
+    pr.reserved = 0;
+    pr.N = 2 * I;
+    pr.y = h;
+    Batch b;
+    if ((st = validate_batch(x, M, K, &pr, 1, /*out_kind=*/0, &b)) != BITNET_OK) return st;
+    return run_batch(x, nullptr, M, K, b, 0, workspace, workspace_bytes, path,
+                     static_cast<cudaStream_t>(stream), /*swiglu=*/true);
 }
 
 bitnet_status bitnet_check_device_errors(int32_t* flags) {

@@ -23,6 +23,9 @@ inline size_t ws_total_bytes(int64_t M, int64_t K) {
     return ws_q_bytes(M, K) + 3 * ws_scale_bytes(M);
 }
 
+// SwiGLU of the MLP: interleaved gate/up weight rows come in blocks of this many rows.
+constexpr int kSwigluBlock = 16;
+
 // Optional split-K area after the base workspace: one int32 arrival counter and one int32
 // accumulation tile (128 weight rows x BN tokens) per split tile; the quantiser zeroes the
 // area on every call. Split-K runs only when the caller's workspace holds it.
@@ -57,6 +60,9 @@ struct GemvParams {
     int32_t nproj;
     int32_t out_kind;  // 0 bf16, 1 f32, 2 int32 accumulator
     int32_t stage_x;   // set by the launcher: stage x in shared memory
+    int32_t swiglu;    // 1: proj[0] is an interleaved gate/up matrix, total_rows counts
+                       // output pairs, y = SwiGLU (bf16, (M, proj[0].N))
+    int32_t pad;
     GemvProj proj[kMaxProj];
 };
 
@@ -86,7 +92,7 @@ struct TcProj {
     int32_t per_row;
     int32_t tile_begin;  // first n-tile index of this projection in the flattened grid
     int32_t tma_store;   // 1: tmap_y is valid and the epilogue stores through it
-    int32_t pad;
+    int32_t sw_pair;     // SwiGLU with per-tensor scales: s_w = {s_gate, s_up}
 };
 
 struct alignas(64) TcParams {
@@ -100,7 +106,7 @@ struct alignas(64) TcParams {
     int32_t* split_cnt;   // split-K: arrival counter per tile (zeroed by the quantiser)
     int32_t* split_acc;   // split-K: int32 accumulation tile per tile, [tile][token][row]
     int32_t splits;       // K splits per tile (1 = none)
-    int32_t pad2;
+    int32_t swiglu;       // 1: interleaved gate/up rows, outputs h = SwiGLU (bf16, M x N/2)
     int64_t K;
     int32_t M;
     int32_t nproj;

@@ -19,6 +19,7 @@
 
 #include "bitnet_device.cuh"
 #include "bitnet_internal.h"
+#include "swiglu_device.cuh"
 
 namespace bitnet {
 namespace {
@@ -63,8 +64,11 @@ __device__ __forceinline__ uint2 permute_group_half(uint2 nat, int h) {
 
 // MT: token capacity (compile time); p.M <= MT tokens are real, the rest are zero.
 // CPL: 16-byte chunks per lane (K <= CPL * 32 * 64). RW: weight rows per warp.
-template <int MT, int CPL, int RW>
+// SW: SwiGLU of an interleaved gate/up matrix; each warp takes one output pair, the gate
+// row and the up row of output j (RW = 2), and writes h = SwiGLU(g, u).
+template <int MT, int CPL, int RW, bool SW>
 __global__ void __launch_bounds__(kThreads, MT <= 2 ? 2 : 1) gemv_w2a8_kernel(const __grid_constant__ GemvParams p) {
+    static_assert(!SW || RW == 2, "a SwiGLU warp holds one gate row and one up row");
     extern __shared__ uint4 s_q[];  // [MT][4][C] permuted q: word i of group 4c + j
     __shared__ uint32_t s_red[kWarps][MT];  // per-warp amax bits
     __shared__ int32_t s_qsum[kWarps][MT];  // per-warp partial sums of q
@@ -84,12 +88,19 @@ __global__ void __launch_bounds__(kThreads, MT <= 2 ? 2 : 1) gemv_w2a8_kernel(co
     float sw[RW];
 #pragma unroll
     for (int r = 0; r < RW; ++r) {
-        gr[r] = (int64_t(blockIdx.x) * kWarps + warp) * RW + r;
-        rvalid[r] = gr[r] < p.total_rows;
         pj[r] = 0;
+        if constexpr (SW) {
+            // output pair j: gate row 32 (j / 16) + j % 16, up row 16 further
+            const int64_t j = int64_t(blockIdx.x) * kWarps + warp;
+            gr[r] = (j / kSwigluBlock) * (2 * kSwigluBlock) + j % kSwigluBlock + r * kSwigluBlock;
+            rvalid[r] = j < p.total_rows;
+        } else {
+            gr[r] = (int64_t(blockIdx.x) * kWarps + warp) * RW + r;
+            rvalid[r] = gr[r] < p.total_rows;
 #pragma unroll
-        for (int jj = 1; jj < kMaxProj; ++jj)
-            if (jj < p.nproj && gr[r] >= p.proj[jj].row_begin) pj[r] = jj;
+            for (int jj = 1; jj < kMaxProj; ++jj)
+                if (jj < p.nproj && gr[r] >= p.proj[jj].row_begin) pj[r] = jj;
+        }
         nrow[r] = gr[r] - p.proj[pj[r]].row_begin;
         const uint8_t* rowp = p.proj[pj[r]].packed + nrow[r] * (K >> 2);
 #pragma unroll
@@ -99,8 +110,9 @@ __global__ void __launch_bounds__(kThreads, MT <= 2 ? 2 : 1) gemv_w2a8_kernel(co
                                                : make_uint4(0u, 0u, 0u, 0u);
         }
         sw[r] = 0.0f;
-        if (rvalid[r] && p.out_kind != 2)
-            sw[r] = p.proj[pj[r]].per_row ? p.proj[pj[r]].s_w[nrow[r]] : p.proj[pj[r]].s_w[0];
+        if (rvalid[r] && p.out_kind != 2)  // per-tensor SwiGLU scales are {s_gate, s_up}
+            sw[r] = p.proj[pj[r]].per_row ? p.proj[pj[r]].s_w[nrow[r]]
+                                          : p.proj[pj[r]].s_w[SW ? r : 0];
     }
 
     pdl_trigger();
@@ -249,6 +261,23 @@ __global__ void __launch_bounds__(kThreads, MT <= 2 ? 2 : 1) gemv_w2a8_kernel(co
         for (int ww = 0; ww < kWarps; ++ww) t += s_qsum[ww][m];
         qs_tot[m] = t;
     }
+    if constexpr (SW) {
+        // g and u of this warp's output pair for every token; lane m writes token m's h.
+        const int64_t j = int64_t(blockIdx.x) * kWarps + warp;
+#pragma unroll
+        for (int m = 0; m < MT; ++m) {
+            const int32_t tg = __reduce_add_sync(0xFFFFFFFFu, acc[0][m][0] + acc[0][m][1]);
+            const int32_t tu = __reduce_add_sync(0xFFFFFFFFu, acc[1][m][0] + acc[1][m][1]);
+            if (lane == m && rvalid[0] && m < Mreal) {
+                const float rx = __frcp_rn(s_tok[m]);
+                const float g = __fmul_rn(__int2float_rn(tg - qs_tot[m]), __fmul_rn(sw[0], rx));
+                const float u = __fmul_rn(__int2float_rn(tu - qs_tot[m]), __fmul_rn(sw[1], rx));
+                static_cast<uint16_t*>(p.proj[0].y)[int64_t(m) * p.proj[0].N + j] =
+                    swiglu_bf16_bits(g, u);
+            }
+        }
+        return;
+    }
 #pragma unroll
     for (int r = 0; r < RW; ++r) {
 #pragma unroll
@@ -286,19 +315,22 @@ int num_sms() {
     return cached[dev];
 }
 
-template <int MT, int CPL, int RW>
+template <int MT, int CPL, int RW, bool SW = false>
 cudaError_t launch_one(const GemvParams& p, cudaStream_t stream, bool pdl) {
     // q (MT*K bytes) plus, when it fits, the staged bf16 activations (2*MT*K bytes)
     GemvParams q = p;
     q.stage_x = (p.q_in == nullptr && 3 * int64_t(MT) * p.K <= 96 * 1024) ? 1 : 0;
     const size_t smem = size_t(MT) * size_t(p.K) * (q.stage_x ? 3 : 1);
-    auto kern = gemv_w2a8_kernel<MT, CPL, RW>;
-    if (smem > 48 * 1024) {
+    auto kern = gemv_w2a8_kernel<MT, CPL, RW, SW>;
+    // Above 48 KB in total (dynamic plus the kernel's static reduction arrays) a launch needs
+    // the opt-in attribute.
+    const size_t static_smem = sizeof(uint32_t) * kWarps * MT + sizeof(int32_t) * kWarps * MT;
+    if (smem + static_smem > 48 * 1024) {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              static_cast<int>(smem));
         if (e != cudaSuccess) return e;
     }
-    const int64_t rows_per_cta = int64_t(kWarps) * RW;
+    const int64_t rows_per_cta = SW ? int64_t(kWarps) : int64_t(kWarps) * RW;  // SW: pairs
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>((p.total_rows + rows_per_cta - 1) / rows_per_cta));
     cfg.blockDim = dim3(kThreads);
@@ -323,6 +355,7 @@ cudaError_t launch_one(const GemvParams& p, cudaStream_t stream, bool pdl) {
 template <int MT, int CPL>
 cudaError_t launch_cpl(const GemvParams& p, cudaStream_t stream, bool pdl) {
     const int64_t slots = int64_t(num_sms()) * kWarps;  // warps of one CTA per SM
+    if (p.swiglu) return launch_one<MT, CPL, 2, true>(p, stream, pdl);  // one pair per warp
     if constexpr (MT <= 2) {
         if constexpr (CPL <= 2) {
             if (p.total_rows > slots) return launch_one<MT, CPL, 2>(p, stream, pdl);

@@ -50,6 +50,7 @@
 
 #include "bitnet_device.cuh"
 #include "bitnet_internal.h"
+#include "swiglu_device.cuh"
 
 namespace bitnet {
 namespace {
@@ -526,8 +527,10 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
             const TcProj& pr = p.proj[tc.proj];
             const int64_t n = int64_t(tc.n0) + n_local;
             const bool nvalid = n < pr.N;
-            // s_w is absent (nullptr) when the raw int32 accumulator is the output.
+            // s_w is absent (nullptr) when the raw int32 accumulator is the output. SwiGLU
+            // with per-tensor scales: lanes 0-15 hold gate rows (s_gate), 16-31 up rows (s_up).
             const float sw = p.out_kind == 2 ? 0.0f
+                             : pr.sw_pair   ? pr.s_w[(lane >> 4) & 1]
                              : pr.per_row   ? (nvalid ? pr.s_w[n] : 0.0f)
                                             : pr.s_w[0];
             const int buf = i & 1;
@@ -577,7 +580,34 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
                     }
                     float f[kHC];
                     table_factors<kHC>(tab + col0, pr.per_row != 0, sw, f);
-                    if (staged) {
+                    if (p.swiglu) {
+                        // Interleaved gate/up rows: lane l < 16 holds gate row j, lane l + 16
+                        // the up row of the same output j = n0 / 2 + 16 quarter + l. Both
+                        // dequantise as in the plain epilogue; the up value moves down 16
+                        // lanes and the gate lanes write h = SwiGLU(g, u), 16 outputs per token.
+#pragma unroll
+                        for (int c = 0; c < kHC; ++c) {
+                            const float yv = __fmul_rn(__int2float_rn(int32_t(v[c])), f[c]);
+                            const float up = __shfl_down_sync(0xFFFFFFFFu, yv, 16);
+                            v[c] = swiglu_bf16_bits(yv, up);
+                        }
+                        uint8_t* sb = stage + (staged_stores & 1u) * 1024u;
+                        if (lane == 0) bulk_wait_group_read<1>();
+                        __syncwarp();
+                        if (lane < kSwigluBlock) {
+                            uint16_t* b = reinterpret_cast<uint16_t*>(sb) + lane;
+#pragma unroll
+                            for (int c = 0; c < kHC; ++c) b[c * kSwigluBlock] = uint16_t(v[c]);
+                        }
+                        fence_proxy_async_smem();
+                        __syncwarp();
+                        const int x = (tc.n0 >> 1) + quarter * kSwigluBlock, y = tc.m0 + col0;
+                        if (lane == 0 && x < (pr.N >> 1) && y < p.M) {
+                            tma_store_2d(&p.tmap_y[tc.proj], sb, x, y);
+                            bulk_commit_group();
+                        }
+                        ++staged_stores;
+                    } else if (staged) {
                         // 2-byte outputs alternate between the two 1 KB halves of the staging
                         // tile; 4-byte outputs use all 2 KB, so the previous store must have
                         // read it out first.

@@ -131,3 +131,31 @@ def test_other_calls_argument_errors(bn):
     assert L.bitnet_linear_i32(FAKE, 16, 64, FAKE, 16, FAKE, FAKE, 1 << 30, 9, None) == \
         bn.ERR_UNSUPPORTED
     assert L.bitnet_check_device_errors(None) == bn.ERR_NULL
+
+
+def test_swiglu_calls_argument_errors(bn):
+    """bitnet_interleave_gate_up and bitnet_linear_swiglu check shapes, pointers, alignment,
+    mode and path before touching the device."""
+    L = bn.lib
+
+    def il(pg=FAKE, sg=FAKE, pu=FAKE, su=FAKE, mode=0, I=64, K=512, out=FAKE, sout=FAKE):
+        return L.bitnet_interleave_gate_up(pg, sg, pu, su, mode, I, K, out, sout, None)
+
+    assert il(pg=None) == bn.ERR_NULL and il(sout=None) == bn.ERR_NULL
+    assert il(I=40) == bn.ERR_SHAPE          # I not a multiple of the 16-row block
+    assert il(I=0) == bn.ERR_SHAPE and il(K=6) == bn.ERR_SHAPE
+    assert il(K=96) == bn.ERR_UNSUPPORTED    # K % 64
+    assert il(mode=2) == bn.ERR_UNSUPPORTED
+    assert il(out=FAKE + 8) == bn.ERR_ALIGN and il(sg=FAKE + 2) == bn.ERR_ALIGN
+
+    def sw(x=FAKE, M=4, K=512, pgu=FAKE, s=FAKE, mode=0, I=64, h=FAKE, ws=None, wb=0, path=0):
+        return L.bitnet_linear_swiglu(x, M, K, pgu, s, mode, I, h, ws, wb, path, None)
+
+    assert sw(h=None) == bn.ERR_NULL and sw(x=None) == bn.ERR_NULL and sw(s=None) == bn.ERR_NULL
+    assert sw(I=24) == bn.ERR_SHAPE and sw(I=0) == bn.ERR_SHAPE and sw(M=0) == bn.ERR_SHAPE
+    assert sw(K=96) == bn.ERR_UNSUPPORTED and sw(mode=5) == bn.ERR_UNSUPPORTED
+    assert sw(path=7) == bn.ERR_UNSUPPORTED
+    assert sw(h=FAKE + 2) == bn.ERR_ALIGN and sw(pgu=FAKE + 4) == bn.ERR_ALIGN
+    # the tensor-core path needs the workspace
+    assert sw(M=300, path=bn.PATH_TC) == bn.ERR_WORKSPACE
+    assert sw(M=300, ws=FAKE, wb=16, path=bn.PATH_TC) == bn.ERR_WORKSPACE

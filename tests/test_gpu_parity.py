@@ -178,6 +178,7 @@ LINEAR_CASES = [  # (M, N, K, per_row)
     (31, 640, 2560, False), (64, 300, 512, True), (100, 256, 1024, False),
     (129, 131, 640, True), (300, 256, 512, False), (200, 640, 1024, True),
     (40, 300, 4096, True),  # split-K, ragged tokens and rows
+    (4, 200, 4096, False), (8, 100, 2048, True),  # GEMV shared memory at exactly 48 KB dynamic
 ]
 
 

@@ -425,3 +425,21 @@ def test_swiglu_gate_up_end_to_end_exact(oracle):
             sb = _silu_exact_bf16(gb)
             assert int(r["s_bits"][m, n]) == sb
             assert int(r["h_bits"][m, n]) == _rne_bf16(_bf16_value(sb) * _bf16_value(ub))
+
+
+def test_swiglu_bound_helper_accepts_exact_and_rejects_far(oracle):
+    """The GPU tests' SwiGLU bound: the oracle's own h passes; h moved 3 bf16 steps away
+    from a value whose neighbourhood is flat fails."""
+    from util import assert_swiglu_within_bound, bf16_from_ordered, bf16_ordered
+    rng = np.random.default_rng(3)
+    y_g = rng.normal(0, 4, (4, 64))
+    y_u = rng.normal(0, 4, (4, 64))
+    g_bits, u_bits = oracle.round_bf16(y_g), oracle.round_bf16(y_u)
+    s_bits, h_bits = oracle.swiglu(g_bits, u_bits)
+    ref = {"g": y_g, "u": y_u, "g_bits": g_bits, "u_bits": u_bits, "s_bits": s_bits,
+           "h_bits": h_bits}
+    assert_swiglu_within_bound(h_bits, ref, oracle)
+    bad = h_bits.copy()
+    bad[1, 5] = bf16_from_ordered(bf16_ordered(bad[1:2, 5:6]) + 40)[0, 0]
+    with pytest.raises(AssertionError):
+        assert_swiglu_within_bound(bad, ref, oracle)
