@@ -231,6 +231,82 @@ def run_stack(bn, torch, dev, name, stack, M, steps, warmup, flush, world, peaks
             else "tensor", "launches_per_pass": launches}, launches
 
 
+MLP_SPECS = {
+    # name: (layers, hidden, ffn, token counts M, per_row scales)
+    "2B-4T MLP gate/up": (30, 2560, 6912, (1, 64, 2048), False),
+    "8B-class MLP gate/up": (32, 4096, 14336, (1, 4096), True),
+}
+
+
+def build_mlp(bn, torch, dev, name):
+    """Per layer: the gate and up projections packed separately (for the unfused arm) and
+    interleaved (bitnet_interleave_gate_up, for the fused call). Layer 0 follows the stack
+    recipe and is copied into every layer's own buffers, as in build_stack."""
+    layers = MLP_SPECS[name][0]
+    if name.startswith("2B"):
+        d = synth.stack2b_layer(0)
+        pg, sg, pu, su, per_row = (bn.bitnet_pack_ternary(torch.from_numpy(d["gate"]["t"]).to(dev)),
+                                   torch.from_numpy(d["gate"]["s_w"]).to(dev),
+                                   bn.bitnet_pack_ternary(torch.from_numpy(d["up"]["t"]).to(dev)),
+                                   torch.from_numpy(d["up"]["s_w"]).to(dev), False)
+    else:
+        Wg = torch.from_numpy(synth.stack8b_latent(0, "gate")).to(dev)
+        Wu = torch.from_numpy(synth.stack8b_latent(0, "up")).to(dev)
+        (pg, sg), (pu, su), per_row = bn.bitnet_pack_weights(Wg, True), \
+            bn.bitnet_pack_weights(Wu, True), True
+        del Wg, Wu
+    pgu, sgu = bn.bitnet_interleave_gate_up(pg, sg, pu, su, per_row)
+    torch.cuda.synchronize()
+    base = {"gate": (pg, sg, per_row), "up": (pu, su, per_row), "gu": (pgu, sgu, per_row)}
+    return [base] + [{k: (a.clone(), b.clone(), r) for k, (a, b, r) in base.items()}
+                     for _ in range(layers - 1)]
+
+
+def run_mlp(bn, torch, dev, name, layers_w, M, steps, warmup, flush, world, peaks):
+    """One pass = the gate/up + SwiGLU of every layer back to back, fused
+    (bitnet_linear_swiglu) and unfused (bitnet_linear_batch of gate and up, then the
+    elementwise silu(g) * u in PyTorch, for comparison). Returns the line object."""
+    layers, hidden, ffn, _, per_row = MLP_SPECS[name]
+    gen = synth.stack2b_x if name.startswith("2B") else synth.stack8b_x
+    x = torch.from_numpy(gen(M, hidden, which=2).view(np.int16).copy()).to(dev).view(torch.bfloat16)
+    h = torch.empty((M, ffn), dtype=torch.bfloat16, device=dev)
+    g = torch.empty((M, ffn), dtype=torch.bfloat16, device=dev)
+    u = torch.empty((M, ffn), dtype=torch.bfloat16, device=dev)
+    tc = M > bn.GEMV_AUTO_M
+    ws = bn.make_workspace(M, hidden, dev) if tc else None
+
+    def fused():
+        for L in layers_w:
+            bn.bitnet_linear_swiglu(x, *L["gu"], h=h, workspace=ws)
+
+    def unfused():
+        for L in layers_w:
+            bn.bitnet_linear_batch(x, [L["gate"], L["up"]], ys=[g, u], workspace=ws)
+            torch.mul(torch.nn.functional.silu(g), u, out=h)
+
+    res = {}
+    for arm, fn in (("fused", fused), ("unfused", unfused)):
+        gr = capture(torch, fn)
+        ms = timed_steps(torch, gr.replay, steps, warmup, flush, world)
+        ms_max, _ = reduce_over_ranks(ms, 0.0, world)
+        res[arm] = ms_max * 1e-3 / steps
+        del gr
+    assert bn.bitnet_check_device_errors() == 0
+    w_bytes = layers * (2 * ffn * hidden // 4 + 4 * (2 * ffn if per_row else 2))
+    act_bytes = layers * (2 * M * hidden + 2 * M * ffn)
+    ops = layers * 2.0 * M * (2 * ffn) * hidden
+    int8_peak = peaks["bf16_tflops"] * INT8_PER_BF16
+    roof = max((w_bytes + act_bytes) / (peaks["hbm_gbs"] * 1e9), ops / (int8_peak * 1e12))
+    t = res["fused"]
+    launches = layers * (2 if tc else 1)
+    return {"mlp": name, "M": M, "us_per_layer": t / layers * 1e6,
+            "unfused_us_per_layer": res["unfused"] / layers * 1e6,
+            "speedup_vs_unfused": res["unfused"] / t, "GB_per_s": (w_bytes + act_bytes) / t / 1e9,
+            "TOPS": ops / t / 1e12, "roofline_us_per_layer": roof / layers * 1e6, "frac": roof / t,
+            "bound": "hbm" if (w_bytes + act_bytes) / (peaks["hbm_gbs"] * 1e9) >= ops / (int8_peak * 1e12)
+            else "tensor"}, launches * steps + layers * (2 if tc else 1) * steps
+
+
 def run_calls(bn, calls):
     for c in calls:
         bn.bitnet_linear(c["x"], c["packed"], c["s_w"], False, y=c["y"], workspace=c.get("ws"))
@@ -435,6 +511,19 @@ def run_ours(args):
             del st
             torch.cuda.empty_cache()
 
+    # ---------------- fused MLP gate/up + SwiGLU against the unfused sequence
+    mlp = []
+    if args.stacks == "all" and args.only == "all":
+        for name, spec in MLP_SPECS.items():
+            lw = build_mlp(bn, torch, dev, name)
+            for M in spec[3]:
+                r, nl = run_mlp(bn, torch, dev, name, lw, M, min(args.steps, 5), args.warmup,
+                                flush, world, peaks)
+                mlp.append(r)
+                stack_launches += nl
+            del lw
+            torch.cuda.empty_cache()
+
     cpu = oracle_sample(args.cpu_seconds) if (rank == 0 and world == 1 and args.cpu_seconds > 0) \
         else None
 
@@ -467,6 +556,7 @@ def run_ours(args):
             "clocks": clk.summary(),
             "gemm": gemm,
             "stacks": stacks,
+            "mlp": mlp,
             "cpu_baseline": cpu,
         }
         print(json.dumps(line), flush=True)
@@ -491,7 +581,8 @@ def main():
     ap.add_argument("--prefill-m", type=int, default=PREFILL_M,
                     help="tokens of the prefill GEMM part")
     ap.add_argument("--stacks", choices=["all", "none"], default="all",
-                    help="time the 2B-4T and 8B-class layer stacks (extra objects on the line)")
+                    help="time the 2B-4T and 8B-class layer stacks and MLP gate/up + SwiGLU "
+                         "(extra objects on the line)")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)  # at least 3 untimed warm-up steps
     if args.impl == "reference":

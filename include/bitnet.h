@@ -206,8 +206,8 @@ bitnet_status bitnet_interleave_gate_up(const uint8_t* packed_gate, const float*
  * intermediate in memory. Per token m and output j:
  *   g = bf16 output of gate row j for x (the arithmetic of bitnet_linear, bit for bit);
  *   u = the same for up row j;
- *   s = bf16(silu(g)), silu evaluated in binary32: g / (1 + e^-g) for g >= 0 and
- *       g e^g / (1 + e^g) for g < 0 (expf, IEEE multiply, add and divide);
+ *   s = bf16(silu(g)), silu evaluated in binary32 with e = expf(-|g|): g / (1 + e) for
+ *       g >= 0 and g e / (1 + e) for g < 0 (a fast divide: the divisor lies in [1, 2]);
  *   h = bf16(s * u) (the product of two bf16 values, exact in binary32 above 2^-126).
  *   x [in] (M, K) bf16 bits.  packed_gu, s_w_gu [in] from bitnet_interleave_gate_up.
  *   h [out] (M, I) bf16 bits, 16-byte aligned.

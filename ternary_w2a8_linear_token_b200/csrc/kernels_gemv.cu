@@ -276,26 +276,26 @@ __global__ void __launch_bounds__(kThreads, MT <= 2 ? 2 : 1) gemv_w2a8_kernel(co
                     swiglu_bf16_bits(g, u);
             }
         }
-        return;
-    }
+    } else {
 #pragma unroll
-    for (int r = 0; r < RW; ++r) {
+        for (int r = 0; r < RW; ++r) {
 #pragma unroll
-        for (int m = 0; m < MT; ++m) {
-            const int32_t total = __reduce_add_sync(0xFFFFFFFFu, acc[r][m][0] + acc[r][m][1]);
-            if (lane == r * MT + m && rvalid[r] && m < Mreal) {
-                const GemvProj& pr = p.proj[pj[r]];
-                const int32_t v = total - qs_tot[m];
-                const int64_t o = int64_t(m) * pr.N + nrow[r];
-                if (p.out_kind == 2) {
-                    reinterpret_cast<int32_t*>(pr.y)[o] = v;
-                } else {
-                    const float rx = __frcp_rn(s_tok[m]);
-                    const float yv = __fmul_rn(__int2float_rn(v), __fmul_rn(sw[r], rx));
-                    if (p.out_kind == 0)
-                        reinterpret_cast<__nv_bfloat16*>(pr.y)[o] = __float2bfloat16_rn(yv);
-                    else
-                        reinterpret_cast<float*>(pr.y)[o] = yv;
+            for (int m = 0; m < MT; ++m) {
+                const int32_t total = __reduce_add_sync(0xFFFFFFFFu, acc[r][m][0] + acc[r][m][1]);
+                if (lane == r * MT + m && rvalid[r] && m < Mreal) {
+                    const GemvProj& pr = p.proj[pj[r]];
+                    const int32_t v = total - qs_tot[m];
+                    const int64_t o = int64_t(m) * pr.N + nrow[r];
+                    if (p.out_kind == 2) {
+                        reinterpret_cast<int32_t*>(pr.y)[o] = v;
+                    } else {
+                        const float rx = __frcp_rn(s_tok[m]);
+                        const float yv = __fmul_rn(__int2float_rn(v), __fmul_rn(sw[r], rx));
+                        if (p.out_kind == 0)
+                            reinterpret_cast<__nv_bfloat16*>(pr.y)[o] = __float2bfloat16_rn(yv);
+                        else
+                            reinterpret_cast<float*>(pr.y)[o] = yv;
+                    }
                 }
             }
         }

@@ -583,21 +583,32 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
                     if (p.swiglu) {
                         // Interleaved gate/up rows: lane l < 16 holds gate row j, lane l + 16
                         // the up row of the same output j = n0 / 2 + 16 quarter + l. Both
-                        // dequantise as in the plain epilogue; the up value moves down 16
-                        // lanes and the gate lanes write h = SwiGLU(g, u), 16 outputs per token.
+                        // dequantise as in the plain epilogue. Partner lanes (l, l + 16) then
+                        // split the columns: one shuffle per column pair gives lane l the up
+                        // value of column c and lane l + 16 the gate value of column
+                        // c + kHC / 2, so every lane computes SwiGLU for half of the columns.
+                        constexpr int kHalf = kHC / 2;
+                        const bool gate_lane = lane < kSwigluBlock;
 #pragma unroll
-                        for (int c = 0; c < kHC; ++c) {
-                            const float yv = __fmul_rn(__int2float_rn(int32_t(v[c])), f[c]);
-                            const float up = __shfl_down_sync(0xFFFFFFFFu, yv, 16);
-                            v[c] = swiglu_bf16_bits(yv, up);
+                        for (int c = 0; c < kHalf; ++c) {
+                            const float y0 = __fmul_rn(__int2float_rn(int32_t(v[c])), f[c]);
+                            const float y1 =
+                                __fmul_rn(__int2float_rn(int32_t(v[c + kHalf])), f[c + kHalf]);
+                            const float other =
+                                __shfl_xor_sync(0xFFFFFFFFu, gate_lane ? y1 : y0, kSwigluBlock);
+                            // lane l: column c; lane l + 16: column c + kHalf
+                            const float g = gate_lane ? y0 : other;
+                            const float u = gate_lane ? other : y1;
+                            v[c] = swiglu_bf16_bits(g, u);
                         }
                         uint8_t* sb = stage + (staged_stores & 1u) * 1024u;
                         if (lane == 0) bulk_wait_group_read<1>();
                         __syncwarp();
-                        if (lane < kSwigluBlock) {
-                            uint16_t* b = reinterpret_cast<uint16_t*>(sb) + lane;
+                        {  // staging tile [token][16 outputs]
+                            uint16_t* b = reinterpret_cast<uint16_t*>(sb) +
+                                          (gate_lane ? lane : kHalf * kSwigluBlock + lane - kSwigluBlock);
 #pragma unroll
-                            for (int c = 0; c < kHC; ++c) b[c * kSwigluBlock] = uint16_t(v[c]);
+                            for (int c = 0; c < kHalf; ++c) b[c * kSwigluBlock] = uint16_t(v[c]);
                         }
                         fence_proxy_async_smem();
                         __syncwarp();

@@ -9,15 +9,16 @@
 
 namespace bitnet {
 
-// silu(z) = z * sigmoid(z) in binary32 without overflow: z / (1 + e^-z) for z >= 0 and
-// z e^z / (1 + e^z) for z < 0, so the exponential's argument is never positive. expf is
-// CUDA's (within 2 binary32 steps); multiply, add and divide are single IEEE roundings.
-// Below z = -104 e^z underflows to 0 and the result is -0, as is the exactly rounded bf16
-// value there (|silu(z)| < 2^-134).
+// silu(z) = z * sigmoid(z) in binary32, branch-free and without overflow: with
+// e = exp(-|z|) in (0, 1], silu(z) = z / (1 + e) for z >= 0 and z e / (1 + e) for z < 0.
+// expf is CUDA's (within 2 binary32 steps); the divisor lies in [1, 2], where __fdividef is
+// within 2 steps, so the result is within a few binary32 steps of the exact value, far
+// below the bf16 step it is rounded to next. Below z = -104 e underflows to 0 and the
+// result is -0, as is the exactly rounded bf16 value there (|silu(z)| < 2^-134).
 __device__ __forceinline__ float silu_f32(float z) {
-    if (z >= 0.0f) return __fdiv_rn(z, __fadd_rn(1.0f, expf(-z)));
-    const float e = expf(z);
-    return __fdiv_rn(__fmul_rn(z, e), __fadd_rn(1.0f, e));
+    const float e = expf(-fabsf(z));
+    const float num = z >= 0.0f ? z : __fmul_rn(z, e);
+    return __fdividef(num, __fadd_rn(1.0f, e));
 }
 
 __device__ __forceinline__ float bf16_round_f32(float v) {
