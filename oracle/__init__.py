@@ -65,6 +65,8 @@ def _load():
             lib.oracle_bitlinear_sampled.argtypes = [P, I64, I64, P, P, I, I64, P, I64, P, I64,
                                                      P, P, P, P, P, P, P]
             lib.oracle_swiglu.argtypes = [P, P, I64, P, P]
+            lib.oracle_quant_act_per_tensor.argtypes = [P, I64, I64, P, P]
+            lib.oracle_quant_act_per_tensor.restype = ctypes.c_int
             for name in ("oracle_absmean_scale", "oracle_ternarize", "oracle_pack",
                          "oracle_unpack", "oracle_quant_act", "oracle_ternary_matmul",
                          "oracle_dequant", "oracle_bitlinear_sampled", "oracle_swiglu"):
@@ -141,6 +143,18 @@ def quant_act(x_bf16_bits: np.ndarray):
     return q, s
 
 
+def quant_act_per_tensor(x_bf16_bits: np.ndarray):
+    """Per-tensor absmax int8 quantiser ("BitNet 1-bit LLM推理优化", §2.2 I2_S and §3.2): one
+    scale for the whole (M, K) input. Returns (q, s_x) with s_x holding that scale M times."""
+    x = np.ascontiguousarray(x_bf16_bits, dtype=np.uint16)
+    M, K = x.shape
+    q = np.empty((M, K), dtype=np.int8)
+    s = np.empty(M, dtype=np.float32)
+    _check(_load().oracle_quant_act_per_tensor(_ptr(x), M, K, _ptr(q), _ptr(s)),
+           "quant_act_per_tensor")
+    return q, s
+
+
 def ternary_matmul(q: np.ndarray, t: np.ndarray) -> np.ndarray:
     """int32 acc[m,n] = sum_k q[m,k] t[n,k] by add / subtract / skip ("BitNet 深度实战", §4.4)."""
     q = np.ascontiguousarray(q, dtype=np.int8)
@@ -174,9 +188,10 @@ def round_bf16(y: np.ndarray) -> np.ndarray:
 
 
 def bitlinear(x_bf16_bits: np.ndarray, packed: np.ndarray, s_w: np.ndarray, per_row: bool,
-              K: int):
-    """Full forward on packed weights. Returns dict(y=fp64 (M,N), acc, q, s_x)."""
-    q, s_x = quant_act(x_bf16_bits)
+              K: int, act_per_tensor: bool = False):
+    """Full forward on packed weights. Returns dict(y=fp64 (M,N), acc, q, s_x). The
+    activation scale is per token, or one per tensor with act_per_tensor."""
+    q, s_x = (quant_act_per_tensor if act_per_tensor else quant_act)(x_bf16_bits)
     t = unpack(packed, K)
     acc = ternary_matmul(q, t)
     y = dequant(acc, s_x, s_w, per_row)
@@ -243,3 +258,18 @@ def swiglu_gate_up_sampled(x_bf16_bits: np.ndarray, packed_gate: np.ndarray,
     s_bits, h_bits = swiglu(g_bits, u_bits)
     return {"g": yg, "u": yu, "g_bits": g_bits, "u_bits": u_bits, "s_bits": s_bits,
             "h_bits": h_bits}
+
+
+def bitlinear_sampled_per_tensor_act(x_bf16_bits: np.ndarray, packed: np.ndarray,
+                                     s_w: np.ndarray, per_row: bool, K: int, m_idx, n_idx):
+    """The forward with a per-tensor activation scale on sampled tokens m_idx and outputs
+    n_idx: the scale needs all of x, so x is quantised whole, then the sampled rows of q meet
+    the sampled weight rows (the oracle's own steps, composed)."""
+    q, s_x = quant_act_per_tensor(x_bf16_bits)
+    m_idx = np.asarray(m_idx, dtype=np.int64)
+    n_idx = np.asarray(n_idx, dtype=np.int64)
+    t = unpack(np.ascontiguousarray(packed[n_idx]), K)
+    acc = ternary_matmul(q[m_idx], t)
+    sw = np.ascontiguousarray(s_w[n_idx] if per_row else s_w, dtype=np.float32)
+    y = dequant(acc, s_x[m_idx], sw, per_row)
+    return {"y": y, "acc": acc, "q": q[m_idx], "s_x": s_x[m_idx]}

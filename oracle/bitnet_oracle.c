@@ -27,7 +27,10 @@
  *           "技术架构：融合内核的三重优化": weights stored (N, K/4) uint8, four per
  *           byte; activations quantised to int8 for an int8 matmul.
  *  [P2-3.2] "BitNet 1-bit LLM推理优化：内存布局、量化策略与硬件加速", section 3.2
- *           "激活量化策略": int8 activations with an absmax-style scale.
+ *           "激活量化策略": int8 activations with an absmax-style scale, per-tensor
+ *           or per-channel.
+ *  [P2-2.2] same page, section 2.2 "I2_S（Int2 with Scale）内核": follows the
+ *           per-tensor int8 activation quantisation BitNet b1.58 was trained with.
  *
  * Readings where the pages are silent (each one is listed in the design notes):
  *  - code = t + 1 (00 = -1, 01 = 0, 10 = +1); code 11 never appears. Section 4.3
@@ -169,6 +172,35 @@ int oracle_quant_act(const uint16_t* x, int64_t M, int64_t K, int8_t* q, float* 
         }
         float denom = amax < ORACLE_EPS ? ORACLE_EPS : amax;
         float s = 127.0f / denom;
+        s_x[m] = s;
+        for (int64_t k = 0; k < K; ++k) {
+            float v = bf16_to_float(x[m * K + k]) * s;
+            float r = rintf(v);
+            if (r > 127.0f) r = 127.0f;
+            if (r < -128.0f) r = -128.0f;
+            q[m * K + k] = (int8_t)r;
+        }
+    }
+    return ORACLE_OK;
+}
+
+/* ---------------------------------------------------------------------------
+ * Per-tensor absmax int8 activation quantiser ([P2-2.2] I2_S keeps BitNet
+ * b1.58's per-tensor int8 activation setting; [P2-3.2] lists per-tensor scales):
+ * one scale for the whole (M, K) input, amax = max over every m and k, then the
+ * same s = 127 / max(amax, eps) and q = clamp(rint(x * s), -128, 127) as the
+ * per-token quantiser. s_x receives s in each of its M entries.
+ * ------------------------------------------------------------------------- */
+int oracle_quant_act_per_tensor(const uint16_t* x, int64_t M, int64_t K, int8_t* q, float* s_x) {
+    if (!x || !q || !s_x || M <= 0 || K <= 0) return ORACLE_BAD_ARG;
+    float amax = 0.0f;
+    for (int64_t i = 0; i < M * K; ++i) {
+        float a = fabsf(bf16_to_float(x[i]));
+        if (a > amax) amax = a;
+    }
+    float denom = amax < ORACLE_EPS ? ORACLE_EPS : amax;
+    float s = 127.0f / denom;
+    for (int64_t m = 0; m < M; ++m) {
         s_x[m] = s;
         for (int64_t k = 0; k < K; ++k) {
             float v = bf16_to_float(x[m * K + k]) * s;

@@ -443,3 +443,60 @@ def test_swiglu_bound_helper_accepts_exact_and_rejects_far(oracle):
     bad[1, 5] = bf16_from_ordered(bf16_ordered(bad[1:2, 5:6]) + 40)[0, 0]
     with pytest.raises(AssertionError):
         assert_swiglu_within_bound(bad, ref, oracle)
+
+
+# ---------------------------------------------------------------- per-tensor activation scale
+
+def test_quant_per_tensor_hand_example(oracle):
+    """x = [[1, -2], [4, 0.5]]: amax 4 over the whole tensor, s = 127/4 = 31.75, q = rint of
+    [31.75, -63.5, 127, 15.875] = [32, -64 (tie to even), 127, 16]; both rows share s."""
+    x = synth.to_bf16_bits(np.array([[1.0, -2.0], [4.0, 0.5]], dtype=np.float32))
+    q, s = oracle.quant_act_per_tensor(x)
+    assert s.tolist() == [31.75, 31.75]
+    assert q.tolist() == [[32, -64], [127, 16]]
+    q_tok, s_tok = oracle.quant_act(x)  # per token the first row has its own scale 63.5
+    assert s_tok.tolist() == [63.5, 31.75] and q_tok[0].tolist() == [64, -127]
+
+
+def test_quant_per_tensor_reduces_and_invariants(oracle):
+    """One token: per tensor is per token. Many: |q| <= 127 with max |q| = 127 once over the
+    tensor, the row holding the global amax equals its per-token quantisation, rows permute
+    with q, scaling x by 2 (exact) leaves q unchanged, and an all-zero x gives q = 0."""
+    rng = np.random.default_rng(21)
+    x1 = synth.to_bf16_bits(rng.normal(0, 1, (1, 640)).astype(np.float32))
+    assert all(np.array_equal(a, b) for a, b in zip(oracle.quant_act_per_tensor(x1),
+                                                    oracle.quant_act(x1)))
+    xf = rng.normal(0, 1, (7, 256)).astype(np.float32)
+    xf[3] *= 5.0
+    x = synth.to_bf16_bits(xf)
+    q, s = oracle.quant_act_per_tensor(x)
+    assert np.all(s == s[0]) and np.abs(q).max() == 127 and np.abs(q.astype(int)).max() <= 127
+    r = int(np.argmax(np.abs(synth.bf16_bits_to_f32(x)).max(axis=1)))
+    q_tok, _ = oracle.quant_act(x)
+    assert np.array_equal(q[r], q_tok[r])
+    assert np.abs(q[(r + 1) % 7]).max() < 127  # other rows use the larger common scale
+    perm = rng.permutation(7)
+    assert np.array_equal(oracle.quant_act_per_tensor(np.ascontiguousarray(x[perm]))[0], q[perm])
+    x2 = synth.to_bf16_bits(synth.bf16_bits_to_f32(x) * np.float32(2.0))
+    q2, s2 = oracle.quant_act_per_tensor(x2)
+    assert np.array_equal(q2, q) and s2[0] == s[0] / 2
+    qz, sz = oracle.quant_act_per_tensor(np.zeros((3, 64), dtype=np.uint16))
+    assert not qz.any() and sz[0] == np.float32(127.0) / np.float32(1e-5)
+
+
+def test_bitlinear_per_tensor_act_matches_float_linear(oracle):
+    """The forward with a per-tensor activation scale equals linear(q / s_x, t * s_w) in fp64
+    ("BitNet 深度实战" §3.2), and its sampled form equals the full one on the sample."""
+    rng = np.random.default_rng(22)
+    M, N, K = 5, 24, 128
+    x = synth.to_bf16_bits(rng.normal(0, 1, (M, K)).astype(np.float32))
+    t = rng.integers(-1, 2, (N, K)).astype(np.int8)
+    s_w = rng.uniform(0.5, 2, N).astype(np.float32)
+    r = oracle.bitlinear(x, oracle.pack(t), s_w, True, K, act_per_tensor=True)
+    q, s = oracle.quant_act_per_tensor(x)
+    ref = (q.astype(np.float64) / s.astype(np.float64)[:, None]) @ \
+          (t.astype(np.float64) * s_w.astype(np.float64)[:, None]).T
+    np.testing.assert_allclose(r["y"], ref, rtol=1e-12, atol=1e-12)
+    m_idx, n_idx = np.array([0, 3, 4]), np.array([1, 7, 23])
+    rs = oracle.bitlinear_sampled_per_tensor_act(x, oracle.pack(t), s_w, True, K, m_idx, n_idx)
+    assert np.array_equal(rs["y"], r["y"][np.ix_(m_idx, n_idx)])
