@@ -63,6 +63,16 @@ typedef enum {
     BITNET_OUT_F32 = 1   /* y is (M, N) fp32                                          */
 } bitnet_out_dtype;
 
+/* Granularity of the activation scale s_x. Per token is the default of every call without
+ * an `act` argument; per tensor is one scale for the whole (M, K) input, the setting the I2_S
+ * kernel keeps from BitNet b1.58's training ("BitNet 1-bit LLM推理优化" section 2.2; section 3.2
+ * lists per-tensor and per-channel scales). A scale per K channel is not offered: it would
+ * sit inside the sum over k, so the contraction could no longer run in integers. */
+typedef enum {
+    BITNET_ACT_PER_TOKEN = 0, /* s_x[m] = 127 / max(max_k |x[m,k]|, 1e-5)                   */
+    BITNET_ACT_PER_TENSOR = 1 /* one s = 127 / max(max_{m,k} |x[m,k]|, 1e-5) for every token */
+} bitnet_act_mode;
+
 typedef enum {
     BITNET_PATH_AUTO = 0, /* GEMV for M <= BITNET_GEMV_AUTO_M; for M up to                */
                           /* BITNET_GEMV_MAX_M the tensor-core GEMM when the workspace    */
@@ -110,6 +120,18 @@ bitnet_status bitnet_pack_ternary(const int8_t* t, int64_t N, int64_t K, uint8_t
  */
 bitnet_status bitnet_quant_act(const uint16_t* x, int64_t M, int64_t K, int8_t* q, float* s_x,
                                void* stream);
+
+/*
+ * bitnet_quant_act_ex — bitnet_quant_act with a choice of scale granularity. With
+ * BITNET_ACT_PER_TENSOR all M entries of s_x receive the one scale, and the call needs
+ * `workspace` (device, 4-byte aligned) of at least BITNET_QUANT_WORKSPACE_BYTES bytes for the
+ * partial maxima of |x|; per token it may be NULL. Two kernels run per tensor: partial maxima
+ * of |x|, then the quantiser reducing them.
+ */
+#define BITNET_QUANT_WORKSPACE_BYTES 4096
+bitnet_status bitnet_quant_act_ex(const uint16_t* x, int64_t M, int64_t K, bitnet_act_mode act,
+                                  int8_t* q, float* s_x, void* workspace, size_t workspace_bytes,
+                                  void* stream);
 
 /*
  * Workspace bytes the tensor-core path of bitnet_linear / bitnet_linear_batch needs for
@@ -173,6 +195,18 @@ bitnet_status bitnet_linear_batch_ex(const uint16_t* x, int64_t M, int64_t K,
                                      const bitnet_proj* projs, int32_t nproj,
                                      bitnet_out_dtype out_dtype, void* workspace,
                                      size_t workspace_bytes, bitnet_path path, void* stream);
+
+/*
+ * bitnet_linear_batch_act — bitnet_linear_batch_ex with a choice of activation scale
+ * granularity (bitnet_act_mode). Per tensor: the quantiser uses one scale for all M tokens
+ * (the tensor-core path adds one small kernel for the partial maxima of |x|; the GEMV takes
+ * the maximum over its tokens in the same launch), and the epilogue divides by that scale.
+ */
+bitnet_status bitnet_linear_batch_act(const uint16_t* x, int64_t M, int64_t K,
+                                      const bitnet_proj* projs, int32_t nproj,
+                                      bitnet_out_dtype out_dtype, bitnet_act_mode act,
+                                      void* workspace, size_t workspace_bytes, bitnet_path path,
+                                      void* stream);
 
 /*
  * bitnet_linear_i32 — the contraction alone, for bit-exact checks: acc[m, n] =

@@ -41,6 +41,8 @@ OK, ERR_NULL, ERR_SHAPE, ERR_ALIGN, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT, ERR_
 SCALE_PER_TENSOR, SCALE_PER_ROW = 0, 1
 OUT_BF16, OUT_F32 = 0, 1
 PATH_AUTO, PATH_GEMV, PATH_TC = 0, 1, 2
+ACT_PER_TOKEN, ACT_PER_TENSOR = 0, 1
+QUANT_WORKSPACE_BYTES = 4096
 GEMV_MAX_M = 8
 GEMV_AUTO_M = 4  # PATH_AUTO: GEMV up to here; 5..8 tokens take the tensor-core path given a workspace
 WATCHDOG_TMA_FULL, WATCHDOG_UNPACK, WATCHDOG_EMPTY, WATCHDOG_ACCUM, WATCHDOG_DRAIN = (
@@ -62,6 +64,9 @@ _SIGS = {
     "bitnet_pack_ternary": ([_P, _I64, _I64, _P, _P], ctypes.c_int),
     "bitnet_quant_act": ([_P, _I64, _I64, _P, _P, _P], ctypes.c_int),
     "bitnet_linear_workspace_size": ([_I64, _I64], _SZ),
+    "bitnet_quant_act_ex": ([_P, _I64, _I64, ctypes.c_int, _P, _P, _P, _SZ, _P], ctypes.c_int),
+    "bitnet_linear_batch_act": ([_P, _I64, _I64, ctypes.POINTER(bitnet_proj), _I32, ctypes.c_int,
+                                 ctypes.c_int, _P, _SZ, ctypes.c_int, _P], ctypes.c_int),
     "bitnet_linear": ([_P, _I64, _I64, _P, _P, ctypes.c_int, _I64, _P, ctypes.c_int, _P, _SZ, _P],
                       ctypes.c_int),
     "bitnet_linear_ex": ([_P, _I64, _I64, _P, _P, ctypes.c_int, _I64, _P, ctypes.c_int, _P, _SZ,
@@ -158,6 +163,18 @@ def bitnet_quant_act(x: torch.Tensor, stream=None):
     return q, s_x
 
 
+def bitnet_quant_act_ex(x: torch.Tensor, act: int = ACT_PER_TOKEN, stream=None):
+    """bitnet_quant_act with a choice of scale granularity (ACT_PER_TOKEN / ACT_PER_TENSOR)."""
+    M, K = x.shape
+    q = torch.empty((M, K), dtype=torch.int8, device=x.device)
+    s_x = torch.empty(M, dtype=torch.float32, device=x.device)
+    ws = torch.empty(QUANT_WORKSPACE_BYTES, dtype=torch.uint8, device=x.device)
+    _check(lib.bitnet_quant_act_ex(_x_ptr(x), M, K, act, q.data_ptr(), s_x.data_ptr(),
+                                   ws.data_ptr(), ws.numel(), _stream(stream)),
+           "bitnet_quant_act_ex")
+    return q, s_x
+
+
 def _ws_args(workspace: Optional[torch.Tensor], M: int, K: int, path: int, device):
     need_tc = path == PATH_TC or (path == PATH_AUTO and M > GEMV_AUTO_M)
     if workspace is None:
@@ -208,6 +225,33 @@ def bitnet_linear_batch(x: torch.Tensor, projs: Sequence, out_dtype: torch.dtype
     wp, wb, _keep = _ws_args(workspace, M, K, path, x.device)
     _check(lib.bitnet_linear_batch_ex(_x_ptr(x), M, K, arr, n, od, wp, wb, path, _stream(stream)),
            "bitnet_linear_batch")
+    return list(ys)
+
+
+def bitnet_linear_batch_act(x: torch.Tensor, projs: Sequence, act: int,
+                            out_dtype: torch.dtype = torch.bfloat16,
+                            ys: Optional[Sequence[torch.Tensor]] = None,
+                            workspace: Optional[torch.Tensor] = None, path: int = PATH_AUTO,
+                            stream=None):
+    """bitnet_linear_batch with a choice of activation scale granularity (act)."""
+    M, K = x.shape
+    n = len(projs)
+    if not 1 <= n <= MAX_PROJ:
+        raise ValueError(f"1..{MAX_PROJ} projections")
+    if ys is None:
+        ys = [torch.empty((M, p[0].shape[0]), dtype=out_dtype, device=x.device) for p in projs]
+    od = OUT_BF16 if ys[0].dtype == torch.bfloat16 else OUT_F32
+    arr = (bitnet_proj * n)()
+    for i, (packed, s_w, per_row) in enumerate(projs):
+        arr[i].packed = _dev(packed, torch.uint8, "packed")
+        arr[i].s_w = _dev(s_w, torch.float32, "s_w")
+        arr[i].mode = int(bool(per_row))
+        arr[i].reserved = 0
+        arr[i].N = packed.shape[0]
+        arr[i].y = _dev(ys[i], ys[i].dtype, "y")
+    wp, wb, _keep = _ws_args(workspace, M, K, path, x.device)
+    _check(lib.bitnet_linear_batch_act(_x_ptr(x), M, K, arr, n, od, act, wp, wb, path,
+                                       _stream(stream)), "bitnet_linear_batch_act")
     return list(ys)
 
 

@@ -90,7 +90,8 @@ bool use_gemv(int64_t M, int64_t K, bitnet_path path, const void* ws, size_t ws_
 // batch is one interleaved gate/up matrix of N = 2I rows whose output is h (M, I) bf16.
 bitnet_status run_batch(const uint16_t* x_bf16, const int8_t* q_in, int64_t M, int64_t K,
                         const Batch& b, int out_kind, void* workspace, size_t workspace_bytes,
-                        bitnet_path path, cudaStream_t stream, bool swiglu = false) {
+                        bitnet_path path, cudaStream_t stream, bool swiglu = false,
+                        bool act_per_tensor = false) {
     if (use_gemv(M, K, path, workspace, workspace_bytes)) {
         if (!gemv_supported(M, K)) return BITNET_ERR_UNSUPPORTED;
         GemvParams p;
@@ -101,6 +102,7 @@ bitnet_status run_batch(const uint16_t* x_bf16, const int8_t* q_in, int64_t M, i
         p.M = static_cast<int32_t>(M);
         p.nproj = b.nproj;
         p.out_kind = out_kind;
+        p.act_per_tensor = act_per_tensor ? 1 : 0;
         int64_t rows = 0;
         for (int i = 0; i < b.nproj; ++i) {
             p.proj[i].packed = b.proj[i].packed;
@@ -127,6 +129,8 @@ bitnet_status run_batch(const uint16_t* x_bf16, const int8_t* q_in, int64_t M, i
     float* s_x = reinterpret_cast<float*>(ws + ws_q_bytes(M, K));
     float* r_x = reinterpret_cast<float*>(ws + ws_q_bytes(M, K) + ws_scale_bytes(M));
     int32_t* qsum = reinterpret_cast<int32_t*>(ws + ws_q_bytes(M, K) + 2 * ws_scale_bytes(M));
+    uint32_t* amax_parts =
+        reinterpret_cast<uint32_t*>(ws + ws_q_bytes(M, K) + 3 * ws_scale_bytes(M));
 
     TcParams p;
     std::memset(&p, 0, sizeof(p));
@@ -232,9 +236,14 @@ bitnet_status run_batch(const uint16_t* x_bf16, const int8_t* q_in, int64_t M, i
         }
     }
 
+    const bool per_tensor = act_per_tensor && !q_in;
+    if (per_tensor && launch_amax_parts(x_bf16, M, K, amax_parts, stream, /*pdl=*/true) !=
+                          cudaSuccess)
+        return BITNET_ERR_CUDA;
     cudaError_t e = launch_quant(x_bf16, q_in, M, K, q_ws, q_in ? nullptr : s_x,
                                  q_in ? nullptr : r_x, /*permuted=*/1, stream, /*pdl=*/true, zero,
-                                 zero_bytes, qsum);
+                                 zero_bytes, qsum, per_tensor ? amax_parts : nullptr,
+                                 per_tensor ? amax_parts_count(M, K) : 0);
     if (e != cudaSuccess) return BITNET_ERR_CUDA;
     return from_cuda(launch_tc_gemm(p, bn, stream, /*pdl=*/true));
 }
@@ -317,6 +326,26 @@ bitnet_status bitnet_quant_act(const uint16_t* x, int64_t M, int64_t K, int8_t* 
                                   static_cast<cudaStream_t>(stream), /*pdl=*/false));
 }
 
+bitnet_status bitnet_quant_act_ex(const uint16_t* x, int64_t M, int64_t K, bitnet_act_mode act,
+                                  int8_t* q, float* s_x, void* workspace, size_t workspace_bytes,
+                                  void* stream) {
+    if (act != BITNET_ACT_PER_TOKEN && act != BITNET_ACT_PER_TENSOR) return BITNET_ERR_UNSUPPORTED;
+    if (act == BITNET_ACT_PER_TOKEN) return bitnet_quant_act(x, M, K, q, s_x, stream);
+    if (!x || !q || !s_x) return BITNET_ERR_NULL;
+    bitnet_status st = check_mk(M, K);
+    if (st != BITNET_OK) return st;
+    if (!aligned(x, 16) || !aligned(q, 16) || !aligned(s_x, 4)) return BITNET_ERR_ALIGN;
+    static_assert(BITNET_QUANT_WORKSPACE_BYTES >= kMaxAmaxParts * 4, "partial maxima fit");
+    if (!workspace || workspace_bytes < BITNET_QUANT_WORKSPACE_BYTES) return BITNET_ERR_WORKSPACE;
+    if (!aligned(workspace, 4)) return BITNET_ERR_ALIGN;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    uint32_t* parts = static_cast<uint32_t*>(workspace);
+    if (launch_amax_parts(x, M, K, parts, s, /*pdl=*/false) != cudaSuccess) return BITNET_ERR_CUDA;
+    return from_cuda(launch_quant(x, nullptr, M, K, q, s_x, nullptr, /*permuted=*/0, s,
+                                  /*pdl=*/true, nullptr, 0, nullptr, parts,
+                                  amax_parts_count(M, K)));
+}
+
 size_t bitnet_linear_workspace_size(int64_t M, int64_t K) {
     if (M < 1 || K < 1) return 0;
     return ws_total_bytes(M, K) + ws_split_bytes(M);
@@ -334,6 +363,23 @@ bitnet_status bitnet_linear_batch_ex(const uint16_t* x, int64_t M, int64_t K,
     if (st != BITNET_OK) return st;
     return run_batch(x, nullptr, M, K, b, int(out_dtype), workspace, workspace_bytes, path,
                      static_cast<cudaStream_t>(stream));
+}
+
+bitnet_status bitnet_linear_batch_act(const uint16_t* x, int64_t M, int64_t K,
+                                      const bitnet_proj* projs, int32_t nproj,
+                                      bitnet_out_dtype out_dtype, bitnet_act_mode act,
+                                      void* workspace, size_t workspace_bytes, bitnet_path path,
+                                      void* stream) {
+    if (act != BITNET_ACT_PER_TOKEN && act != BITNET_ACT_PER_TENSOR) return BITNET_ERR_UNSUPPORTED;
+    if (out_dtype != BITNET_OUT_BF16 && out_dtype != BITNET_OUT_F32) return BITNET_ERR_UNSUPPORTED;
+    if (path != BITNET_PATH_AUTO && path != BITNET_PATH_GEMV && path != BITNET_PATH_TC)
+        return BITNET_ERR_UNSUPPORTED;
+    Batch b;
+    bitnet_status st = validate_batch(x, M, K, projs, nproj, int(out_dtype), &b);
+    if (st != BITNET_OK) return st;
+    return run_batch(x, nullptr, M, K, b, int(out_dtype), workspace, workspace_bytes, path,
+                     static_cast<cudaStream_t>(stream), /*swiglu=*/false,
+                     act == BITNET_ACT_PER_TENSOR);
 }
 
 bitnet_status bitnet_linear_batch(const uint16_t* x, int64_t M, int64_t K,

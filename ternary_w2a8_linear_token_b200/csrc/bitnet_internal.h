@@ -19,8 +19,11 @@ constexpr int kMaxProj = BITNET_MAX_PROJ;
 inline size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 inline size_t ws_q_bytes(int64_t M, int64_t K) { return align256(size_t(M) * size_t(K)); }
 inline size_t ws_scale_bytes(int64_t M) { return align256(size_t(M) * 4); }
+// Then the partial maxima of |x| for a per-tensor activation scale (kMaxAmaxParts words).
+constexpr int kMaxAmaxParts = 1024;
+inline size_t ws_parts_bytes() { return size_t(kMaxAmaxParts) * 4; }
 inline size_t ws_total_bytes(int64_t M, int64_t K) {
-    return ws_q_bytes(M, K) + 3 * ws_scale_bytes(M);
+    return ws_q_bytes(M, K) + 3 * ws_scale_bytes(M) + ws_parts_bytes();
 }
 
 // SwiGLU of the MLP: interleaved gate/up weight rows come in blocks of this many rows.
@@ -62,7 +65,7 @@ struct GemvParams {
     int32_t stage_x;   // set by the launcher: stage x in shared memory
     int32_t swiglu;    // 1: proj[0] is an interleaved gate/up matrix, total_rows counts
                        // output pairs, y = SwiGLU (bf16, (M, proj[0].N))
-    int32_t pad;
+    int32_t act_per_tensor;  // 1: one activation scale for all M tokens
     GemvProj proj[kMaxProj];
 };
 
@@ -74,9 +77,16 @@ bool gemv_supported(int64_t M, int64_t K);
 // the tensor-core path. q_in != nullptr: copy-permute given int8 q (no scales).
 // zero / zero_bytes: a 16-byte aligned region (multiple of 16 bytes) the launch clears, spread
 // over its CTAs (the split-K area of the GEMM that follows), or null.
+// amax_parts / n_parts: when set, every token uses the one scale of the whole input, whose
+// amax is the maximum of these partial maxima (written by launch_amax_parts).
 cudaError_t launch_quant(const uint16_t* x, const int8_t* q_in, int64_t M, int64_t K, int8_t* q,
                          float* s_x, float* r_x, int permuted, cudaStream_t stream, bool pdl,
-                         void* zero = nullptr, int64_t zero_bytes = 0, int32_t* qsum = nullptr);
+                         void* zero = nullptr, int64_t zero_bytes = 0, int32_t* qsum = nullptr,
+                         const uint32_t* amax_parts = nullptr, int n_parts = 0);
+// Partial maxima of |x| over all of x (M, K) into parts[0 .. amax_parts_count(M, K)).
+int amax_parts_count(int64_t M, int64_t K);
+cudaError_t launch_amax_parts(const uint16_t* x, int64_t M, int64_t K, uint32_t* parts,
+                              cudaStream_t stream, bool pdl);
 
 // ----------------------------------------------------------------------------- packing
 cudaError_t launch_pack_weights(const float* W, int64_t N, int64_t K, int per_row,

@@ -152,13 +152,23 @@ __global__ void __launch_bounds__(kThreads, MT <= 2 ? 2 : 1) gemv_w2a8_kernel(co
             if (lane == 0) s_red[warp][m] = r;
         }
         __syncthreads();
+        uint32_t all[MT];
 #pragma unroll
         for (int m = 0; m < MT; ++m) {
-            uint32_t all = s_red[0][m];
+            all[m] = s_red[0][m];
 #pragma unroll
-            for (int ww = 1; ww < kWarps; ++ww) all = max(all, s_red[ww][m]);
-            s_tok[m] = __fdiv_rn(127.0f, fmaxf(__uint_as_float(all << 16), kEps));
+            for (int ww = 1; ww < kWarps; ++ww) all[m] = max(all[m], s_red[ww][m]);
         }
+        if (p.act_per_tensor) {  // one scale for all real tokens ("推理优化" §2.2, I2_S)
+            uint32_t t = 0;
+#pragma unroll
+            for (int m = 0; m < MT; ++m) t = m < Mreal ? max(t, all[m]) : t;
+#pragma unroll
+            for (int m = 0; m < MT; ++m) all[m] = t;
+        }
+#pragma unroll
+        for (int m = 0; m < MT; ++m)
+            s_tok[m] = __fdiv_rn(127.0f, fmaxf(__uint_as_float(all[m] << 16), kEps));
     } else {
 #pragma unroll
         for (int m = 0; m < MT; ++m) s_tok[m] = 0.0f;

@@ -71,6 +71,14 @@ __device__ __forceinline__ uint2 permute_group_half(uint2 nat, int h) {
     return make_uint2(__byte_perm(lo, hi, 0x5410), __byte_perm(lo, hi, 0x7632));
 }
 
+// Per-tensor activation scale ("BitNet 1-bit LLM推理优化" §2.2, I2_S; §3.2): the amax of the
+// whole input is the maximum of the partial maxima amax_parts_kernel wrote (whole warp).
+__device__ __forceinline__ uint32_t parts_max(const uint32_t* __restrict__ parts, int n, int lane) {
+    uint32_t m = 0;
+    for (int i = lane; i < n; i += 32) m = max(m, parts[i]);
+    return __reduce_max_sync(0xFFFFFFFFu, m);
+}
+
 // One warp per token row; each lane keeps 8 loads in flight. Pass 1 finds amax, pass 2
 // re-reads the row (an L1/L2 hit) and writes q.
 constexpr int kRowsPerCta = kThreads / 32;
@@ -86,7 +94,9 @@ __global__ void __launch_bounds__(kThreads) quant_rows_kernel(const uint16_t* __
                                                               int permuted,
                                                               uint4* __restrict__ zero,
                                                               int64_t zero_words,
-                                                              int32_t* __restrict__ qsum) {
+                                                              int32_t* __restrict__ qsum,
+                                                              const uint32_t* __restrict__ amax_parts,
+                                                              int n_parts) {
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const int64_t m = int64_t(blockIdx.x) * kRowsPerCta + warp;
@@ -115,6 +125,7 @@ __global__ void __launch_bounds__(kThreads) quant_rows_kernel(const uint16_t* __
 #pragma unroll
         for (int u = 0; u < kRegPieces; ++u) mx = max(mx, absmax8_bits(v[u]));
         mx = __reduce_max_sync(0xFFFFFFFFu, mx);
+        if (amax_parts) mx = parts_max(amax_parts, n_parts, lane);  // one scale per tensor
         s = __fdiv_rn(127.0f, fmaxf(bf16_bits_to_float(mx), kEps));
         if (lane == 0) {
             if (s_x) s_x[m] = s;
@@ -149,6 +160,7 @@ __global__ void __launch_bounds__(kThreads) quant_rows_kernel(const uint16_t* __
             for (int u = 0; u < kUnroll; ++u) mx = max(mx, absmax8_bits(v[u]));
         }
         mx = __reduce_max_sync(0xFFFFFFFFu, mx);
+        if (amax_parts) mx = parts_max(amax_parts, n_parts, lane);  // one scale per tensor
         s = __fdiv_rn(127.0f, fmaxf(bf16_bits_to_float(mx), kEps));
         if (lane == 0) {
             if (s_x) s_x[m] = s;
@@ -201,7 +213,8 @@ constexpr int64_t kLongMaxK = int64_t(kLongRowThreads) * kLongPieces * 8;
 __global__ void __launch_bounds__(kLongThreads) quant_long_rows_kernel(
     const uint16_t* __restrict__ x, int64_t M, int64_t K, int8_t* __restrict__ q,
     float* __restrict__ s_x, float* __restrict__ r_x, int permuted, uint4* __restrict__ zero,
-    int64_t zero_words, int32_t* __restrict__ qsum) {
+    int64_t zero_words, int32_t* __restrict__ qsum, const uint32_t* __restrict__ amax_parts,
+    int n_parts) {
     __shared__ uint32_t s_mx[kLongRows][kLongRowThreads / 32];
     __shared__ int32_t s_qs[kLongRows][kLongRowThreads / 32];
     const int row = threadIdx.x / kLongRowThreads;
@@ -233,6 +246,7 @@ __global__ void __launch_bounds__(kLongThreads) quant_long_rows_kernel(
     uint32_t all = 0;
 #pragma unroll
     for (int w = 0; w < kLongRowThreads / 32; ++w) all = max(all, s_mx[row][w]);
+    if (amax_parts) all = parts_max(amax_parts, n_parts, lane);  // one scale per tensor
     const float s = __fdiv_rn(127.0f, fmaxf(bf16_bits_to_float(all), kEps));
     if (active && t == 0) {
         if (s_x) s_x[m] = s;
@@ -262,11 +276,71 @@ __global__ void __launch_bounds__(kLongThreads) quant_long_rows_kernel(
     }
 }
 
+// Partial maxima of |x| over the whole input (bf16 bit patterns, |x| ordered as unsigned
+// integers): CTA b writes the maximum of its grid-stride share to parts[b]. The per-tensor
+// quantiser then reduces the parts; no zeroing or atomics are needed.
+constexpr int kAmaxThreads = 256;
+constexpr int kAmaxUnroll = 4;
+
+__global__ void __launch_bounds__(kAmaxThreads) amax_parts_kernel(const uint4* __restrict__ x,
+                                                                  int64_t pieces,
+                                                                  uint32_t* __restrict__ parts) {
+    __shared__ uint32_t s_w[kAmaxThreads / 32];
+    pdl_wait();
+    pdl_trigger();
+    uint32_t mx = 0;
+    const int64_t stride = int64_t(gridDim.x) * kAmaxThreads;
+    for (int64_t c0 = int64_t(blockIdx.x) * kAmaxThreads + threadIdx.x; c0 < pieces;
+         c0 += stride * kAmaxUnroll) {
+        uint4 v[kAmaxUnroll];
+#pragma unroll
+        for (int u = 0; u < kAmaxUnroll; ++u) {  // independent loads in flight
+            const int64_t c = c0 + u * stride;
+            v[u] = c < pieces ? x[c] : make_uint4(0u, 0u, 0u, 0u);
+        }
+#pragma unroll
+        for (int u = 0; u < kAmaxUnroll; ++u) mx = max(mx, absmax8_bits(v[u]));
+    }
+    mx = __reduce_max_sync(0xFFFFFFFFu, mx);
+    if ((threadIdx.x & 31) == 0) s_w[threadIdx.x >> 5] = mx;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        uint32_t a = 0;
+#pragma unroll
+        for (int w = 0; w < kAmaxThreads / 32; ++w) a = max(a, s_w[w]);
+        parts[blockIdx.x] = a;
+    }
+}
+
 }  // namespace
+
+int amax_parts_count(int64_t M, int64_t K) {
+    const int64_t pieces = M * K / 8;
+    const int64_t per_cta = int64_t(kAmaxThreads) * kAmaxUnroll * 2;
+    int64_t n = (pieces + per_cta - 1) / per_cta;
+    if (n > kMaxAmaxParts) n = kMaxAmaxParts;
+    return static_cast<int>(n < 1 ? 1 : n);
+}
+
+cudaError_t launch_amax_parts(const uint16_t* x, int64_t M, int64_t K, uint32_t* parts,
+                              cudaStream_t stream, bool pdl) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(amax_parts_count(M, K)));
+    cfg.blockDim = dim3(kAmaxThreads);
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, amax_parts_kernel, reinterpret_cast<const uint4*>(x),
+                              M * K / 8, parts);
+}
 
 cudaError_t launch_quant(const uint16_t* x, const int8_t* q_in, int64_t M, int64_t K, int8_t* q,
                          float* s_x, float* r_x, int permuted, cudaStream_t stream, bool pdl,
-                         void* zero, int64_t zero_bytes, int32_t* qsum) {
+                         void* zero, int64_t zero_bytes, int32_t* qsum,
+                         const uint32_t* amax_parts, int n_parts) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>((M + kRowsPerCta - 1) / kRowsPerCta));
     cfg.blockDim = dim3(kThreads);
@@ -281,10 +355,12 @@ cudaError_t launch_quant(const uint16_t* x, const int8_t* q_in, int64_t M, int64
         cfg.gridDim = dim3(static_cast<unsigned>((M + kLongRows - 1) / kLongRows));
         cfg.blockDim = dim3(kLongThreads);
         return cudaLaunchKernelEx(&cfg, quant_long_rows_kernel, x, M, K, q, s_x, r_x, permuted,
-                                  static_cast<uint4*>(zero), zero_bytes / 16, qsum);
+                                  static_cast<uint4*>(zero), zero_bytes / 16, qsum, amax_parts,
+                                  n_parts);
     }
     return cudaLaunchKernelEx(&cfg, quant_rows_kernel, x, q_in, M, K, q, s_x, r_x, permuted,
-                              static_cast<uint4*>(zero), zero_bytes / 16, qsum);
+                              static_cast<uint4*>(zero), zero_bytes / 16, qsum, amax_parts,
+                              n_parts);
 }
 
 }  // namespace bitnet

@@ -159,3 +159,19 @@ def test_swiglu_calls_argument_errors(bn):
     # the tensor-core path needs the workspace
     assert sw(M=300, path=bn.PATH_TC) == bn.ERR_WORKSPACE
     assert sw(M=300, ws=FAKE, wb=16, path=bn.PATH_TC) == bn.ERR_WORKSPACE
+
+
+def test_act_mode_calls_argument_errors(bn):
+    L = bn.lib
+    assert L.bitnet_quant_act_ex(FAKE, 4, 512, 7, FAKE, FAKE, FAKE, 4096, None) == bn.ERR_UNSUPPORTED
+    assert L.bitnet_quant_act_ex(FAKE, 4, 512, 1, FAKE, FAKE, None, 0, None) == bn.ERR_WORKSPACE
+    assert L.bitnet_quant_act_ex(FAKE, 4, 512, 1, FAKE, FAKE, FAKE, 100, None) == bn.ERR_WORKSPACE
+    assert L.bitnet_quant_act_ex(FAKE, 4, 512, 1, FAKE, FAKE, FAKE + 2, 4096, None) == bn.ERR_ALIGN
+    assert L.bitnet_quant_act_ex(None, 4, 512, 1, FAKE, FAKE, FAKE, 4096, None) == bn.ERR_NULL
+    assert L.bitnet_quant_act_ex(FAKE, 4, 96, 1, FAKE, FAKE, FAKE, 4096, None) == bn.ERR_UNSUPPORTED
+    pr = (bn.bitnet_proj * 1)()
+    pr[0].packed, pr[0].s_w, pr[0].mode, pr[0].reserved, pr[0].N, pr[0].y = FAKE, FAKE, 0, 0, 128, FAKE
+    assert L.bitnet_linear_batch_act(FAKE, 4, 512, pr, 1, 0, 9, None, 0, 0, None) == bn.ERR_UNSUPPORTED
+    assert L.bitnet_linear_batch_act(FAKE, 4, 512, pr, 1, 3, 1, None, 0, 0, None) == bn.ERR_UNSUPPORTED
+    assert L.bitnet_linear_batch_act(FAKE, 300, 512, pr, 1, 0, 1, None, 0, 0, None) == bn.ERR_WORKSPACE
+    assert L.bitnet_linear_batch_act(None, 4, 512, pr, 1, 0, 1, None, 0, 0, None) == bn.ERR_NULL
