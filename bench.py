@@ -473,7 +473,7 @@ def run_ours(args):
     e2e_gbs = total_bytes / (e2e_ms_max * 1e-3) / 1e9
 
     # ---------------- prefill GEMM
-    if args.only == "decode":
+    if args.only in ("decode", "mlp"):
         pcalls = []
     else:
         pcalls = build_prefill(bn, torch, dev, args.prefill_m)
@@ -496,6 +496,18 @@ def run_ours(args):
                              "peak_src": f"{peaks['src']} bf16 x {INT8_PER_BF16} "
                                          "(nominal int8:bf16)",
                              "note": "per-call time includes the quantiser launch"}}
+        # the same calls with one activation scale per tensor (partial maxima kernel added)
+        def run_pt():
+            for c in pcalls:
+                bn.bitnet_linear_batch_act(c["x"], [(c["packed"], c["s_w"], False)],
+                                           bn.ACT_PER_TENSOR, ys=[c["y"]], workspace=c["ws"])
+        g_pt = capture(torch, run_pt)
+        pt_ms = timed_steps(torch, g_pt.replay, args.steps, args.warmup, flush, world)
+        assert bn.bitnet_check_device_errors() == 0
+        pt_ms_max, pt_ops = reduce_over_ranks(pt_ms, ops_step * args.steps, world)
+        gemm["act_per_tensor"] = {"value": pt_ops / (pt_ms_max * 1e-3) / 1e12, "unit": "TOPS",
+                                  "ms_per_step": pt_ms_max / args.steps}
+        del g_pt
 
     # ---------------- layer stacks (2B-4T and 8B-class, every layer back to back)
     stacks = []
@@ -513,10 +525,14 @@ def run_ours(args):
 
     # ---------------- fused MLP gate/up + SwiGLU against the unfused sequence
     mlp = []
-    if args.stacks == "all" and args.only == "all":
+    if args.stacks == "all" and args.only in ("all", "mlp"):
+        mlp_m = [int(v) for v in args.mlp_m.split(",")] if args.mlp_m else None
         for name, spec in MLP_SPECS.items():
+            ms = [M for M in spec[3] if mlp_m is None or M in mlp_m]
+            if not ms:
+                continue
             lw = build_mlp(bn, torch, dev, name)
-            for M in spec[3]:
+            for M in ms:
                 r, nl = run_mlp(bn, torch, dev, name, lw, M, min(args.steps, 5), args.warmup,
                                 flush, world, peaks)
                 mlp.append(r)
@@ -551,7 +567,7 @@ def run_ours(args):
             "e2e": {"value": e2e_gbs, "unit": "GB/s",
                     "h2d_bytes_per_step": int(h_x.numel() * 2),
                     "d2h_bytes_per_step": int(h_y.numel() * 2)},
-            "gpu_launches": args.steps * launches_per_step * 2 + args.steps * 2 * len(pcalls)
+            "gpu_launches": args.steps * launches_per_step * 2 + args.steps * 5 * len(pcalls)
                             + stack_launches,
             "clocks": clk.summary(),
             "gemm": gemm,
@@ -574,8 +590,11 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
-    ap.add_argument("--only", choices=["all", "decode"], default="all",
-                    help="decode: skip the prefill GEMM part (small profiling runs)")
+    ap.add_argument("--only", choices=["all", "decode", "mlp"], default="all",
+                    help="decode: skip everything after the decode sweep; mlp: decode sweep "
+                         "and the MLP gate/up + SwiGLU part only (small profiling runs)")
+    ap.add_argument("--mlp-m", default="",
+                    help="comma-separated token counts of the MLP part (default: all listed)")
     ap.add_argument("--replicas", type=int, default=0,
                     help="weight replicas per decode step (0: enough to exceed 2x L2)")
     ap.add_argument("--prefill-m", type=int, default=PREFILL_M,
