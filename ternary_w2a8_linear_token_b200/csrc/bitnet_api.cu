@@ -119,6 +119,18 @@ bitnet_status run_batch(const uint16_t* x_bf16, const int8_t* q_in, int64_t M, i
             p.total_rows = rows / 2;
             p.proj[0].N = rows / 2;
         }
+        // One token and a matrix too large for one wave of the register-resident kernel:
+        // stream it through a shared-memory ring instead.
+        int64_t n_stages = 0;
+        int depth = 0;
+        uint32_t stage_bytes = 0;
+        if (rows * (K / 4) >= kStreamMinBytes &&
+            gemv_stream_plan(p, &n_stages, &depth, &stage_bytes)) {
+            int32_t* err = device_error_word();
+            if (!err) return BITNET_ERR_CUDA;
+            return from_cuda(launch_gemv_stream(p, n_stages, depth, stage_bytes, tc_num_sms(),
+                                                err, stream, /*pdl=*/true));
+        }
         return from_cuda(launch_gemv(p, stream, /*pdl=*/true));
     }
 

@@ -116,6 +116,17 @@ __device__ __forceinline__ void tma_load_2d(void* smem_dst, const void* tmap, ui
         : "memory");
 }
 
+// Untiled bulk copy global -> shared of `bytes` (a multiple of 16; both addresses 16-byte
+// aligned), completion counted on `bar`. No multicast.
+__device__ __forceinline__ void bulk_load_1d(void* smem_dst, const void* gsrc, uint32_t bytes,
+                                             uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+        ::"r"(smem_addr(smem_dst)), "l"(reinterpret_cast<uint64_t>(gsrc)), "r"(bytes),
+        "r"(smem_addr(bar))
+        : "memory");
+}
+
 // 2-D tiled TMA store shared -> global, tracked by this thread's bulk async-groups. The
 // tensor map clips the box at the tensor bounds, so ragged edges need no masking.
 __device__ __forceinline__ void tma_store_2d(const void* tmap, const void* smem_src, int32_t x,

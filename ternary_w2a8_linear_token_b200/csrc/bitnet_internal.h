@@ -72,6 +72,16 @@ struct GemvParams {
 cudaError_t launch_gemv(const GemvParams& p, cudaStream_t stream, bool pdl);
 bool gemv_supported(int64_t M, int64_t K);
 
+// Streaming GEMV for one token and large matrices (a producer warp fills a shared-memory
+// ring of 16-row weight stages with bulk copies; one CTA per SM). gemv_stream_plan returns
+// false where it does not apply (M != 1, contraction-only input, K > 16384, or a ring of
+// fewer than two stages). Used from kStreamMinBytes of packed weights per call.
+constexpr int64_t kStreamMinBytes = int64_t(6) << 20;
+bool gemv_stream_plan(const GemvParams& p, int64_t* n_stages, int* depth, uint32_t* stage_bytes);
+cudaError_t launch_gemv_stream(const GemvParams& p, int64_t n_stages, int depth,
+                               uint32_t stage_bytes, int sms, int32_t* err, cudaStream_t stream,
+                               bool pdl);
+
 // ----------------------------------------------------------------------------- quantisation
 // mode 0: natural-order q (public bitnet_quant_act); mode 1: permuted q + s_x + r_x for
 // the tensor-core path. q_in != nullptr: copy-permute given int8 q (no scales).

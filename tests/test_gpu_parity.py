@@ -257,3 +257,45 @@ def test_8b_stack_projection_sampled(bn, oracle):
                                    m_idx, n_idx)
     got = bits_from_bf16_tensor(y)[np.ix_(m_idx, n_idx)]
     assert_bf16_within_1ulp(got, ref["y"], oracle, "8b down")
+
+
+# One token and at least 6 MB of packed weights per call: the streaming GEMV (producer warp,
+# shared-memory ring of 16-row stages). Ragged projections (N not a multiple of 16), every
+# chunks-per-lane class, per-row scales, fp32 output, whole outputs against the oracle.
+STREAM_CASES = [  # (Ns of the batch, K, per_row)
+    ((2560, 640, 640, 6912, 6912), 2560, False),  # the 2B-4T layer's batched projections
+    ((4096, 14336 + 7), 4096, True),              # ragged last stage
+    ((4096,), 14336, True),                       # 8B down projection, K = 14336
+    ((9001,), 6912, False),                       # 4 chunks per lane, ragged
+    ((3000, 30011), 1024, True),                  # 1 chunk per lane
+]
+
+
+@pytest.mark.parametrize("Ns,K,per_row", STREAM_CASES)
+def test_stream_gemv_matches_oracle(bn, oracle, Ns, K, per_row):
+    assert sum(Ns) * K // 4 >= 6 << 20
+    g = synth.rng(0, 99, len(Ns), K, synth.KIND_T)
+    x = synth.normal_x(1, K, g)
+    projs, refs = [], []
+    for N in Ns:
+        t = synth.ternary(N, K, g, 0.4)
+        s_w = synth.uniform_scale(N if per_row else 1, g)
+        packed = _packed_dev(oracle, t)
+        projs.append((packed, torch.from_numpy(s_w).cuda(), per_row))
+        refs.append(oracle.bitlinear(x, packed.cpu().numpy(), s_w, per_row, K)["y"])
+    xd = bf16_tensor_from_bits(x)
+    for dtype in (torch.bfloat16, torch.float32):
+        ys = bn.bitnet_linear_batch(xd, projs, out_dtype=dtype)
+        for y, ref, N in zip(ys, refs, Ns):
+            _check_y(y, ref, oracle, f"stream N={N} K={K} {dtype}")
+
+
+def test_stream_gemv_i32_contraction(bn, oracle):
+    """The contraction-only call keeps the register-resident kernel (no quantiser there)."""
+    N, K = 6000, 4096
+    g = synth.rng(0, 99, 7, K, synth.KIND_T)
+    t = synth.ternary(N, K, g, 0.4)
+    q = g.integers(-127, 128, size=(1, K)).astype(np.int8)
+    packed = _packed_dev(oracle, t)
+    acc = bn.bitnet_linear_i32(torch.from_numpy(q).cuda(), packed, path=bn.PATH_GEMV)
+    assert np.array_equal(acc.cpu().numpy(), oracle.ternary_matmul(q, t))

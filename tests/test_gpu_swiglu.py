@@ -161,3 +161,19 @@ def test_swiglu_8b_mlp_per_row_sampled(bn, oracle):
     ref = oracle.swiglu_gate_up_sampled(x, pg, sg, pu, su, True, 4096, m_idx, n_idx)
     got = bits_from_bf16_tensor(h)[np.ix_(m_idx, n_idx)]
     assert_swiglu_within_bound(got, ref, oracle, where="8B M=128")
+
+
+def test_swiglu_8b_mlp_decode_stream(bn, oracle):
+    """8B-class MLP gate/up at M = 1 (29 MB interleaved, the streaming GEMV), per-row scales,
+    every output."""
+    Wg = synth.stack8b_latent(0, "gate")
+    Wu = synth.stack8b_latent(0, "up")
+    pg, sg = oracle.pack_weights(Wg, True)
+    pu, su = oracle.pack_weights(Wu, True)
+    dev = lambda a: torch.from_numpy(a).cuda()
+    packed_gu, s_gu = bn.bitnet_interleave_gate_up(dev(pg), dev(sg), dev(pu), dev(su), True)
+    x = synth.stack8b_x(1, 4096)
+    h = bn.bitnet_linear_swiglu(bf16_tensor_from_bits(x), packed_gu, s_gu, True)
+    torch.cuda.synchronize()
+    ref = oracle.swiglu_gate_up(x, pg, sg, pu, su, True, 4096)
+    assert_swiglu_within_bound(bits_from_bf16_tensor(h), ref, oracle, where="8B decode")
