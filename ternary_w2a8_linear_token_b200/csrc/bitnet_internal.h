@@ -75,8 +75,10 @@ bool gemv_supported(int64_t M, int64_t K);
 // Streaming GEMV for one token and large matrices (a producer warp fills a shared-memory
 // ring of 16-row weight stages with bulk copies; one CTA per SM). gemv_stream_plan returns
 // false where it does not apply (M != 1, contraction-only input, K > 16384, or a ring of
-// fewer than two stages). Used from kStreamMinBytes of packed weights per call.
-constexpr int64_t kStreamMinBytes = int64_t(6) << 20;
+// fewer than two stages). Used from kStreamMinBytes of packed weights per call: below that
+// (measured on B200 in chains of calls) the register-resident kernel wins, because its
+// grid leaves room for the next call's CTAs to start their weight loads early.
+constexpr int64_t kStreamMinBytes = int64_t(12) << 20;
 bool gemv_stream_plan(const GemvParams& p, int64_t* n_stages, int* depth, uint32_t* stage_bytes);
 cudaError_t launch_gemv_stream(const GemvParams& p, int64_t n_stages, int depth,
                                uint32_t stage_bytes, int sms, int32_t* err, cudaStream_t stream,
