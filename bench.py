@@ -43,6 +43,12 @@ PREFILL_M = 2048
 INT8_PER_BF16 = 2.0
 
 
+# DRAM bytes per decode-sweep GEMV launch, read + write, from one ncu capture of the four
+# shapes (2560 x 2560, 640 x 2560, 6912 x 2560, 2560 x 6912 at M = 1: 1662976, 430336,
+# 4447744, 4455168 bytes), averaged; the kernel has not changed since.
+GEMV_DECODE_TRAFFIC_BYTES = 2749056
+
+
 def decode_bytes(M, N, K):
     """Algorithmic bytes of one BitLinear call: packed W + x + y + s_w (per tensor)."""
     return N * K // 4 + 2 * M * K + 2 * M * N + 4
@@ -82,7 +88,8 @@ def reduce_over_ranks(local_ms: float, local_units: float, world: int):
 
 # ---------------------------------------------------------------------------- clocks
 class ClockSampler:
-    """Samples SM clock and clock-event reasons through NVML (read-only) every 50 ms."""
+    """Samples SM clock and clock-event reasons through NVML (read-only) every 5 ms while
+    `active` is set; timed_steps sets it around every timed region."""
 
     REASONS = {"hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
                "sw_power_cap": 0x4}
@@ -91,6 +98,8 @@ class ClockSampler:
         self.index = index
         self.samples, self.reasons, self.max_mhz = [], set(), None
         self._stop = None
+        import threading
+        self.active = threading.Event()
 
     def _run(self):
         import pynvml
@@ -99,12 +108,14 @@ class ClockSampler:
             h = pynvml.nvmlDeviceGetHandleByIndex(self.index)
             self.max_mhz = float(pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM))
             while not self._stop.is_set():
-                self.samples.append(float(pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)))
-                bits = pynvml.nvmlDeviceGetCurrentClocksThrottleReasons(h)
-                for name, bit in self.REASONS.items():
-                    if bits & bit:
-                        self.reasons.add(name)
-                self._stop.wait(0.05)
+                if self.active.is_set():
+                    self.samples.append(
+                        float(pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)))
+                    bits = pynvml.nvmlDeviceGetCurrentClocksThrottleReasons(h)
+                    for name, bit in self.REASONS.items():
+                        if bits & bit:
+                            self.reasons.add(name)
+                self._stop.wait(0.005)
         except Exception as e:  # sampling is best effort; the line says so
             self.error = repr(e)
 
@@ -326,6 +337,9 @@ def capture(torch, fn):
     return g
 
 
+_CLOCKS = None  # the run's ClockSampler; timed regions switch its sampling on
+
+
 def timed_steps(torch, step_fn, steps, warmup, flush_buf, world):
     import torch.distributed as dist
     for _ in range(warmup):
@@ -337,12 +351,16 @@ def timed_steps(torch, step_fn, steps, warmup, flush_buf, world):
     torch.cuda.synchronize()
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
           for _ in range(steps)]
+    if _CLOCKS is not None:
+        _CLOCKS.active.set()
     for a, b in ev:
         flush_buf.add_(1)  # evict L2 (outside the step's events)
         a.record()
         step_fn()
         b.record()
     torch.cuda.synchronize()
+    if _CLOCKS is not None:
+        _CLOCKS.active.clear()
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
@@ -433,8 +451,10 @@ def run_ours(args):
     launches_per_step = len(calls)
     step_bytes = sum(decode_bytes(DECODE_M, c["N"], c["K"]) for c in calls)
     g_dec = capture(torch, lambda: run_calls(bn, calls))
-    with ClockSampler(local) as clk:
-        dec_ms = timed_steps(torch, g_dec.replay, args.steps, args.warmup, flush, world)
+    global _CLOCKS
+    clk = ClockSampler(local).__enter__()  # samples inside every timed region below
+    _CLOCKS = clk
+    dec_ms = timed_steps(torch, g_dec.replay, args.steps, args.warmup, flush, world)
     assert bn.bitnet_check_device_errors() == 0
     dec_ms_max, total_bytes = reduce_over_ranks(dec_ms, step_bytes * args.steps, world)
     gbs = total_bytes / (dec_ms_max * 1e-3) / 1e9
@@ -540,6 +560,9 @@ def run_ours(args):
             del lw
             torch.cuda.empty_cache()
 
+    clk.__exit__(None, None, None)
+    _CLOCKS = None
+
     cpu = oracle_sample(args.cpu_seconds) if (rank == 0 and world == 1 and args.cpu_seconds > 0) \
         else None
 
@@ -562,8 +585,12 @@ def run_ours(args):
             },
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"],
                          "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
-                         "traffic": None, "peak_src": peaks["src"],
-                         "kernel": "gemv_w2a8_kernel"},
+                         "traffic": GEMV_DECODE_TRAFFIC_BYTES,
+                         "traffic_src": "ncu dram__bytes_read.sum + dram__bytes_write.sum per "
+                                        "launch, mean over the four decode-sweep shapes "
+                                        "(profiles/gemv_w2a8_decode_m1.md)",
+                         "algorithmic_bytes_per_launch": per_launch_bytes,
+                         "peak_src": peaks["src"], "kernel": "gemv_w2a8_kernel"},
             "e2e": {"value": e2e_gbs, "unit": "GB/s",
                     "h2d_bytes_per_step": int(h_x.numel() * 2),
                     "d2h_bytes_per_step": int(h_y.numel() * 2)},
