@@ -587,8 +587,8 @@ def run_ours(args):
                          "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
                          "traffic": GEMV_DECODE_TRAFFIC_BYTES,
                          "traffic_src": "ncu dram__bytes_read.sum + dram__bytes_write.sum per "
-                                        "launch, mean over the four decode-sweep shapes "
-                                        "(profiles/gemv_w2a8_decode_m1.md)",
+                                        "launch, one capture of the four decode-sweep shapes, "
+                                        "mean",
                          "algorithmic_bytes_per_launch": per_launch_bytes,
                          "peak_src": peaks["src"], "kernel": "gemv_w2a8_kernel"},
             "e2e": {"value": e2e_gbs, "unit": "GB/s",
