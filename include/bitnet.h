@@ -135,7 +135,8 @@ bitnet_status bitnet_quant_act_ex(const uint16_t* x, int64_t M, int64_t K, bitne
 
 /*
  * Workspace bytes the tensor-core path of bitnet_linear / bitnet_linear_batch needs for
- * M tokens of width K (quantised activations and per-token scales). The GEMV path uses
+ * M tokens of width K (quantised activations, per-token scales, the partial maxima of a
+ * per-tensor activation scale, and room for split-K partial tiles). The GEMV path uses
  * none: under BITNET_PATH_AUTO, calls with M <= BITNET_GEMV_MAX_M may pass workspace =
  * NULL and then run the GEMV (for 5 <= M <= 8 a sufficient workspace selects the faster
  * tensor-core path instead).
