@@ -11,16 +11,16 @@
 // token tile of up to 192 tokens.
 //
 // The unpacked weights go from registers straight into TMEM and feed the MMA as its A
-// operand from there. The main loop is bound by shared-memory traffic (TMA writes plus the
-// tensor core's operand reads, measured on B200), and this keeps the weight operand out
-// of shared memory altogether; TMEM then holds two accumulators and a 4-stage weight ring,
-// which caps the token tile at 192.
+// operand from there, so the weight operand never takes a shared-memory round trip (on B200
+// this removed the unpack warps' shared-memory stores and the tensor core's reads of them
+// from the main loop); TMEM holds two accumulators and a weight ring of 2 (BN = 192), 3
+// (BN = 160) or 4 stages, which caps the token tile at 192.
 //
 // One CTA per SM walks a static list of 128 x BN output tiles. Two shared-memory rings and
 // the TMEM weight ring decouple the stages of the main loop, and two TMEM accumulators let
 // the epilogue of one tile overlap the main loop of the next:
 //  warp 0      TMEM allocation; lane 0 loads token tiles (two BN-row x 128-byte boxes per
-//              256-byte K stage, 128-byte swizzle) into ring B with TMA;
+//              256-byte K stage, 128-byte swizzle, no multicast) into ring B with TMA;
 //  warps 1, 19 lane 0 of each issues 8 tcgen05.mma.kind::i8 (K = 32 each) per 256-byte K
 //              stage, the two threads taking alternate stages, and commits them to the A/B
 //              slots they read and, per tile, to the accumulator (barrier round trips of a
@@ -30,13 +30,16 @@
 //              ring P with TMA;
 //  warps 3-10  epilogue, two warps per TMEM lane quarter splitting the columns; they zero
 //              each accumulator as they read it (every MMA accumulates): TMEM ->
-//              registers -> y = acc * (s_w * 1/s_x) -> a per-warp staging tile in shared
-//              memory -> TMA store (the tensor map clips ragged edges); the dequantisation
-//              factors of the tile's tokens sit in a shared table filled before the
-//              accumulator is ready, and the accumulator goes back to the MMA warp as soon
-//              as its last columns are in registers;
-//  warps 11-18 unpack ring P into the TMEM weight ring: codes - 1 per byte, one row per
-//              TMEM lane, four K bytes per column.
+//              registers -> acc = D - sum_k q -> y = acc * (s_w * 1/s_x) -> a per-warp
+//              staging tile in shared memory -> TMA store (the tensor map clips ragged
+//              edges); the dequantisation factors and sum_k q of the tile's tokens sit in a
+//              shared table filled before the accumulator is ready, and the accumulator goes
+//              back to the MMA warps as soon as its last columns are in registers. For the
+//              MLP's interleaved gate/up matrix the epilogue instead pairs lanes l and l + 16
+//              (gate and up rows of one output) and stores h = SwiGLU(g, u);
+//  warps 11-18 unpack ring P into the TMEM weight ring: the codes t + 1 themselves (the
+//              MMA's A operand is unsigned; the epilogue removes sum_k q), one row per TMEM
+//              lane, four K bytes per column.
 // The token tile arrives in the permuted in-group K order produced by the quantiser, which
 // is the order a packed word unpacks into with shifts and masks alone.
 //
