@@ -3,8 +3,12 @@
 // framework ops; page "BitNet 1-bit LLM推理优化", section 3.2 "激活量化策略").
 //   amax = max_k |x[m,k]|, s_x = 127 / max(amax, 1e-5), q = clamp(rint(x * s_x), -128, 127).
 //
-// One warp per token. Pass 1 reduces amax over the bf16 bit patterns (|x| ordered as an
-// unsigned integer), pass 2 re-reads x (an L1/L2 hit) and writes q. Two output layouts:
+// amax is reduced over the bf16 bit patterns (|x| ordered as an unsigned integer, so it is
+// exact). Rows of K <= 4096 take one warp each and stay in registers (x read once); rows of
+// 4096 < K <= 14336 take four warps each, also in registers; longer rows take one warp and
+// two passes (the second an L1/L2 hit). With a per-tensor scale ("BitNet 1-bit LLM推理优化"
+// section 2.2, I2_S), amax_parts_kernel first writes partial maxima of the whole input and
+// every warp reduces those instead of its row. Two output layouts:
 //  - natural (M, K) int8, the public bitnet_quant_act result;
 //  - permuted, the operand layout of the tensor-core path: inside every group of 16
 //    values along K, byte 4i + b holds k = 4b + i. That is the order in which a packed
