@@ -39,6 +39,7 @@ METRIC = "W2A8 ternary GEMV HBM GB/s (M=1) and GEMM int8 TOPS (M>=512) vs roofli
 L2_BYTES = 126 * 1024 * 1024
 DECODE_M = 1
 PREFILL_M = 2048
+PREFILL_M_SMALL = 512  # the prefill configuration's other token count
 # nominal dense int8 : bf16 tensor-core ratio on B200 (4.5 vs 2.25 PFLOP/s)
 INT8_PER_BF16 = 2.0
 
@@ -528,6 +529,19 @@ def run_ours(args):
         gemm["act_per_tensor"] = {"value": pt_ops / (pt_ms_max * 1e-3) / 1e12, "unit": "TOPS",
                                   "ms_per_step": pt_ms_max / args.steps}
         del g_pt
+        # the prefill configuration's other token count
+        if args.prefill_m != PREFILL_M_SMALL:
+            scalls = build_prefill(bn, torch, dev, PREFILL_M_SMALL)
+            g_s = capture(torch, lambda: run_calls(bn, scalls))
+            s_ms = timed_steps(torch, g_s.replay, args.steps, args.warmup, flush, world)
+            assert bn.bitnet_check_device_errors() == 0
+            s_ops_step = sum(2.0 * PREFILL_M_SMALL * c["N"] * c["K"] for c in scalls)
+            s_ms_max, s_ops = reduce_over_ranks(s_ms, s_ops_step * args.steps, world)
+            s_tops = s_ops / (s_ms_max * 1e-3) / 1e12
+            gemm[f"m{PREFILL_M_SMALL}"] = {"value": s_tops, "unit": "TOPS",
+                                           "ms_per_step": s_ms_max / args.steps,
+                                           "frac": s_tops / int8_peak}
+            del g_s, scalls
 
     # ---------------- layer stacks (2B-4T and 8B-class, every layer back to back)
     stacks = []
@@ -594,7 +608,7 @@ def run_ours(args):
             "e2e": {"value": e2e_gbs, "unit": "GB/s",
                     "h2d_bytes_per_step": int(h_x.numel() * 2),
                     "d2h_bytes_per_step": int(h_y.numel() * 2)},
-            "gpu_launches": args.steps * launches_per_step * 2 + args.steps * 5 * len(pcalls)
+            "gpu_launches": args.steps * launches_per_step * 2 + args.steps * 7 * len(pcalls)
                             + stack_launches,
             "clocks": clk.summary(),
             "gemm": gemm,
