@@ -59,7 +59,6 @@ namespace bitnet {
 namespace {
 
 constexpr int kBM = 128;  // weight rows per tile (MMA M)
-constexpr int kBK = 256;   // K bytes per stage: 8 MMAs between barrier round trips
 constexpr int kSub = 128;  // K bytes per token sub-tile (TMA box width, 128-byte swizzle atom)
 constexpr int kWarpB = 0, kWarpMma = 1, kWarpP = 2, kEpiWarp0 = 3, kEpiWarps = 8,
               kUnpWarp0 = 11, kUnpWarps = 8, kWarpMma2 = 19;
@@ -70,8 +69,13 @@ constexpr int kHalfCols = 16;                           // columns per epilogue 
 
 template <int BN>
 struct TcLayout {
+    // K bytes per stage: 8 MMAs between barrier round trips, 16 for token tiles of at most
+    // 32, where the round trip rather than the MMAs sets the stage's pace (measured on B200).
+    static constexpr int kBK = BN <= 32 ? 512 : 256;
     static constexpr int kB = BN * kBK;       // token tile: kBK / kSub sub-tiles of BN x kSub
-    static constexpr int kP = kBM * kBK / 4;  // packed weights, 8 KB
+    static constexpr int kP = kBM * kBK / 4;  // packed weights, 8 or 16 KB
+    static constexpr int kPBoxes = kBK / 256;        // 64-byte-wide packed TMA boxes per stage
+    static constexpr int kChunksPerWarp = kBK / 128; // 16-byte packed chunks per unpack warp
     // Ring depths. The unpacked weights live in TMEM (kDA stages of 64 columns), so shared
     // memory carries only the token and packed-weight rings and the epilogue staging.
     // The two MMA issuers take the global K stages by parity. The token ring has an even
@@ -80,7 +84,7 @@ struct TcLayout {
     // fill has not landed (a parity wait cannot tell the two phases apart). The weight ring
     // needs no such rule: the unpack warps arrive in stage order, so when an issuer has
     // consumed its previous stage g - 2, every stage up to g - 2 >= g - kDA has completed.
-    static constexpr int kDA = BN > 160 ? 2 : BN > 128 ? 3 : 4;
+    static constexpr int kDA = BN > 160 ? 2 : BN > 128 ? 3 : kBK == 512 ? 3 : 4;
     static constexpr int kDB = BN > 64 ? 4 : 6;
     static constexpr int kDP = BN > 160 ? 2 : 4;
     static_assert(kDB % 2 == 0, "one issuer per token-ring slot");
@@ -132,11 +136,7 @@ struct TileCoord {
     int kt0;  // first K stage of the tile's main loop
 };
 
-__device__ __forceinline__ int num_k_of(const TcParams& p) {
-    return static_cast<int>((p.K + kBK - 1) / kBK);
-}
-
-__device__ __forceinline__ TileCoord tile_coord(const TcParams& p, int t, int bn) {
+__device__ __forceinline__ TileCoord tile_coord(const TcParams& p, int t, int bn, int num_k) {
     const int nt = t % p.n_tiles_total;
     TileCoord c;
     c.proj = 0;
@@ -148,7 +148,7 @@ __device__ __forceinline__ TileCoord tile_coord(const TcParams& p, int t, int bn
     // Tiles that share a token tile run at the same time on different SMs; starting their K
     // loops at different stages spreads their reads of that tile over L2. The int32 sum is
     // exact, so the order of the K stages does not change the result.
-    c.kt0 = static_cast<int>((int64_t(nt) * 7) % num_k_of(p));
+    c.kt0 = static_cast<int>((int64_t(nt) * 7) % num_k);
     return c;
 }
 
@@ -308,7 +308,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int num_k = static_cast<int>((p.K + kBK - 1) / kBK);
+    const int num_k = static_cast<int>((p.K + L::kBK - 1) / L::kBK);
     const int m_tiles = (p.M + BN - 1) / BN;
     const int num_tiles = m_tiles * p.n_tiles_total;
     const int splits = p.splits;
@@ -354,15 +354,15 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
             int kc = 0;
             for (int u = blockIdx.x; u < num_units; u += gridDim.x) {
                 const Unit w = unit_of(u, splits, num_k);
-                const TileCoord tc = tile_coord(p, w.t, BN);
+                const TileCoord tc = tile_coord(p, w.t, BN, num_k);
                 for (int kt = 0; kt < w.ns; ++kt, ++kc, rb.next()) {
                     mbar_wait_bounded(&b_empty[rb.slot], rb.phase ^ 1, p.err, kErrWaitEmpty, abort_flag);
                     mbar_arrive_expect_tx(&b_full[rb.slot], L::kB);
                     const int kr = stage_k(w, tc, kt, splits, num_k);
 #pragma unroll
-                    for (int h = 0; h < kBK / kSub; ++h)
+                    for (int h = 0; h < L::kBK / kSub; ++h)
                         tma_load_2d(smem + L::kOffB + rb.slot * L::kB + h * BN * kSub, &p.tmap_q,
-                                    &b_full[rb.slot], kr * kBK + h * kSub, tc.m0);
+                                    &b_full[rb.slot], kr * L::kBK + h * kSub, tc.m0);
                 }
             }
             for (int k = kc > L::kDB ? kc - L::kDB : 0; k < kc; ++k)  // drain
@@ -377,13 +377,16 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
             int kc = 0;
             for (int u = blockIdx.x; u < num_units; u += gridDim.x) {
                 const Unit w = unit_of(u, splits, num_k);
-                const TileCoord tc = tile_coord(p, w.t, BN);
+                const TileCoord tc = tile_coord(p, w.t, BN, num_k);
                 for (int kt = 0; kt < w.ns; ++kt, ++kc, rp.next()) {
                     mbar_wait_bounded(&p_empty[rp.slot], rp.phase ^ 1, p.err, kErrWaitEmpty, abort_flag);
                     mbar_arrive_expect_tx(&p_full[rp.slot], L::kP);
                     const int kr = stage_k(w, tc, kt, splits, num_k);
-                    tma_load_2d(smem + L::kOffP + rp.slot * L::kP, &p.tmap_w[tc.proj],
-                                &p_full[rp.slot], kr * (kBK / 4), tc.n0);
+#pragma unroll
+                    for (int b = 0; b < L::kPBoxes; ++b)  // 64-byte boxes, [box][row][64 bytes]
+                        tma_load_2d(smem + L::kOffP + rp.slot * L::kP + b * (kBM * 64),
+                                    &p.tmap_w[tc.proj], &p_full[rp.slot],
+                                    kr * (L::kBK / 4) + b * 64, tc.n0);
                 }
             }
             for (int k = kc > L::kDP ? kc - L::kDP : 0; k < kc; ++k)  // drain
@@ -422,7 +425,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
                     const uint32_t at = a_tmem0 + uint32_t(ra.slot) * L::kAStageCols;
                     const uint64_t bd = b_desc0 + uint64_t(rb.slot * (L::kB >> 4));
 #pragma unroll
-                    for (int kk = 0; kk < kBK / 32; ++kk) {
+                    for (int kk = 0; kk < L::kBK / 32; ++kk) {
                         const int h = kk / (kSub / 32), k32 = kk % (kSub / 32);
                         mma_i8_tmem_a(d, at + uint32_t(8 * kk),
                                       bd + uint64_t((h * BN * kSub) >> 4) + uint64_t(2 * k32), idesc,
@@ -453,31 +456,48 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
             const Unit w = unit_of(u, splits, num_k);
             for (int kt = 0; kt < w.ns; ++kt, rp.next(), ra.next()) {
                 mbar_wait_bounded(&p_full[rp.slot], rp.phase, p.err, kErrWaitTmaFull, abort_flag);
-                // The packed tile arrives with the 64-byte TMA swizzle: 16-byte chunk c of row r
-                // sits at chunk c ^ ((r >> 1) & 3), so the 32 lanes' reads (one row each) spread
-                // over all banks instead of four rows sharing each bank.
-                const uint8_t* prow = smem + L::kOffP + rp.slot * L::kP + row * (kBK / 4);
+                // The packed tile arrives in 64-byte-wide TMA boxes with the 64-byte swizzle:
+                // 16-byte chunk c of row r sits at chunk c ^ ((r >> 1) & 3) of its box, so the
+                // 32 lanes' reads (one row each) spread over all banks instead of four rows
+                // sharing each bank. This warp takes chunks kChunksPerWarp * half ... of the row.
+                const uint8_t* pslot = smem + L::kOffP + rp.slot * L::kP;
                 const int sw = (row >> 1) & 3;
-                const uint4 pk0 = *reinterpret_cast<const uint4*>(prow + (((2 * half) ^ sw) << 4));
-                const uint4 pk1 = *reinterpret_cast<const uint4*>(prow + (((2 * half + 1) ^ sw) << 4));
+                uint4 pk[L::kChunksPerWarp];
+#pragma unroll
+                for (int i = 0; i < L::kChunksPerWarp; ++i) {
+                    const int gc = L::kChunksPerWarp * half + i;  // chunk of the row's stage
+                    pk[i] = *reinterpret_cast<const uint4*>(pslot + (gc >> 2) * (kBM * 64) +
+                                                            row * 64 + (((gc & 3) ^ sw) << 4));
+                }
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&p_empty[rp.slot]);
                 // The MMA multiplies the codes c = t + 1 in {0, 1, 2} themselves (unsigned A
                 // operand); the epilogue removes sum_k q once per token (sum q t = sum q c -
                 // sum q). Packed word c holds 16 weights; its shifts by 0, 2, 4, 6 give the
                 // four 32-bit columns in the permuted in-group K order of the token operand.
-                const uint32_t words[8] = {pk0.x, pk0.y, pk0.z, pk0.w, pk1.x, pk1.y, pk1.z, pk1.w};
-                uint32_t t[32];
+                // Two chunks (8 words) fill 32 TMEM columns.
 #pragma unroll
-                for (int c = 0; c < 8; ++c) {
-                    t[4 * c + 0] = words[c] & 0x03030303u;
-                    t[4 * c + 1] = (words[c] >> 2) & 0x03030303u;
-                    t[4 * c + 2] = (words[c] >> 4) & 0x03030303u;
-                    t[4 * c + 3] = (words[c] >> 6) & 0x03030303u;
+                for (int g2 = 0; g2 < L::kChunksPerWarp / 2; ++g2) {
+                    const uint32_t words[8] = {pk[2 * g2].x,     pk[2 * g2].y,     pk[2 * g2].z,
+                                               pk[2 * g2].w,     pk[2 * g2 + 1].x, pk[2 * g2 + 1].y,
+                                               pk[2 * g2 + 1].z, pk[2 * g2 + 1].w};
+                    uint32_t t[32];
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) {
+                        t[4 * c + 0] = words[c] & 0x03030303u;
+                        t[4 * c + 1] = (words[c] >> 2) & 0x03030303u;
+                        t[4 * c + 2] = (words[c] >> 4) & 0x03030303u;
+                        t[4 * c + 3] = (words[c] >> 6) & 0x03030303u;
+                    }
+                    if (g2 == 0) {  // the ring slot must be free before the first store
+                        mbar_wait_bounded(&a_empty[ra.slot], ra.phase ^ 1, p.err, kErrWaitEmpty,
+                                          abort_flag);
+                        tc_fence_after();
+                    }
+                    tmem_st_32x32b_x32(a_lane + uint32_t(ra.slot) * L::kAStageCols +
+                                           uint32_t(32 * g2),
+                                       t);
                 }
-                mbar_wait_bounded(&a_empty[ra.slot], ra.phase ^ 1, p.err, kErrWaitEmpty, abort_flag);
-                tc_fence_after();
-                tmem_st_32x32b_x32(a_lane + uint32_t(ra.slot) * L::kAStageCols, t);
                 tmem_st_wait();
                 tc_fence_before();
                 __syncwarp();
@@ -526,7 +546,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
         int i = 0;
         for (int u = blockIdx.x; u < num_units; u += gridDim.x, ++i) {
             const Unit w = unit_of(u, splits, num_k);
-            const TileCoord tc = tile_coord(p, w.t, BN);
+            const TileCoord tc = tile_coord(p, w.t, BN, num_k);
             const TcProj& pr = p.proj[tc.proj];
             const int64_t n = int64_t(tc.n0) + n_local;
             const bool nvalid = n < pr.N;
