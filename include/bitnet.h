@@ -153,6 +153,9 @@ size_t bitnet_linear_workspace_size(int64_t M, int64_t K);
  *   workspace, workspace_bytes: device scratch of at least bitnet_linear_workspace_size(M, K)
  *            bytes when the tensor-core path runs (M > BITNET_GEMV_AUTO_M); its contents
  *            on entry are ignored, and it must not be shared by calls that may overlap.
+ * Kernels, chosen per call (results identical): the dp4a GEMV with the quantiser fused for
+ * few tokens (a shared-memory streaming variant at one token and >= 12 MiB of packed weights
+ * per call), otherwise the quantiser followed by the tcgen05 GEMM.
  * Epilogue arithmetic: acc = exact int32 sum; r = 1/s_x[m] (binary32, rounded);
  * y = (float)acc * (s_w[n or 0] * r), each product rounded; bf16 is RNE of that fp32
  * value. The result differs from the exact acc * s_w / s_x by at most 3 binary32
