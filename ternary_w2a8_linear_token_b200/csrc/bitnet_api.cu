@@ -224,8 +224,8 @@ bitnet_status run_batch(const uint16_t* x_bf16, const int8_t* q_in, int64_t M, i
     // each tile's K range is cut into `splits` units (at least 512 K bytes each) so that about
     // one unit runs per SM; units add their int32 partial tiles into a zeroed accumulation tile.
     p.splits = 1;
-    // K stages of the kernel: 512 bytes for token tiles of at most 32, else 256 bytes.
-    const int64_t kstage = bn <= 32 ? 512 : 256;
+    // K stages of the kernel: 512 bytes for token tiles of at most 64, else 256 bytes.
+    const int64_t kstage = bn <= 64 ? 512 : 256;
     const int64_t num_k = (K + kstage - 1) / kstage;
     const int64_t m_tiles = (M + bn - 1) / bn;
     const int64_t tiles_all = m_tiles * tiles;
@@ -234,7 +234,7 @@ bitnet_status run_batch(const uint16_t* x_bf16, const int8_t* q_in, int64_t M, i
     // Measured on B200: splitting pays for token tiles of up to 32, and of 64 with long K
     // loops; for wider tiles the atomic reduction of the partial tiles costs more than the
     // shorter main loop saves.
-    const bool split_pays = !swiglu && (bn <= 32 || (bn == 64 && num_k >= 16));
+    const bool split_pays = !swiglu && (bn <= 32 || (bn == 64 && K >= 4096));
     const int64_t unit_stages = 512 / kstage;  // a split unit spans at least 512 K bytes
     if (split_pays && tiles_all * 4 <= sms && tiles_all <= kMaxSplitTiles &&
         num_k >= 2 * unit_stages && workspace_bytes >= ws_total_bytes(M, K) + ws_split_bytes(M)) {

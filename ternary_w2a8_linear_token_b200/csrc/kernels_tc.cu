@@ -70,8 +70,8 @@ constexpr int kHalfCols = 16;                           // columns per epilogue 
 template <int BN>
 struct TcLayout {
     // K bytes per stage: 8 MMAs between barrier round trips, 16 for token tiles of at most
-    // 32, where the round trip rather than the MMAs sets the stage's pace (measured on B200).
-    static constexpr int kBK = BN <= 32 ? 512 : 256;
+    // 64, where the round trip rather than the MMAs sets the stage's pace (measured on B200).
+    static constexpr int kBK = BN <= 64 ? 512 : 256;
     static constexpr int kB = BN * kBK;       // token tile: kBK / kSub sub-tiles of BN x kSub
     static constexpr int kP = kBM * kBK / 4;  // packed weights, 8 or 16 KB
     static constexpr int kPBoxes = kBK / 256;        // 64-byte-wide packed TMA boxes per stage
@@ -85,7 +85,7 @@ struct TcLayout {
     // needs no such rule: the unpack warps arrive in stage order, so when an issuer has
     // consumed its previous stage g - 2, every stage up to g - 2 >= g - kDA has completed.
     static constexpr int kDA = BN > 160 ? 2 : BN > 128 ? 3 : kBK == 512 ? 3 : 4;
-    static constexpr int kDB = BN > 64 ? 4 : 6;
+    static constexpr int kDB = BN > 32 ? 4 : 6;
     static constexpr int kDP = BN > 160 ? 2 : 4;
     static_assert(kDB % 2 == 0, "one issuer per token-ring slot");
     static constexpr int kStage = 2048;  // per epilogue warp: 32 rows x 16 tokens x 4 bytes
