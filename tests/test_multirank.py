@@ -53,3 +53,21 @@ def test_two_rank_max_time_sum_work():
 def test_single_rank_is_identity():
     import bench
     assert bench.reduce_over_ranks(3.5, 7.0, 1) == (3.5, 7.0)
+
+
+def test_bench_reference_arm_json_line():
+    """`bench.py --impl reference` (the CPU oracle on the decode sweep) prints one JSON line
+    with the fields the driver reads, on rank 0, without a GPU."""
+    import json
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    out = subprocess.run([sys.executable, os.path.join(root, "bench.py"), "--impl", "reference",
+                          "--steps", "1", "--warmup", "3"], capture_output=True, text=True,
+                         timeout=300, cwd=root)
+    assert out.returncode == 0, out.stderr[-2000:]
+    line = json.loads(out.stdout.strip().splitlines()[-1])
+    assert line["impl"] == "reference" and line["unit"] == "GB/s" and line["value"] > 0
+    assert line["higher_is_better"] is True and line["steps"] == 1 and line["warmup"] == 3
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] >= 1
+    assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["value"] == line["value"]
