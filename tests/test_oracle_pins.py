@@ -427,6 +427,36 @@ def test_swiglu_gate_up_end_to_end_exact(oracle):
             assert int(r["h_bits"][m, n]) == _rne_bf16(_bf16_value(sb) * _bf16_value(ub))
 
 
+@pytest.mark.parametrize("per_row", [False, True])
+def test_swiglu_gate_up_sampled_equals_full_on_its_sample(oracle, per_row):
+    """The sampled MLP gate/up (used by the full-size GPU tests) against the whole-matrix
+    form on a tiny MLP: every g, u, s and h of the sample must match exactly. The gate and
+    up scales differ (per tensor and per row), and the sample has more outputs than tokens
+    in an unsorted order, so swapped scales or a swapped token/output index fail here."""
+    rng = np.random.default_rng(23)
+    M, I, K = 5, 48, 128
+    x = synth.to_bf16_bits(rng.normal(0, 1, (M, K)).astype(np.float32))
+    tg = rng.integers(-1, 2, (I, K)).astype(np.int8)
+    tu = rng.integers(-1, 2, (I, K)).astype(np.int8)
+    if per_row:
+        sg = rng.uniform(0.5, 2.0, I).astype(np.float32)
+        su = rng.uniform(3.0, 5.0, I).astype(np.float32)
+    else:
+        sg = np.array([0.625], dtype=np.float32)
+        su = np.array([3.5], dtype=np.float32)
+    pg, pu = oracle.pack(tg), oracle.pack(tu)
+    full = oracle.swiglu_gate_up(x, pg, sg, pu, su, per_row, K)
+    m_idx, n_idx = np.array([4, 0, 2]), np.array([47, 3, 20, 0, 31, 9, 46])
+    smp = oracle.swiglu_gate_up_sampled(x, pg, sg, pu, su, per_row, K, m_idx, n_idx)
+    sel = np.ix_(m_idx, n_idx)
+    for key in ("g", "u", "g_bits", "u_bits", "s_bits", "h_bits"):
+        assert smp[key].shape == (3, 7), key
+        assert np.array_equal(smp[key], full[key][sel]), key
+    # the sample is not degenerate: gate and up differ, and h is not all zero
+    assert not np.array_equal(smp["g_bits"], smp["u_bits"])
+    assert np.count_nonzero(smp["h_bits"] & 0x7FFF) > 10
+
+
 def test_swiglu_bound_helper_accepts_exact_and_rejects_far(oracle):
     """The GPU tests' SwiGLU bound: the oracle's own h passes; h moved 3 bf16 steps away
     from a value whose neighbourhood is flat fails."""
