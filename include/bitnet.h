@@ -28,9 +28,13 @@
  *  - NaN or Inf in x or W give unspecified (but memory-safe) results.
  *  - Rounding: every float step is IEEE binary32 round-to-nearest-even, with no
  *    contraction into FMA where the order below is stated.
- *  - Thread safety: calls may be made from several host threads. The library
- *    holds one piece of device state, the watchdog word read by
- *    bitnet_check_device_errors().
+ *  - Thread safety: calls may be made from several host threads. The library holds two
+ *    pieces of device state per device: the watchdog word read by
+ *    bitnet_check_device_errors(), and the fixed scratch array of bitnet_linear_noalloc
+ *    (the only call that uses it). Their device addresses are looked up on first use on
+ *    each device and cached, so the library must not be used on a device again after
+ *    cudaDeviceReset of that device. Every other call keeps its scratch in the caller's
+ *    workspace.
  */
 #ifndef BITNET_H
 #define BITNET_H
@@ -263,21 +267,23 @@ bitnet_status bitnet_linear_swiglu(const uint16_t* x, int64_t M, int64_t K,
 /*
  * bitnet_linear_noalloc — bitnet_linear for callers that cannot allocate device memory.
  * The pages have no counterpart to this call; it exists for callers such as a serving
- * loop in which cudaMalloc could synchronise the device and stall other streams, a plug-in
- * whose host runtime owns all device memory, or code running while its stream is captured
- * into a graph. It takes the same arguments as bitnet_linear minus the workspace: the
- * tensor-core path's scratch is a fixed device array of BITNET_NOALLOC_SCRATCH_BYTES inside
- * the library, which every GPU that loads the library holds until the process exits.
- *  - Sizes whose scratch (bitnet_linear_workspace_size(M, K)) exceeds that array are
- *    rejected with BITNET_ERR_WORKSPACE before anything is launched (M <= BITNET_GEMV_MAX_M
- *    runs the GEMV, which needs no scratch).
- *  - The first call on each device looks the array's address up (cudaGetSymbolAddress);
- *    make that first call before any stream capture on that device.
- *  - All calls share the one array and it keeps the last call's contents (nothing in it
- *    needs to start at zero). Calls that may overlap on the GPU — on different streams, or
- *    from different threads without ordering — race on it and give wrong results.
+ * loop in which cudaMalloc could synchronise the device and stall other streams, or a
+ * plug-in whose host runtime owns all device memory and forbids allocations of its own.
+ * It takes the same arguments as bitnet_linear minus the workspace: the tensor-core path's
+ * scratch is a fixed device array of BITNET_NOALLOC_SCRATCH_BYTES inside the library,
+ * which every GPU that loads the library holds until the process exits.
+ *  - Calls that run the tensor-core path (every M > BITNET_GEMV_AUTO_M, since the array
+ *    is always there to serve as the workspace) and whose bitnet_linear_workspace_size(M, K)
+ *    exceeds the array are rejected with BITNET_ERR_WORKSPACE before anything is launched.
+ *    M <= BITNET_GEMV_AUTO_M runs the GEMV, which needs no scratch.
+ *  - The first call on each device looks the array's address up (cudaGetSymbolAddress) and
+ *    caches it for the process; make that first call before any stream capture on that
+ *    device, and do not use the library on a device after cudaDeviceReset of it.
+ *  - All calls share the one array and it keeps the last call's contents (each call writes
+ *    or clears every part it reads). Calls that may overlap on the GPU — on different
+ *    streams, or from different threads without ordering — race on it and give wrong results.
  *  - It calls no cudaMalloc, cudaFree or allocating library routine.
- * Results equal bitnet_linear's bit for bit.
+ * Results equal bitnet_linear's bit for bit (the same kernels on the same inputs).
  */
 #define BITNET_NOALLOC_SCRATCH_BYTES (16 * 1024 * 1024)
 bitnet_status bitnet_linear_noalloc(const uint16_t* x, int64_t M, int64_t K,

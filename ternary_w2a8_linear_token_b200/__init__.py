@@ -125,6 +125,27 @@ def _x_ptr(x: torch.Tensor) -> int:
     return _dev(x, torch.int16, "x (bf16 bits)")
 
 
+def _check_proj(packed: torch.Tensor, s_w: torch.Tensor, per_row: bool, K: int,
+                name: str = "packed") -> int:
+    """Shape checks the C side cannot make (it sees only pointers): packed (N, K/4) and s_w
+    of N (per row) or 1 (per tensor) elements. Returns N."""
+    if packed.dim() != 2 or packed.shape[1] * 4 != K:
+        raise ValueError(f"{name} must be (N, K/4) = (N, {K // 4}), got {tuple(packed.shape)}")
+    N = packed.shape[0]
+    want = N if per_row else 1
+    if s_w.numel() != want:
+        raise ValueError(f"s_w must have {want} element(s) ({'per row' if per_row else 'per tensor'})"
+                         f", got {s_w.numel()}")
+    return N
+
+
+def _check_out(y: torch.Tensor, M: int, N: int, name: str = "y"):
+    if tuple(y.shape) != (M, N):
+        raise ValueError(f"{name} must be ({M}, {N}), got {tuple(y.shape)}")
+    if y.dtype not in (torch.bfloat16, torch.float32):
+        raise ValueError(f"{name} must be bfloat16 or float32, got {y.dtype}")
+
+
 def workspace_size(M: int, K: int) -> int:
     return int(lib.bitnet_linear_workspace_size(M, K))
 
@@ -188,11 +209,10 @@ def bitnet_linear(x: torch.Tensor, packed: torch.Tensor, s_w: torch.Tensor, per_
                   out_dtype: torch.dtype = torch.bfloat16, y: Optional[torch.Tensor] = None,
                   workspace: Optional[torch.Tensor] = None, path: int = PATH_AUTO, stream=None):
     M, K = x.shape
-    N = packed.shape[0]
-    if packed.shape[1] * 4 != K:
-        raise ValueError("packed must be (N, K/4)")
+    N = _check_proj(packed, s_w, per_row, K)
     if y is None:
         y = torch.empty((M, N), dtype=out_dtype, device=x.device)
+    _check_out(y, M, N)
     od = OUT_BF16 if y.dtype == torch.bfloat16 else OUT_F32
     wp, wb, _keep = _ws_args(workspace, M, K, path, x.device)
     _check(lib.bitnet_linear_ex(_x_ptr(x), M, K, _dev(packed, torch.uint8, "packed"),
@@ -211,8 +231,15 @@ def bitnet_linear_batch(x: torch.Tensor, projs: Sequence, out_dtype: torch.dtype
     n = len(projs)
     if not 1 <= n <= MAX_PROJ:
         raise ValueError(f"1..{MAX_PROJ} projections")
+    Ns = [_check_proj(p[0], p[1], p[2], K) for p in projs]
     if ys is None:
-        ys = [torch.empty((M, p[0].shape[0]), dtype=out_dtype, device=x.device) for p in projs]
+        ys = [torch.empty((M, N), dtype=out_dtype, device=x.device) for N in Ns]
+    if len(ys) != n:
+        raise ValueError(f"{n} projections need {n} outputs, got {len(ys)}")
+    for yi, N in zip(ys, Ns):
+        _check_out(yi, M, N)
+    if any(yi.dtype != ys[0].dtype for yi in ys):
+        raise ValueError("all outputs of a batch must have one dtype")
     od = OUT_BF16 if ys[0].dtype == torch.bfloat16 else OUT_F32
     arr = (bitnet_proj * n)()
     for i, (packed, s_w, per_row) in enumerate(projs):
@@ -238,8 +265,15 @@ def bitnet_linear_batch_act(x: torch.Tensor, projs: Sequence, act: int,
     n = len(projs)
     if not 1 <= n <= MAX_PROJ:
         raise ValueError(f"1..{MAX_PROJ} projections")
+    Ns = [_check_proj(p[0], p[1], p[2], K) for p in projs]
     if ys is None:
-        ys = [torch.empty((M, p[0].shape[0]), dtype=out_dtype, device=x.device) for p in projs]
+        ys = [torch.empty((M, N), dtype=out_dtype, device=x.device) for N in Ns]
+    if len(ys) != n:
+        raise ValueError(f"{n} projections need {n} outputs, got {len(ys)}")
+    for yi, N in zip(ys, Ns):
+        _check_out(yi, M, N)
+    if any(yi.dtype != ys[0].dtype for yi in ys):
+        raise ValueError("all outputs of a batch must have one dtype")
     od = OUT_BF16 if ys[0].dtype == torch.bfloat16 else OUT_F32
     arr = (bitnet_proj * n)()
     for i, (packed, s_w, per_row) in enumerate(projs):
@@ -258,6 +292,8 @@ def bitnet_linear_batch_act(x: torch.Tensor, projs: Sequence, act: int,
 def bitnet_linear_i32(q: torch.Tensor, packed: torch.Tensor, path: int = PATH_AUTO,
                       workspace: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
     M, K = q.shape
+    if packed.dim() != 2 or packed.shape[1] * 4 != K:
+        raise ValueError(f"packed must be (N, K/4) = (N, {K // 4}), got {tuple(packed.shape)}")
     N = packed.shape[0]
     acc = torch.empty((M, N), dtype=torch.int32, device=q.device)
     wp, wb, _keep = _ws_args(workspace, M, K, path, q.device)
@@ -294,11 +330,17 @@ def bitnet_linear_swiglu(x: torch.Tensor, packed_gu: torch.Tensor, s_w_gu: torch
                          stream=None) -> torch.Tensor:
     """h = bf16(bf16(silu(gate(x))) * up(x)), (M, I), from the interleaved gate/up matrix."""
     M, K = x.shape
+    if packed_gu.dim() != 2 or packed_gu.shape[1] * 4 != K or packed_gu.shape[0] % 2:
+        raise ValueError(f"packed_gu must be (2I, K/4) = (2I, {K // 4}), got "
+                         f"{tuple(packed_gu.shape)}")
     I = packed_gu.shape[0] // 2
-    if packed_gu.shape[1] * 4 != K:
-        raise ValueError("packed_gu must be (2I, K/4)")
+    want = 2 * I if per_row else 2
+    if s_w_gu.numel() != want:
+        raise ValueError(f"s_w_gu must have {want} elements, got {s_w_gu.numel()}")
     if h is None:
         h = torch.empty((M, I), dtype=torch.bfloat16, device=x.device)
+    if tuple(h.shape) != (M, I):
+        raise ValueError(f"h must be ({M}, {I}), got {tuple(h.shape)}")
     wp, wb, _keep = _ws_args(workspace, M, K, path, x.device)
     _check(lib.bitnet_linear_swiglu(_x_ptr(x), M, K, _dev(packed_gu, torch.uint8, "packed_gu"),
                                     _dev(s_w_gu, torch.float32, "s_w_gu"), int(bool(per_row)), I,
@@ -313,13 +355,17 @@ NOALLOC_SCRATCH_BYTES = 16 * 1024 * 1024
 def bitnet_linear_noalloc(x: torch.Tensor, packed: torch.Tensor, s_w: torch.Tensor,
                           per_row: bool, out_dtype: torch.dtype = torch.bfloat16,
                           y: Optional[torch.Tensor] = None, stream=None):
-    """bitnet_linear without a workspace: for callers that cannot allocate device memory
-    during execution. Uses the library's fixed 16 MiB device scratch array; calls that can
-    overlap on the GPU race on it. Sizes beyond the array raise BitnetError (workspace)."""
+    """bitnet_linear without a workspace, for callers that cannot allocate device memory
+    while they run (a serving loop where cudaMalloc could synchronise the device, a plug-in
+    whose host runtime owns all device memory). The tensor-core path uses the library's
+    fixed 16 MiB device scratch array; calls that can overlap on the GPU race on it. Sizes
+    whose workspace exceeds the array raise BitnetError (ERR_WORKSPACE). Pass y to make the
+    call itself allocate nothing (with y=None this wrapper allocates the output)."""
     M, K = x.shape
-    N = packed.shape[0]
+    N = _check_proj(packed, s_w, per_row, K)
     if y is None:
         y = torch.empty((M, N), dtype=out_dtype, device=x.device)
+    _check_out(y, M, N)
     od = OUT_BF16 if y.dtype == torch.bfloat16 else OUT_F32
     _check(lib.bitnet_linear_noalloc(_x_ptr(x), M, K, _dev(packed, torch.uint8, "packed"),
                                      _dev(s_w, torch.float32, "s_w"), int(bool(per_row)), N,

@@ -74,6 +74,8 @@ bitnet_status check_workspace(void* ws, size_t bytes, int64_t M, int64_t K) {
     return BITNET_OK;
 }
 
+}  // namespace
+
 // Five to eight tokens take the tensor-core path when the caller's workspace holds it: the
 // GEMV's per-CTA quantisation and dp4a work grow with the token count, and on B200 the
 // tensor-core path with 16-token tiles is as fast or faster there (2B-4T shapes, 8 tokens:
@@ -85,6 +87,8 @@ bool use_gemv(int64_t M, int64_t K, bitnet_path path, const void* ws, size_t ws_
     if (M <= BITNET_GEMV_AUTO_M) return true;
     return !(ws && ws_bytes >= ws_total_bytes(M, K) && aligned(ws, 256));
 }
+
+namespace {
 
 // Runs a validated batch. x_bf16 or q_in (int8, contraction-only) is the input. swiglu: the
 // batch is one interleaved gate/up matrix of N = 2I rows whose output is h (M, I) bf16.

@@ -71,6 +71,9 @@ struct GemvParams {
 
 cudaError_t launch_gemv(const GemvParams& p, cudaStream_t stream, bool pdl);
 bool gemv_supported(int64_t M, int64_t K);
+// The kernel-path choice of bitnet_linear / bitnet_linear_batch: true when a call with this
+// token count, width, path and workspace runs the GEMV (which uses no workspace).
+bool use_gemv(int64_t M, int64_t K, bitnet_path path, const void* ws, size_t ws_bytes);
 
 // Streaming GEMV for one token and large matrices (a producer warp fills a shared-memory
 // ring of 16-row weight stages with bulk copies; one CTA per SM). gemv_stream_plan returns

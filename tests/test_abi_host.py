@@ -7,6 +7,7 @@ import os
 import re
 
 import pytest
+import torch
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 HEADER = os.path.join(ROOT, "include", "bitnet.h")
@@ -175,3 +176,31 @@ def test_act_mode_calls_argument_errors(bn):
     assert L.bitnet_linear_batch_act(FAKE, 4, 512, pr, 1, 3, 1, None, 0, 0, None) == bn.ERR_UNSUPPORTED
     assert L.bitnet_linear_batch_act(FAKE, 300, 512, pr, 1, 0, 1, None, 0, 0, None) == bn.ERR_WORKSPACE
     assert L.bitnet_linear_batch_act(None, 4, 512, pr, 1, 0, 1, None, 0, 0, None) == bn.ERR_NULL
+
+
+def test_binding_rejects_wrong_shapes_before_the_call(bn):
+    """The C side sees only pointers, so the binding checks every shape it can: packed
+    (N, K/4), s_w of N (per row) or 1 (per tensor) elements, and outputs (M, N). These raise
+    ValueError on CPU tensors, before any pointer is taken."""
+    x = torch.zeros((3, 64), dtype=torch.bfloat16)
+    good_p = torch.zeros((8, 16), dtype=torch.uint8)
+    one = torch.ones(1, dtype=torch.float32)
+    cases = [
+        lambda: bn.bitnet_linear(x, torch.zeros((8, 15), dtype=torch.uint8), one, False),
+        lambda: bn.bitnet_linear(x, good_p, one, True),  # per row needs 8 scales
+        lambda: bn.bitnet_linear(x, good_p, torch.ones(8), False),  # per tensor needs 1
+        lambda: bn.bitnet_linear(x, good_p, one, False, y=torch.zeros((3, 7), dtype=torch.bfloat16)),
+        lambda: bn.bitnet_linear_noalloc(x, torch.zeros((8, 32), dtype=torch.uint8), one, False),
+        lambda: bn.bitnet_linear_noalloc(x, good_p, torch.ones(7), True),
+        lambda: bn.bitnet_linear_noalloc(x, good_p, one, False,
+                                         y=torch.zeros((2, 8), dtype=torch.bfloat16)),
+        lambda: bn.bitnet_linear_batch(x, [(good_p, one, False), (good_p, torch.ones(3), True)]),
+        lambda: bn.bitnet_linear_batch(x, [(good_p, one, False)],
+                                       ys=[torch.zeros((3, 9), dtype=torch.bfloat16)]),
+        lambda: bn.bitnet_linear_swiglu(x, torch.zeros((32, 16), dtype=torch.uint8), one, False),
+        lambda: bn.bitnet_linear_i32(torch.zeros((3, 64), dtype=torch.int8),
+                                     torch.zeros((8, 17), dtype=torch.uint8)),
+    ]
+    for i, call in enumerate(cases):
+        with pytest.raises(ValueError):
+            call()
