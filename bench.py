@@ -232,7 +232,7 @@ def run_stack(bn, torch, dev, name, stack, M, steps, warmup, flush, world, peaks
                            for p, (N, K) in zip(L0, shapes))
     act_bytes = layers * sum(2 * M * K + 2 * M * N for N, K in shapes)
     ops = layers * sum(2.0 * M * N * K for N, K in shapes)
-    int8_peak = peaks["bf16_tflops"] * INT8_PER_BF16
+    int8_peak = peaks["int8_tops"]
     roof = max((w_bytes + act_bytes) / (peaks["hbm_gbs"] * 1e9), ops / (int8_peak * 1e12))
     launches = layers * 3 * (2 if tc else 1)
     del g
@@ -307,7 +307,7 @@ def run_mlp(bn, torch, dev, name, layers_w, M, steps, warmup, flush, world, peak
     w_bytes = layers * (2 * ffn * hidden // 4 + 4 * (2 * ffn if per_row else 2))
     act_bytes = layers * (2 * M * hidden + 2 * M * ffn)
     ops = layers * 2.0 * M * (2 * ffn) * hidden
-    int8_peak = peaks["bf16_tflops"] * INT8_PER_BF16
+    int8_peak = peaks["int8_tops"]
     roof = max((w_bytes + act_bytes) / (peaks["hbm_gbs"] * 1e9), ops / (int8_peak * 1e12))
     t = res["fused"]
     launches = layers * (2 if tc else 1)
@@ -369,8 +369,18 @@ def timed_steps(torch, step_fn, steps, warmup, flush_buf, world):
 
 
 # ---------------------------------------------------------------------------- CPU oracle
-def oracle_sample(seconds_min: float):
-    """Times the oracle (as it stands, one thread) on whole decode sweeps at M = 1."""
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+def _oracle_sweep_cases():
     import oracle
     oracle.build()
     cases = []
@@ -378,41 +388,59 @@ def oracle_sample(seconds_min: float):
         c = synth.decode_case(si, replica=0, M=DECODE_M)
         cases.append((c, oracle.pack(c["t"])))
     sweep_bytes = sum(decode_bytes(DECODE_M, c["N"], c["K"]) for c, _ in cases)
-    done, t0 = 0, time.perf_counter()
-    while True:
+
+    def sweep():
         for c, packed in cases:
             oracle.bitlinear(c["x"], packed, c["s_w"], False, c["K"])
+
+    return sweep, sweep_bytes
+
+
+def _threaded_sweeps(sweep, threads: int, rounds: int):
+    """`rounds` rounds of `threads` concurrent whole sweeps (the oracle's C calls release
+    the GIL, so the threads run on separate cores); returns the elapsed seconds."""
+    from concurrent.futures import ThreadPoolExecutor
+    t0 = time.perf_counter()
+    with ThreadPoolExecutor(threads) as ex:
+        for _ in range(rounds):
+            list(ex.map(lambda _: sweep(), range(threads)))
+    return time.perf_counter() - t0
+
+
+def oracle_sample(seconds: float):
+    """Times the oracle (as it stands) on whole decode sweeps at M = 1: one thread for about
+    half of `seconds`, then every host core running independent sweeps for the other half."""
+    sweep, sweep_bytes = _oracle_sweep_cases()
+    done, t0 = 0, time.perf_counter()
+    while True:
+        sweep()
         done += 1
-        el = time.perf_counter() - t0
-        if el >= seconds_min:
+        el1 = time.perf_counter() - t0
+        if el1 >= seconds / 2:
             break
-    return {"value": done * sweep_bytes / el / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
-            "sample": f"{done} full decode sweeps (4 shapes, M=1), {el:.1f} s"}
+    one = done * sweep_bytes / el1 / 1e9
+    n = os.cpu_count() or 1
+    per_round = el1 / done  # one sweep per thread per round, if the cores scale
+    rounds = max(1, int(seconds / 2 / per_round))
+    el = _threaded_sweeps(sweep, n, rounds)
+    return {"value": n * rounds * sweep_bytes / el / 1e9, "unit": "GB/s", "cores": n,
+            "kind": "oracle",
+            "sample": f"{n * rounds} full decode sweeps (4 shapes, M=1) on {n} threads, {el:.1f} s",
+            "one_thread": {"value": one, "unit": "GB/s", "cores": 1,
+                           "sample": f"{done} sweeps, {el1:.1f} s"},
+            "cpu_model": cpu_model(), "nproc": n}
 
 
 def run_reference(args):
     rank, world, _ = dist_env()
     if rank != 0:
         return 0
-    import oracle
-    oracle.build()
-    cases = []
-    for si in range(len(synth.SWEEP_SHAPES)):
-        c = synth.decode_case(si, replica=0, M=DECODE_M)
-        cases.append((c, oracle.pack(c["t"])))
-    sweep_bytes = sum(decode_bytes(DECODE_M, c["N"], c["K"]) for c, _ in cases)
-
-    def step():
-        for c, packed in cases:
-            oracle.bitlinear(c["x"], packed, c["s_w"], False, c["K"])
-
+    sweep, sweep_bytes = _oracle_sweep_cases()
+    n = os.cpu_count() or 1
     for _ in range(args.warmup):
-        step()
-    t0 = time.perf_counter()
-    for _ in range(args.steps):
-        step()
-    el = time.perf_counter() - t0
-    value = args.steps * sweep_bytes / el / 1e9
+        sweep()
+    el = _threaded_sweeps(sweep, n, args.steps)  # one step = one sweep on every core
+    value = args.steps * n * sweep_bytes / el / 1e9
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s",
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
@@ -420,13 +448,48 @@ def run_reference(args):
         "vs_baseline": None, "dtype": "s8xternary->s32", "data": "synthetic",
         "config": {"workload": "decode GEMV sweep M=1, 2B-4T shapes (N,K) in "
                                "{(2560,2560),(640,2560),(6912,2560),(2560,6912)}; one sweep "
-                               "(one weight replica) per step"},
-        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": 1, "kind": "oracle",
-                         "sample": f"{args.steps} sweeps of the 4 shapes at M=1"},
+                               "(one weight replica) per host thread per step"},
+        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": n, "kind": "oracle",
+                         "sample": f"{args.steps} steps of {n} concurrent sweeps of the 4 "
+                                   "shapes at M=1", "cpu_model": cpu_model()},
         "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
     return 0
+
+
+def measure_int8_peak(torch, dev, seconds: float = 1.5):
+    """Dense int8 tensor-core rate of this GPU through torch._int_mm (cuBLASLt) on 8192^3:
+    best of 10 single calls, and the rate of back-to-back calls for `seconds`."""
+    n = 8192
+    a = torch.randint(-128, 127, (n, n), dtype=torch.int8, device=dev)
+    b = torch.randint(-128, 127, (n, n), dtype=torch.int8, device=dev).t()
+    try:
+        for _ in range(3):
+            torch._int_mm(a, b)
+    except RuntimeError as e:  # no int8 GEMM in this build
+        return {"error": repr(e)[:200]}
+    torch.cuda.synchronize()
+    best = float("inf")
+    for _ in range(10):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        torch._int_mm(a, b)
+        e1.record()
+        torch.cuda.synchronize()
+        best = min(best, e0.elapsed_time(e1))
+    calls = max(1, int(seconds / (best * 1e-3)))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(calls):
+        torch._int_mm(a, b)
+    e1.record()
+    torch.cuda.synchronize()
+    ops = 2.0 * n ** 3
+    return {"burst_tops": ops / (best * 1e-3) / 1e12,
+            "sustained_tops": ops * calls / (e0.elapsed_time(e1) * 1e-3) / 1e12,
+            "how": "torch._int_mm int8 8192^3 -> int32: best of 10, and back to back "
+                   f"for {seconds} s"}
 
 
 # ---------------------------------------------------------------------------- main arm
@@ -444,6 +507,15 @@ def run_ours(args):
 
     peaks = load_peaks()
     flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+    # The GEMM's denominator: the larger of the measured int8 rate (cuBLASLt through
+    # torch._int_mm) and the nominal int8 : bf16 ratio times the measured bf16 peak.
+    int8_probe = measure_int8_peak(torch, dev) if args.only == "all" else {}
+    nominal = peaks["bf16_tflops"] * INT8_PER_BF16
+    measured = int8_probe.get("burst_tops", 0.0)
+    peaks["int8_tops"] = max(measured, nominal)
+    peaks["int8_src"] = ("measured torch._int_mm burst" if measured >= nominal else
+                         f"{peaks['src']} bf16 burst x {INT8_PER_BF16} (nominal int8:bf16), above "
+                         "the measured int8 rate")
 
     # ---------------- decode GEMV sweep
     per_replica = sum(N * K // 4 for N, K in synth.SWEEP_SHAPES)
@@ -507,15 +579,17 @@ def run_ours(args):
         ops_step = sum(2.0 * args.prefill_m * c["N"] * c["K"] for c in pcalls)
         pre_ms_max, pre_ops = reduce_over_ranks(pre_ms, ops_step * args.steps, world)
         tops = pre_ops / (pre_ms_max * 1e-3) / 1e12
-        int8_peak = peaks["bf16_tflops"] * INT8_PER_BF16
+        int8_peak = peaks["int8_tops"]
         local_tops = ops_step * args.steps / (pre_ms * 1e-3) / 1e12
         gemm = {"value": tops, "unit": "TOPS", "ms_per_step": pre_ms_max / args.steps,
                 "workload": f"prefill GEMM M={args.prefill_m} on the same 4 shapes, x = 0.5 t_4 "
                             "with 1% x20 outlier channels, ternary P(0)=0.5",
                 "roofline": {"bound": "tensor", "achieved": local_tops, "peak": int8_peak,
-                             "unit": "TOPS", "frac": local_tops / int8_peak, "traffic": None,
-                             "peak_src": f"{peaks['src']} bf16 x {INT8_PER_BF16} "
-                                         "(nominal int8:bf16)",
+                             "unit": "TOPS", "frac": local_tops / int8_peak,
+                             "traffic": None,
+                             "peak_src": peaks["int8_src"],
+                             "frac_vs_measured_int8": (local_tops / int8_probe["burst_tops"]
+                                                       if int8_probe.get("burst_tops") else None),
                              "note": "per-call time includes the quantiser launch"}}
         # the same calls with one activation scale per tensor (partial maxima kernel added)
         def run_pt():
@@ -611,6 +685,12 @@ def run_ours(args):
             "gpu_launches": args.steps * launches_per_step * 2 + args.steps * 7 * len(pcalls)
                             + stack_launches,
             "clocks": clk.summary(),
+            "gemm_tops": gemm["value"] if gemm else None,
+            "gemm_frac": gemm["roofline"]["frac"] if gemm else None,
+            "gemm_m512_tops": gemm[f"m{PREFILL_M_SMALL}"]["value"]
+            if gemm and f"m{PREFILL_M_SMALL}" in gemm else None,
+            "int8_peak": dict(int8_probe, used_tops=peaks["int8_tops"], used_src=peaks["int8_src"])
+            if int8_probe else None,
             "gemm": gemm,
             "stacks": stacks,
             "mlp": mlp,

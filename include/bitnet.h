@@ -80,9 +80,12 @@ typedef enum {
 typedef enum {
     BITNET_PATH_AUTO = 0, /* GEMV for M <= BITNET_GEMV_AUTO_M; for M up to                */
                           /* BITNET_GEMV_MAX_M the tensor-core GEMM when the workspace    */
-                          /* holds it, else the GEMV; tensor-core GEMM above              */
-    BITNET_PATH_GEMV = 1, /* force the dp4a GEMV with fused activation quantisation      */
-    BITNET_PATH_TC = 2    /* force the tcgen05 GEMM (needs the workspace)                 */
+                          /* holds it, else the GEMV; tensor-core GEMM above. Among the   */
+                          /* GEMVs, the kernel measured fastest for the size.             */
+    BITNET_PATH_GEMV = 1, /* force the dp4a GEMV with fused activation quantisation (the  */
+                          /* streaming variant at one token from 12 MiB of weights)       */
+    BITNET_PATH_TC = 2,   /* force the tcgen05 GEMM (needs the workspace)                 */
+    BITNET_PATH_MMA = 3   /* force the warp-level tensor-core GEMV (mma.sync), M <= 8     */
 } bitnet_path;
 
 #define BITNET_GEMV_MAX_M 8
@@ -290,6 +293,61 @@ bitnet_status bitnet_linear_noalloc(const uint16_t* x, int64_t M, int64_t K,
                                     const uint8_t* packed, const float* s_w,
                                     bitnet_scale_mode mode, int64_t N, void* y,
                                     bitnet_out_dtype out_dtype, void* stream);
+
+/*
+ * Tensor-parallel steps ("BitNet：1-bit LLM推理框架技术实战指南", section on the distributed
+ * engine: a model split by layer or by tensor across devices). When a projection's K range is
+ * split over ranks (rank r holds x[:, k0:k1] and packed[:, k0/4 : k1/4], k0 and k1 multiples
+ * of 64), the per-token scale needs the amax of the whole row and the int32 accumulator the
+ * sum over all slices. A rank runs: bitnet_act_amax on its slice; an all-reduce (max) of amax
+ * over the ranks; bitnet_quant_act_amax with that amax; bitnet_linear_i32 on its slices; an
+ * all-reduce (sum) of the int32 accumulators (exact in any order); bitnet_dequant. The result
+ * equals bitnet_linear on the whole row bit for bit. A split over N needs none of these: each
+ * rank runs bitnet_linear on its rows and the outputs are gathered.
+ *
+ * bitnet_act_amax — amax[m] = max_k |x[m, k]| (exact; the value a bf16 element has).
+ *   x [in] (M, K) bf16 bits, 16-byte aligned.  amax [out] (M) fp32.
+ * bitnet_quant_act_amax — bitnet_quant_act with the amax supplied: s_x[m] = 127 /
+ *   max(amax[m], 1e-5) (binary32 divide), q = clamp(rint(x * s_x), -128, 127), natural order.
+ *   amax must be at least max_k |x[m, k]| of this x (as the all-reduced maximum is), so the
+ *   clamp never acts. x, q 16-byte aligned; amax, s_x (M) fp32.
+ * bitnet_dequant — the epilogue alone: y[m, n] = RN(RN(acc[m, n]) * RN(s_w[n or 0] *
+ *   RN(1 / s_x[m]))) in binary32, bf16 by RNE: the rounding steps of bitnet_linear.
+ *   acc (M, N) int32, s_x (M), s_w (1 or N by mode), y (M, N) bf16 or fp32.
+ * All asynchronous on `stream`; argument errors as for the other calls (M * K / 8 and M * N
+ * below 2^39).
+ */
+bitnet_status bitnet_act_amax(const uint16_t* x, int64_t M, int64_t K, float* amax, void* stream);
+bitnet_status bitnet_quant_act_amax(const uint16_t* x, int64_t M, int64_t K, const float* amax,
+                                    int8_t* q, float* s_x, void* stream);
+bitnet_status bitnet_dequant(const int32_t* acc, int64_t M, int64_t N, const float* s_x,
+                             const float* s_w, bitnet_scale_mode mode, void* y,
+                             bitnet_out_dtype out_dtype, void* stream);
+
+/*
+ * bitnet_linear_plan — which kernels a call would run, without running anything (a host-only
+ * query for tests and tuning; the pages have no counterpart). It reports the choices
+ * bitnet_linear_batch_ex makes for nproj projections of widths Ns[0 .. nproj) at M tokens of
+ * width K with a 256-byte aligned workspace of workspace_bytes (0 = no workspace) on path
+ * `path`, or, with swiglu = 1 (nproj = 1, Ns[0] = 2I), those of bitnet_linear_swiglu. It
+ * reads the current device's SM count (148 when no device can be queried). Argument errors
+ * are those of the call it describes.
+ */
+#define BITNET_KERNEL_GEMV 1   /* dp4a GEMV with the quantiser fused, up to 8 tokens          */
+#define BITNET_KERNEL_MMA_GEMV 2 /* warp-level tensor-core GEMV (mma.sync), up to 8 tokens  */
+#define BITNET_KERNEL_STREAM 3 /* one-token streaming GEMV through a shared-memory ring      */
+#define BITNET_KERNEL_TC 4     /* quantiser kernel, then the tcgen05 tensor-core GEMM         */
+typedef struct {
+    int32_t kernel;        /* BITNET_KERNEL_*                                               */
+    int32_t grid;          /* CTAs of the main kernel (0 for BITNET_KERNEL_GEMV)            */
+    int32_t tile_tokens;   /* tensor-core path: tokens per tile (16 .. 192), else 0         */
+    int32_t splits;        /* tensor-core path: K splits per tile (1 = none), else 0        */
+    int32_t tile_rows;     /* warp-MMA GEMV: weight rows per CTA, else 0                     */
+    int32_t reserved[3];
+} bitnet_plan;
+bitnet_status bitnet_linear_plan(int64_t M, int64_t K, const int64_t* Ns, int32_t nproj,
+                                 int32_t swiglu, size_t workspace_bytes, bitnet_path path,
+                                 bitnet_plan* plan);
 
 /*
  * bitnet_check_device_errors — synchronises the current device, returns the library's

@@ -40,7 +40,7 @@ lib = ctypes.CDLL(LIB_PATH)
 OK, ERR_NULL, ERR_SHAPE, ERR_ALIGN, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT, ERR_WORKSPACE = range(8)
 SCALE_PER_TENSOR, SCALE_PER_ROW = 0, 1
 OUT_BF16, OUT_F32 = 0, 1
-PATH_AUTO, PATH_GEMV, PATH_TC = 0, 1, 2
+PATH_AUTO, PATH_GEMV, PATH_TC, PATH_MMA = 0, 1, 2, 3
 ACT_PER_TOKEN, ACT_PER_TENSOR = 0, 1
 QUANT_WORKSPACE_BYTES = 4096
 GEMV_MAX_M = 8
@@ -58,6 +58,13 @@ class bitnet_proj(ctypes.Structure):
     _fields_ = [("packed", _P), ("s_w", _P), ("mode", _I32), ("reserved", _I32), ("N", _I64),
                 ("y", _P)]
 
+
+class bitnet_plan(ctypes.Structure):
+    _fields_ = [("kernel", _I32), ("grid", _I32), ("tile_tokens", _I32), ("splits", _I32),
+                ("tile_rows", _I32), ("reserved", _I32 * 3)]
+
+
+KERNEL_GEMV, KERNEL_MMA_GEMV, KERNEL_STREAM, KERNEL_TC = 1, 2, 3, 4
 
 _SIGS = {
     "bitnet_pack_weights": ([_P, _I64, _I64, ctypes.c_int, _P, _P, _P], ctypes.c_int),
@@ -82,6 +89,11 @@ _SIGS = {
                                   ctypes.c_int),
     "bitnet_linear_swiglu": ([_P, _I64, _I64, _P, _P, ctypes.c_int, _I64, _P, _P, _SZ,
                              ctypes.c_int, _P], ctypes.c_int),
+    "bitnet_act_amax": ([_P, _I64, _I64, _P, _P], ctypes.c_int),
+    "bitnet_quant_act_amax": ([_P, _I64, _I64, _P, _P, _P, _P], ctypes.c_int),
+    "bitnet_dequant": ([_P, _I64, _I64, _P, _P, ctypes.c_int, _P, ctypes.c_int, _P], ctypes.c_int),
+    "bitnet_linear_plan": ([_I64, _I64, ctypes.POINTER(_I64), _I32, _I32, _SZ, ctypes.c_int,
+                            ctypes.POINTER(bitnet_plan)], ctypes.c_int),
     "bitnet_check_device_errors": ([ctypes.POINTER(_I32)], ctypes.c_int),
     "bitnet_selftest_wait_timeout": ([_I64, _P], ctypes.c_int),
     "bitnet_status_string": ([ctypes.c_int], ctypes.c_char_p),
@@ -372,6 +384,60 @@ def bitnet_linear_noalloc(x: torch.Tensor, packed: torch.Tensor, s_w: torch.Tens
                                      _dev(y, y.dtype, "y"), od, _stream(stream)),
            "bitnet_linear_noalloc")
     return y
+
+
+def bitnet_act_amax(x: torch.Tensor, stream=None) -> torch.Tensor:
+    """Per-token max |x| (fp32, exact), the first tensor-parallel step of a K-split projection."""
+    M, K = x.shape
+    amax = torch.empty(M, dtype=torch.float32, device=x.device)
+    _check(lib.bitnet_act_amax(_x_ptr(x), M, K, amax.data_ptr(), _stream(stream)),
+           "bitnet_act_amax")
+    return amax
+
+
+def bitnet_quant_act_amax(x: torch.Tensor, amax: torch.Tensor, stream=None):
+    """Per-token quantiser with the amax supplied (e.g. all-reduced over a K split): (q, s_x)."""
+    M, K = x.shape
+    if amax.numel() != M:
+        raise ValueError(f"amax must have {M} elements, got {amax.numel()}")
+    q = torch.empty((M, K), dtype=torch.int8, device=x.device)
+    s_x = torch.empty(M, dtype=torch.float32, device=x.device)
+    _check(lib.bitnet_quant_act_amax(_x_ptr(x), M, K, _dev(amax, torch.float32, "amax"),
+                                     q.data_ptr(), s_x.data_ptr(), _stream(stream)),
+           "bitnet_quant_act_amax")
+    return q, s_x
+
+
+def bitnet_dequant(acc: torch.Tensor, s_x: torch.Tensor, s_w: torch.Tensor, per_row: bool,
+                   out_dtype: torch.dtype = torch.bfloat16, y: Optional[torch.Tensor] = None,
+                   stream=None) -> torch.Tensor:
+    """The epilogue alone on an int32 accumulator (M, N): y = acc * (s_w * (1 / s_x))."""
+    M, N = acc.shape
+    if s_x.numel() != M or s_w.numel() != (N if per_row else 1):
+        raise ValueError("s_x must have M elements and s_w N (per row) or 1")
+    if y is None:
+        y = torch.empty((M, N), dtype=out_dtype, device=acc.device)
+    _check_out(y, M, N)
+    od = OUT_BF16 if y.dtype == torch.bfloat16 else OUT_F32
+    _check(lib.bitnet_dequant(_dev(acc, torch.int32, "acc"), M, N, _dev(s_x, torch.float32, "s_x"),
+                              _dev(s_w, torch.float32, "s_w"), int(bool(per_row)),
+                              _dev(y, y.dtype, "y"), od, _stream(stream)), "bitnet_dequant")
+    return y
+
+
+def bitnet_linear_plan(M: int, K: int, Ns: Sequence[int], swiglu: bool = False,
+                       workspace_bytes: Optional[int] = None, path: int = PATH_AUTO) -> dict:
+    """The kernels a bitnet_linear_batch (or, with swiglu, bitnet_linear_swiglu with
+    Ns = [2I]) call would run: host-only, nothing is launched. workspace_bytes defaults to
+    workspace_size(M, K), what make_workspace provides."""
+    n = len(Ns)
+    arr = (_I64 * max(n, 1))(*Ns)
+    wb = workspace_size(M, K) if workspace_bytes is None else int(workspace_bytes)
+    pl = bitnet_plan()
+    _check(lib.bitnet_linear_plan(M, K, arr, n, int(bool(swiglu)), wb, path, ctypes.byref(pl)),
+           "bitnet_linear_plan")
+    return {"kernel": pl.kernel, "grid": pl.grid, "tile_tokens": pl.tile_tokens,
+            "splits": pl.splits, "tile_rows": pl.tile_rows}
 
 
 def bitnet_check_device_errors() -> int:

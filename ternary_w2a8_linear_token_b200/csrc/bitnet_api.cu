@@ -81,7 +81,7 @@ bitnet_status check_workspace(void* ws, size_t bytes, int64_t M, int64_t K) {
 // tensor-core path with 16-token tiles is as fast or faster there (2B-4T shapes, 8 tokens:
 // 10.7 / 8.7 / 20.9 / 27.2 us per GEMV call against about 10 / 9 / 11 / 15 us).
 bool use_gemv(int64_t M, int64_t K, bitnet_path path, const void* ws, size_t ws_bytes) {
-    if (path == BITNET_PATH_GEMV) return true;
+    if (path == BITNET_PATH_GEMV || path == BITNET_PATH_MMA) return true;
     if (path == BITNET_PATH_TC) return false;
     if (M > BITNET_GEMV_MAX_M || !gemv_supported(M, K)) return false;
     if (M <= BITNET_GEMV_AUTO_M) return true;
@@ -90,15 +90,25 @@ bool use_gemv(int64_t M, int64_t K, bitnet_path path, const void* ws, size_t ws_
 
 namespace {
 
-// Runs a validated batch. x_bf16 or q_in (int8, contraction-only) is the input. swiglu: the
-// batch is one interleaved gate/up matrix of N = 2I rows whose output is h (M, I) bf16.
-bitnet_status run_batch(const uint16_t* x_bf16, const int8_t* q_in, int64_t M, int64_t K,
-                        const Batch& b, int out_kind, void* workspace, size_t workspace_bytes,
-                        bitnet_path path, cudaStream_t stream, bool swiglu = false,
-                        bool act_per_tensor = false) {
+// The launch decisions of one call, shared by run_batch and bitnet_linear_plan.
+struct Plan {
+    int kernel = 0;  // BITNET_KERNEL_*
+    GemvParams gp;   // GEMV family: the kernel's parameters
+    int rt = 0, grid = 0, cpt = 0;                       // warp-MMA decode GEMV
+    int64_t n_stages = 0;                                // streaming GEMV
+    int depth = 0;
+    uint32_t stage_bytes = 0;
+    int bn = 0, splits = 1, tiles = 0;                   // tensor-core GEMM
+};
+
+// Chooses the kernels of a validated batch (pointers are copied, never dereferenced).
+bitnet_status plan_batch(const uint16_t* x_bf16, const int8_t* q_in, int64_t M, int64_t K,
+                         const Batch& b, int out_kind, const void* workspace,
+                         size_t workspace_bytes, bitnet_path path, bool swiglu,
+                         bool act_per_tensor, Plan* pl) {
     if (use_gemv(M, K, path, workspace, workspace_bytes)) {
         if (!gemv_supported(M, K)) return BITNET_ERR_UNSUPPORTED;
-        GemvParams p;
+        GemvParams& p = pl->gp;
         std::memset(&p, 0, sizeof(p));
         p.x = x_bf16;
         p.q_in = q_in;
@@ -118,25 +128,110 @@ bitnet_status run_batch(const uint16_t* x_bf16, const int8_t* q_in, int64_t M, i
             rows += b.proj[i].N;
         }
         p.total_rows = rows;
-        if (swiglu) {  // one warp per output pair: I pairs, output width I
+        if (swiglu) {  // one output per gate/up row pair: I pairs, output width I
             p.swiglu = 1;
             p.total_rows = rows / 2;
             p.proj[0].N = rows / 2;
         }
-        // One token and a matrix too large for one wave of the register-resident kernel:
-        // stream it through a shared-memory ring instead.
-        int64_t n_stages = 0;
-        int depth = 0;
-        uint32_t stage_bytes = 0;
-        if (rows * (K / 4) >= kStreamMinBytes &&
-            gemv_stream_plan(p, &n_stages, &depth, &stage_bytes)) {
-            int32_t* err = device_error_word();
-            if (!err) return BITNET_ERR_CUDA;
-            return from_cuda(launch_gemv_stream(p, n_stages, depth, stage_bytes, tc_num_sms(),
-                                                err, stream, /*pdl=*/true));
+        // One token and a matrix too large for registers: stream it through a shared-memory
+        // ring. The warp-MMA GEMV where it measured faster than the dp4a GEMV in chains of
+        // calls on B200 (one token from kMmaMinBytesOneToken of packed weights, five to eight
+        // tokens above kMmaMinBytesFewTokens); the dp4a GEMV otherwise.
+        const int64_t wbytes = rows * (K / 4);
+        if (path == BITNET_PATH_MMA) {
+            if (!gemv_mma_plan(p, tc_num_sms(), &pl->rt, &pl->grid, &pl->cpt))
+                return BITNET_ERR_UNSUPPORTED;
+            pl->kernel = BITNET_KERNEL_MMA_GEMV;
+            return BITNET_OK;
         }
-        return from_cuda(launch_gemv(p, stream, /*pdl=*/true));
+        const bool mma_pays = path == BITNET_PATH_AUTO &&
+                              (M == 1 ? wbytes >= kMmaMinBytesOneToken
+                                      : M >= 5 && wbytes > kMmaMinBytesFewTokens);
+        if (wbytes >= kStreamMinBytes &&
+            gemv_stream_plan(p, &pl->n_stages, &pl->depth, &pl->stage_bytes)) {
+            pl->kernel = BITNET_KERNEL_STREAM;
+            pl->grid = static_cast<int>(pl->n_stages < tc_num_sms() ? pl->n_stages : tc_num_sms());
+        } else if (mma_pays && gemv_mma_plan(p, tc_num_sms(), &pl->rt, &pl->grid, &pl->cpt)) {
+            pl->kernel = BITNET_KERNEL_MMA_GEMV;
+        } else {
+            pl->kernel = BITNET_KERNEL_GEMV;
+        }
+        return BITNET_OK;
     }
+
+    if (!workspace || workspace_bytes < ws_total_bytes(M, K)) return BITNET_ERR_WORKSPACE;
+    pl->kernel = BITNET_KERNEL_TC;
+    int tiles = 0;
+    for (int i = 0; i < b.nproj; ++i) tiles += static_cast<int>((b.proj[i].N + 127) / 128);
+    pl->tiles = tiles;
+    // Token tile width: the widest that M needs; past 128 tokens, 192, 160 or 128, whichever
+    // gives the shortest run of tile waves, a K stage of a BN-token tile costing about
+    // BN + 264 units (fitted to per-call times measured on B200 at M = 512 ... 4096).
+    const int sms = tc_num_sms();
+    int bn = tc_pick_bn(M);
+    if (bn > 128) {
+        auto waves_cost = [&](int64_t w) {
+            const int64_t t = int64_t(tiles) * ((M + w - 1) / w);
+            return ((t + sms - 1) / sms) * (w + 264);
+        };
+        int64_t best = waves_cost(bn);
+        for (int w : {160, 128}) {
+            const int64_t c = waves_cost(w);
+            if (c <= best) {
+                best = c;
+                bn = w;
+            }
+        }
+    }
+    pl->bn = bn;
+    // Split-K when the tiles leave most SMs idle and the workspace holds the split area:
+    // each tile's K range is cut into `splits` units (at least 512 K bytes each) so that about
+    // one unit runs per SM; units add their int32 partial tiles into a zeroed accumulation tile.
+    pl->splits = 1;
+    // K stages of the kernel: 512 bytes for token tiles of at most 64, else 256 bytes.
+    const int64_t kstage = bn <= 64 ? 512 : 256;
+    const int64_t num_k = (K + kstage - 1) / kstage;
+    const int64_t m_tiles = (M + bn - 1) / bn;
+    const int64_t tiles_all = m_tiles * tiles;
+    // Measured on B200: splitting pays for token tiles of up to 32, and of 64 with long K
+    // loops; for wider tiles the atomic reduction of the partial tiles costs more than the
+    // shorter main loop saves.
+    const bool split_pays = !swiglu && (bn <= 32 || (bn == 64 && K >= 4096));
+    const int64_t unit_stages = 512 / kstage;  // a split unit spans at least 512 K bytes
+    if (split_pays && tiles_all * 4 <= sms && tiles_all <= kMaxSplitTiles &&
+        num_k >= 2 * unit_stages && workspace_bytes >= ws_total_bytes(M, K) + ws_split_bytes(M)) {
+        int64_t sp = sms / tiles_all;
+        if (sp > num_k / unit_stages) sp = num_k / unit_stages;
+        if (sp > 8) sp = 8;
+        if (sp >= 2) pl->splits = static_cast<int>(sp);
+    }
+    const int64_t units = tiles_all * pl->splits;
+    pl->grid = static_cast<int>(units < sms ? units : sms);
+    return BITNET_OK;
+}
+
+// Runs a validated batch. x_bf16 or q_in (int8, contraction-only) is the input. swiglu: the
+// batch is one interleaved gate/up matrix of N = 2I rows whose output is h (M, I) bf16.
+bitnet_status run_batch(const uint16_t* x_bf16, const int8_t* q_in, int64_t M, int64_t K,
+                        const Batch& b, int out_kind, void* workspace, size_t workspace_bytes,
+                        bitnet_path path, cudaStream_t stream, bool swiglu = false,
+                        bool act_per_tensor = false) {
+    Plan pl;
+    bitnet_status pst = plan_batch(x_bf16, q_in, M, K, b, out_kind, workspace, workspace_bytes,
+                                   path, swiglu, act_per_tensor, &pl);
+    if (pst != BITNET_OK) return pst;
+    if (pl.kernel == BITNET_KERNEL_STREAM) {
+        int32_t* err = device_error_word();
+        if (!err) return BITNET_ERR_CUDA;
+        return from_cuda(launch_gemv_stream(pl.gp, pl.n_stages, pl.depth, pl.stage_bytes,
+                                            tc_num_sms(), err, stream, /*pdl=*/true));
+    }
+    if (pl.kernel == BITNET_KERNEL_MMA_GEMV) {
+        int32_t* err = device_error_word();
+        if (!err) return BITNET_ERR_CUDA;
+        return from_cuda(launch_gemv_mma(pl.gp, pl.rt, pl.grid, pl.cpt, err, stream, /*pdl=*/true));
+    }
+    if (pl.kernel == BITNET_KERNEL_GEMV) return from_cuda(launch_gemv(pl.gp, stream, /*pdl=*/true));
 
     bitnet_status st = check_workspace(workspace, workspace_bytes, M, K);
     if (st != BITNET_OK) return st;
@@ -167,25 +262,7 @@ bitnet_status run_batch(const uint16_t* x_bf16, const int8_t* q_in, int64_t M, i
         p.proj[i].tile_begin = tiles;
         tiles += static_cast<int>((N + 127) / 128);
     }
-    // Token tile width: the widest that M needs; past 128 tokens, 192, 160 or 128, whichever
-    // gives the shortest run of tile waves, a K stage of a BN-token tile costing about
-    // BN + 264 units (fitted to per-call times measured on B200 at M = 512 ... 4096).
-    const int sms = tc_num_sms();
-    int bn = tc_pick_bn(M);
-    if (bn > 128) {
-        auto waves_cost = [&](int64_t w) {
-            const int64_t t = int64_t(tiles) * ((M + w - 1) / w);
-            return ((t + sms - 1) / sms) * (w + 264);
-        };
-        int64_t best = waves_cost(bn);
-        for (int w : {160, 128}) {
-            const int64_t c = waves_cost(w);
-            if (c <= best) {
-                best = c;
-                bn = w;
-            }
-        }
-    }
+    const int bn = pl.bn;
     if (!encode_tmap_2d_u8(&p.tmap_q, q_ws, uint64_t(K), uint64_t(M), uint64_t(K), 128,
                            uint32_t(bn), /*swizzle_bytes=*/128))
         return BITNET_ERR_CUDA;
@@ -224,35 +301,16 @@ bitnet_status run_batch(const uint16_t* x_bf16, const int8_t* q_in, int64_t M, i
     p.n_tiles_total = tiles;
     p.out_kind = out_kind;
 
-    // Split-K when the tiles leave most SMs idle and the workspace holds the split area:
-    // each tile's K range is cut into `splits` units (at least 512 K bytes each) so that about
-    // one unit runs per SM; units add their int32 partial tiles into a zeroed accumulation tile.
-    p.splits = 1;
-    // K stages of the kernel: 512 bytes for token tiles of at most 64, else 256 bytes.
-    const int64_t kstage = bn <= 64 ? 512 : 256;
-    const int64_t num_k = (K + kstage - 1) / kstage;
-    const int64_t m_tiles = (M + bn - 1) / bn;
-    const int64_t tiles_all = m_tiles * tiles;
+    p.splits = pl.splits;
     void* zero = nullptr;
     int64_t zero_bytes = 0;
-    // Measured on B200: splitting pays for token tiles of up to 32, and of 64 with long K
-    // loops; for wider tiles the atomic reduction of the partial tiles costs more than the
-    // shorter main loop saves.
-    const bool split_pays = !swiglu && (bn <= 32 || (bn == 64 && K >= 4096));
-    const int64_t unit_stages = 512 / kstage;  // a split unit spans at least 512 K bytes
-    if (split_pays && tiles_all * 4 <= sms && tiles_all <= kMaxSplitTiles &&
-        num_k >= 2 * unit_stages && workspace_bytes >= ws_total_bytes(M, K) + ws_split_bytes(M)) {
-        int64_t sp = sms / tiles_all;
-        if (sp > num_k / unit_stages) sp = num_k / unit_stages;
-        if (sp > 8) sp = 8;
-        if (sp >= 2) {
-            p.splits = static_cast<int32_t>(sp);
-            uint8_t* split = ws + ws_total_bytes(M, K);
-            p.split_cnt = reinterpret_cast<int32_t*>(split);
-            p.split_acc = reinterpret_cast<int32_t*>(split + ws_split_cnt_bytes());
-            zero = split;
-            zero_bytes = int64_t(ws_split_cnt_bytes() + size_t(tiles_all) * size_t(128) * bn * 4);
-        }
+    if (pl.splits > 1) {
+        const int64_t tiles_all = ((M + bn - 1) / bn) * tiles;
+        uint8_t* split = ws + ws_total_bytes(M, K);
+        p.split_cnt = reinterpret_cast<int32_t*>(split);
+        p.split_acc = reinterpret_cast<int32_t*>(split + ws_split_cnt_bytes());
+        zero = split;
+        zero_bytes = int64_t(ws_split_cnt_bytes() + size_t(tiles_all) * size_t(128) * bn * 4);
     }
 
     const bool per_tensor = act_per_tensor && !q_in;
@@ -375,7 +433,8 @@ bitnet_status bitnet_linear_batch_ex(const uint16_t* x, int64_t M, int64_t K,
                                      bitnet_out_dtype out_dtype, void* workspace,
                                      size_t workspace_bytes, bitnet_path path, void* stream) {
     if (out_dtype != BITNET_OUT_BF16 && out_dtype != BITNET_OUT_F32) return BITNET_ERR_UNSUPPORTED;
-    if (path != BITNET_PATH_AUTO && path != BITNET_PATH_GEMV && path != BITNET_PATH_TC)
+    if (path != BITNET_PATH_AUTO && path != BITNET_PATH_GEMV && path != BITNET_PATH_TC &&
+        path != BITNET_PATH_MMA)
         return BITNET_ERR_UNSUPPORTED;
     Batch b;
     bitnet_status st = validate_batch(x, M, K, projs, nproj, int(out_dtype), &b);
@@ -391,7 +450,8 @@ bitnet_status bitnet_linear_batch_act(const uint16_t* x, int64_t M, int64_t K,
                                       void* stream) {
     if (act != BITNET_ACT_PER_TOKEN && act != BITNET_ACT_PER_TENSOR) return BITNET_ERR_UNSUPPORTED;
     if (out_dtype != BITNET_OUT_BF16 && out_dtype != BITNET_OUT_F32) return BITNET_ERR_UNSUPPORTED;
-    if (path != BITNET_PATH_AUTO && path != BITNET_PATH_GEMV && path != BITNET_PATH_TC)
+    if (path != BITNET_PATH_AUTO && path != BITNET_PATH_GEMV && path != BITNET_PATH_TC &&
+        path != BITNET_PATH_MMA)
         return BITNET_ERR_UNSUPPORTED;
     Batch b;
     bitnet_status st = validate_batch(x, M, K, projs, nproj, int(out_dtype), &b);
@@ -435,7 +495,8 @@ bitnet_status bitnet_linear(const uint16_t* x, int64_t M, int64_t K, const uint8
 bitnet_status bitnet_linear_i32(const int8_t* q, int64_t M, int64_t K, const uint8_t* packed,
                                 int64_t N, int32_t* acc, void* workspace, size_t workspace_bytes,
                                 bitnet_path path, void* stream) {
-    if (path != BITNET_PATH_AUTO && path != BITNET_PATH_GEMV && path != BITNET_PATH_TC)
+    if (path != BITNET_PATH_AUTO && path != BITNET_PATH_GEMV && path != BITNET_PATH_TC &&
+        path != BITNET_PATH_MMA)
         return BITNET_ERR_UNSUPPORTED;
     bitnet_proj pr;
     pr.packed = packed;
@@ -498,7 +559,8 @@ bitnet_status bitnet_linear_swiglu(const uint16_t* x, int64_t M, int64_t K,
                                    bitnet_scale_mode mode, int64_t I, uint16_t* h,
                                    void* workspace, size_t workspace_bytes, bitnet_path path,
                                    void* stream) {
-    if (path != BITNET_PATH_AUTO && path != BITNET_PATH_GEMV && path != BITNET_PATH_TC)
+    if (path != BITNET_PATH_AUTO && path != BITNET_PATH_GEMV && path != BITNET_PATH_TC &&
+        path != BITNET_PATH_MMA)
         return BITNET_ERR_UNSUPPORTED;
     if (!h) return BITNET_ERR_NULL;
     bitnet_status st = check_n(I);
@@ -515,6 +577,81 @@ bitnet_status bitnet_linear_swiglu(const uint16_t* x, int64_t M, int64_t K,
     if ((st = validate_batch(x, M, K, &pr, 1, /*out_kind=*/0, &b)) != BITNET_OK) return st;
     return run_batch(x, nullptr, M, K, b, 0, workspace, workspace_bytes, path,
                      static_cast<cudaStream_t>(stream), /*swiglu=*/true);
+}
+
+bitnet_status bitnet_act_amax(const uint16_t* x, int64_t M, int64_t K, float* amax, void* stream) {
+    if (!x || !amax) return BITNET_ERR_NULL;
+    bitnet_status st = check_mk(M, K);
+    if (st != BITNET_OK) return st;
+    if (!aligned(x, 16) || !aligned(amax, 4)) return BITNET_ERR_ALIGN;
+    return from_cuda(launch_act_amax(x, M, K, amax, static_cast<cudaStream_t>(stream)));
+}
+
+bitnet_status bitnet_quant_act_amax(const uint16_t* x, int64_t M, int64_t K, const float* amax,
+                                    int8_t* q, float* s_x, void* stream) {
+    if (!x || !amax || !q || !s_x) return BITNET_ERR_NULL;
+    bitnet_status st = check_mk(M, K);
+    if (st != BITNET_OK) return st;
+    if (M * (K / 8) >= (int64_t(1) << 39)) return BITNET_ERR_UNSUPPORTED;
+    if (!aligned(x, 16) || !aligned(q, 16) || !aligned(amax, 4) || !aligned(s_x, 4))
+        return BITNET_ERR_ALIGN;
+    return from_cuda(launch_quant_amax(x, amax, M, K, q, s_x, static_cast<cudaStream_t>(stream)));
+}
+
+bitnet_status bitnet_dequant(const int32_t* acc, int64_t M, int64_t N, const float* s_x,
+                             const float* s_w, bitnet_scale_mode mode, void* y,
+                             bitnet_out_dtype out_dtype, void* stream) {
+    if (!acc || !s_x || !s_w || !y) return BITNET_ERR_NULL;
+    if (M < 1 || M >= (int64_t(1) << 31)) return BITNET_ERR_SHAPE;
+    bitnet_status st = check_n(N);
+    if (st != BITNET_OK) return st;
+    if (M * N >= (int64_t(1) << 39)) return BITNET_ERR_UNSUPPORTED;
+    if (mode != BITNET_SCALE_PER_TENSOR && mode != BITNET_SCALE_PER_ROW) return BITNET_ERR_UNSUPPORTED;
+    if (out_dtype != BITNET_OUT_BF16 && out_dtype != BITNET_OUT_F32) return BITNET_ERR_UNSUPPORTED;
+    if (!aligned(acc, 4) || !aligned(s_x, 4) || !aligned(s_w, 4) ||
+        !aligned(y, out_dtype == BITNET_OUT_BF16 ? 2 : 4))
+        return BITNET_ERR_ALIGN;
+    return from_cuda(launch_dequant(acc, M, N, s_x, s_w, mode == BITNET_SCALE_PER_ROW, y,
+                                    int(out_dtype), static_cast<cudaStream_t>(stream)));
+}
+
+bitnet_status bitnet_linear_plan(int64_t M, int64_t K, const int64_t* Ns, int32_t nproj,
+                                 int32_t swiglu, size_t workspace_bytes, bitnet_path path,
+                                 bitnet_plan* plan) {
+    if (!Ns || !plan) return BITNET_ERR_NULL;
+    if (path != BITNET_PATH_AUTO && path != BITNET_PATH_GEMV && path != BITNET_PATH_TC &&
+        path != BITNET_PATH_MMA)
+        return BITNET_ERR_UNSUPPORTED;
+    if (swiglu && nproj != 1) return BITNET_ERR_SHAPE;
+    // Stand-in addresses (never dereferenced): 256-byte aligned, as a real call's would be.
+    static const uintptr_t kFake = uintptr_t(1) << 40;
+    const void* fake = reinterpret_cast<const void*>(kFake);
+    if (nproj < 1 || nproj > kMaxProj) return BITNET_ERR_SHAPE;
+    bitnet_proj pr[kMaxProj];
+    for (int i = 0; i < nproj; ++i) {
+        pr[i].packed = static_cast<const uint8_t*>(fake);
+        pr[i].s_w = static_cast<const float*>(fake);
+        pr[i].mode = BITNET_SCALE_PER_TENSOR;
+        pr[i].reserved = 0;
+        pr[i].N = Ns[i];
+        pr[i].y = const_cast<void*>(fake);
+    }
+    if (swiglu && (Ns[0] % (2 * kSwigluBlock) != 0)) return BITNET_ERR_SHAPE;
+    Batch b;
+    bitnet_status st = validate_batch(fake, M, K, pr, nproj, /*out_kind=*/0, &b);
+    if (st != BITNET_OK) return st;
+    Plan pl;
+    st = plan_batch(static_cast<const uint16_t*>(fake), nullptr, M, K, b, 0,
+                    workspace_bytes ? fake : nullptr, workspace_bytes, path, swiglu != 0, false,
+                    &pl);
+    if (st != BITNET_OK) return st;
+    std::memset(plan, 0, sizeof(*plan));
+    plan->kernel = pl.kernel;
+    plan->grid = pl.kernel == BITNET_KERNEL_GEMV ? 0 : pl.grid;
+    plan->tile_tokens = pl.kernel == BITNET_KERNEL_TC ? pl.bn : 0;
+    plan->splits = pl.kernel == BITNET_KERNEL_TC ? pl.splits : 0;
+    plan->tile_rows = pl.kernel == BITNET_KERNEL_MMA_GEMV ? 16 * pl.rt : 0;
+    return BITNET_OK;
 }
 
 bitnet_status bitnet_check_device_errors(int32_t* flags) {

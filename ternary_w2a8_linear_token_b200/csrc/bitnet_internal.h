@@ -75,6 +75,20 @@ bool gemv_supported(int64_t M, int64_t K);
 // token count, width, path and workspace runs the GEMV (which uses no workspace).
 bool use_gemv(int64_t M, int64_t K, bitnet_path path, const void* ws, size_t ws_bytes);
 
+// Decode GEMV on warp-level tensor-core MMA (mma.sync m16n8k32) for M <= 8 tokens: CTAs of 8
+// warps own rt tiles of 16 weight rows, split over the warps by K. gemv_mma_plan returns false
+// where it does not apply (M > 8, or q of the tokens too large for shared memory); otherwise
+// the tiles per CTA, the grid and the packed chunks per lane.
+bool gemv_mma_plan(const GemvParams& p, int sms, int* rt, int* grid, int* cpt);
+// Where the warp-MMA GEMV runs (chains of calls on B200, 2B-4T and 8B-class shapes): one token
+// from 8 MiB of packed weights (17664 x 2560: 7.0 against 8.2 us per call for the dp4a GEMV;
+// 6912 x 2560: 4.3 against 4.1), five to eight tokens above 4 MiB (6912 x 2560 at 8 tokens:
+// 14.1 against 20.1 us; 4096 x 4096: 15.1 against 11.3). BITNET_PATH_MMA forces it.
+constexpr int64_t kMmaMinBytesOneToken = int64_t(8) << 20;
+constexpr int64_t kMmaMinBytesFewTokens = int64_t(4) << 20;
+cudaError_t launch_gemv_mma(const GemvParams& p, int rt, int grid, int cpt, int32_t* err,
+                            cudaStream_t stream, bool pdl);
+
 // Streaming GEMV for one token and large matrices (a producer warp fills a shared-memory
 // ring of 16-row weight stages with bulk copies; one CTA per SM). gemv_stream_plan returns
 // false where it does not apply (M != 1, contraction-only input, K > 16384, or a ring of
@@ -102,6 +116,16 @@ cudaError_t launch_quant(const uint16_t* x, const int8_t* q_in, int64_t M, int64
 int amax_parts_count(int64_t M, int64_t K);
 cudaError_t launch_amax_parts(const uint16_t* x, int64_t M, int64_t K, uint32_t* parts,
                               cudaStream_t stream, bool pdl);
+
+// ----------------------------------------------------------------------------- tensor parallel
+// The steps a rank runs when a projection's K range is split across ranks (kernels_tp.cu).
+cudaError_t launch_act_amax(const uint16_t* x, int64_t M, int64_t K, float* amax,
+                            cudaStream_t stream);
+cudaError_t launch_quant_amax(const uint16_t* x, const float* amax, int64_t M, int64_t K,
+                              int8_t* q, float* s_x, cudaStream_t stream);
+cudaError_t launch_dequant(const int32_t* acc, int64_t M, int64_t N, const float* s_x,
+                           const float* s_w, int per_row, void* y, int out_kind,
+                           cudaStream_t stream);
 
 // ----------------------------------------------------------------------------- packing
 cudaError_t launch_pack_weights(const float* W, int64_t N, int64_t K, int per_row,

@@ -17,6 +17,7 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include "act_quant_device.cuh"
 #include "bitnet_device.cuh"
 #include "bitnet_internal.h"
 #include "swiglu_device.cuh"
@@ -24,43 +25,9 @@
 namespace bitnet {
 namespace {
 
-constexpr float kEps = 1e-5f;
+constexpr float kEps = kActEps;
 constexpr int kWarps = 16;
 constexpr int kThreads = kWarps * 32;
-
-__device__ __forceinline__ float bf16_lo(uint32_t v) { return __uint_as_float(v << 16); }
-__device__ __forceinline__ float bf16_hi(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }
-
-// q = rint(x * s_x) as the low byte of a binary32. The definition's clamp to [-128, 127]
-// never acts here: s_x = RN(127 / a) with a = max(amax, 1e-5) >= |x|, so |x * s_x| <=
-// 127 (1 + 2^-24)^2 < 127.5. Adding 1.5 * 2^23 to the rounded product lands where the binary32
-// spacing is 1, so the sum is rint(x * s_x) + 1.5 * 2^23 (ties to even) and its low mantissa
-// byte is q in two's complement; both steps are separately rounded (no FMA contraction).
-__device__ __forceinline__ int q8(float xv, float s) {
-    return int(__float_as_uint(__fadd_rn(__fmul_rn(xv, s), 12582912.0f)));
-}
-
-// Low bytes of a, b, c, d -> one word (byte 0 = a).
-__device__ __forceinline__ uint32_t pack4(int a, int b, int c, int d) {
-    const uint32_t lo = __byte_perm(uint32_t(a), uint32_t(b), 0x0040);
-    const uint32_t hi = __byte_perm(uint32_t(c), uint32_t(d), 0x0040);
-    return __byte_perm(lo, hi, 0x5410);
-}
-
-// Sum of the four signed bytes of w.
-__device__ __forceinline__ int bytesum(uint32_t w) { return __dp4a(int(w), 0x01010101, 0); }
-
-// See kernels_quant.cu: lane pair (h = 0, 1) of one 16-group -> this lane's 8 permuted bytes.
-__device__ __forceinline__ uint2 permute_group_half(uint2 nat, int h) {
-    const uint32_t p01 = __byte_perm(nat.x, nat.y, 0x5140);
-    const uint32_t p23 = __byte_perm(nat.x, nat.y, 0x7362);
-    const uint32_t own = h ? p23 : p01;
-    const uint32_t send = h ? p01 : p23;
-    const uint32_t recv = __shfl_xor_sync(0xFFFFFFFFu, send, 1);
-    const uint32_t lo = h ? recv : own;
-    const uint32_t hi = h ? own : recv;
-    return make_uint2(__byte_perm(lo, hi, 0x5410), __byte_perm(lo, hi, 0x7632));
-}
 
 // MT: token capacity (compile time); p.M <= MT tokens are real, the rest are zero.
 // CPL: 16-byte chunks per lane (K <= CPL * 32 * 64). RW: weight rows per warp.
@@ -194,10 +161,10 @@ __global__ void __launch_bounds__(kThreads, MT <= 2 ? 2 : 1) gemv_w2a8_kernel(co
 #pragma unroll
             for (int m = 0; m < MT; ++m) {
                 const float s = s_tok[m];
-                nat[m].x = pack4(q8(bf16_lo(v[m].x), s), q8(bf16_hi(v[m].x), s),
-                                 q8(bf16_lo(v[m].y), s), q8(bf16_hi(v[m].y), s));
-                nat[m].y = pack4(q8(bf16_lo(v[m].z), s), q8(bf16_hi(v[m].z), s),
-                                 q8(bf16_lo(v[m].w), s), q8(bf16_hi(v[m].w), s));
+                nat[m].x = pack4(qbits(bf16_lo(v[m].x), s), qbits(bf16_hi(v[m].x), s),
+                                 qbits(bf16_lo(v[m].y), s), qbits(bf16_hi(v[m].y), s));
+                nat[m].y = pack4(qbits(bf16_lo(v[m].z), s), qbits(bf16_hi(v[m].z), s),
+                                 qbits(bf16_lo(v[m].w), s), qbits(bf16_hi(v[m].w), s));
             }
         } else {
 #pragma unroll

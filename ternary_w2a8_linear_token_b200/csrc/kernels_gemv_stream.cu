@@ -23,6 +23,7 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include "act_quant_device.cuh"
 #include "bitnet_device.cuh"
 #include "bitnet_internal.h"
 #include "swiglu_device.cuh"
@@ -30,42 +31,13 @@
 namespace bitnet {
 namespace {
 
-constexpr float kEps = 1e-5f;
+constexpr float kEps = kActEps;
 constexpr int kConsumers = 16;                     // consumer warps, one unit per stage each
 constexpr int kStreamThreads = (kConsumers + 1) * 32;  // warp 0 produces
 constexpr int kConsumerThreads = kConsumers * 32;
 constexpr int kMaxPiecesPerThread = 4;             // K <= 4 * 512 * 8 = 16384
 constexpr int kMaxDepth = 8;
 constexpr int kRingMax = 180 * 1024;
-
-__device__ __forceinline__ float bf16_lo(uint32_t v) { return __uint_as_float(v << 16); }
-__device__ __forceinline__ float bf16_hi(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }
-
-// q = rint(x * s) as the low byte of a binary32 (see kernels_gemv.cu: the clamp never acts).
-__device__ __forceinline__ int q8(float xv, float s) {
-    return int(__float_as_uint(__fadd_rn(__fmul_rn(xv, s), 12582912.0f)));
-}
-__device__ __forceinline__ uint32_t pack4(int a, int b, int c, int d) {
-    const uint32_t lo = __byte_perm(uint32_t(a), uint32_t(b), 0x0040);
-    const uint32_t hi = __byte_perm(uint32_t(c), uint32_t(d), 0x0040);
-    return __byte_perm(lo, hi, 0x5410);
-}
-__device__ __forceinline__ int bytesum(uint32_t w) { return __dp4a(int(w), 0x01010101, 0); }
-__device__ __forceinline__ uint2 permute_group_half(uint2 nat, int h) {
-    const uint32_t p01 = __byte_perm(nat.x, nat.y, 0x5140);
-    const uint32_t p23 = __byte_perm(nat.x, nat.y, 0x7362);
-    const uint32_t own = h ? p23 : p01;
-    const uint32_t send = h ? p01 : p23;
-    const uint32_t recv = __shfl_xor_sync(0xFFFFFFFFu, send, 1);
-    const uint32_t lo = h ? recv : own;
-    const uint32_t hi = h ? own : recv;
-    return make_uint2(__byte_perm(lo, hi, 0x5410), __byte_perm(lo, hi, 0x7632));
-}
-__device__ __forceinline__ uint32_t absmax8_bits(const uint4 v) {
-    const uint32_t a = max(max(v.x & 0x7FFFu, v.x >> 16 & 0x7FFFu), max(v.y & 0x7FFFu, v.y >> 16 & 0x7FFFu));
-    const uint32_t b = max(max(v.z & 0x7FFFu, v.z >> 16 & 0x7FFFu), max(v.w & 0x7FFFu, v.w >> 16 & 0x7FFFu));
-    return max(a, b);
-}
 
 // Barrier among the 16 consumer warps (named barrier 1); the producer never joins it.
 __device__ __forceinline__ void consumer_bar() {
@@ -193,10 +165,10 @@ __global__ void __launch_bounds__(kStreamThreads, 1)
     for (int t = 0; t < kMaxPiecesPerThread; ++t) {
         const int64_t c = ct + int64_t(t) * kConsumerThreads;  // lane pairs share a 16-group
         uint2 nat;
-        nat.x = pack4(q8(bf16_lo(xv[t].x), s_tok), q8(bf16_hi(xv[t].x), s_tok),
-                      q8(bf16_lo(xv[t].y), s_tok), q8(bf16_hi(xv[t].y), s_tok));
-        nat.y = pack4(q8(bf16_lo(xv[t].z), s_tok), q8(bf16_hi(xv[t].z), s_tok),
-                      q8(bf16_lo(xv[t].w), s_tok), q8(bf16_hi(xv[t].w), s_tok));
+        nat.x = pack4(qbits(bf16_lo(xv[t].x), s_tok), qbits(bf16_hi(xv[t].x), s_tok),
+                      qbits(bf16_lo(xv[t].y), s_tok), qbits(bf16_hi(xv[t].y), s_tok));
+        nat.y = pack4(qbits(bf16_lo(xv[t].z), s_tok), qbits(bf16_hi(xv[t].z), s_tok),
+                      qbits(bf16_lo(xv[t].w), s_tok), qbits(bf16_hi(xv[t].w), s_tok));
         qs += bytesum(nat.x) + bytesum(nat.y);  // padding pieces quantise to 0
         const uint2 out = permute_group_half(nat, lane & 1);
         if (c < pieces) {

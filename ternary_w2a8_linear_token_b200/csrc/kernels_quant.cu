@@ -17,63 +17,15 @@
 //    own the two 8-value halves of a group and swap 16-bit pieces with one shuffle.
 #include <cuda_runtime.h>
 
+#include "act_quant_device.cuh"
 #include "bitnet_device.cuh"
 #include "bitnet_internal.h"
 
 namespace bitnet {
 namespace {
 
-constexpr float kEps = 1e-5f;
+constexpr float kEps = kActEps;
 constexpr int kThreads = 256;
-
-__device__ __forceinline__ float bf16_bits_to_float(uint32_t b) {
-    return __uint_as_float(b << 16);
-}
-
-// q = clamp(rint(x * s_x), -128, 127) for one value, as the bits of a binary32 whose low byte
-// is q. The clamp never acts: s_x = RN(127 / a) with a = max(amax, 1e-5) >= |x|, so
-// |x * s_x| <= 127 (1 + 2^-24)^2 < 127.5. Adding 1.5 * 2^23 to the rounded product lands in
-// [2^23, 2^24), where the binary32 spacing is 1, so that sum is rint(x * s_x) + 1.5 * 2^23
-// (round half to even, as cvt.rni) and its low mantissa byte is q in two's complement.
-// Both steps are separately rounded intrinsics, so nothing is contracted into an FMA.
-__device__ __forceinline__ uint32_t qbits(float xv, float s) {
-    return __float_as_uint(__fadd_rn(__fmul_rn(xv, s), 12582912.0f));
-}
-
-// 8 bf16 (one uint4) -> 8 int8 as two 32-bit words (values k..k+3, k+4..k+7).
-__device__ __forceinline__ uint2 quant8(const uint4 v, float s) {
-    const uint32_t b0 = qbits(bf16_bits_to_float(v.x & 0xFFFFu), s);
-    const uint32_t b1 = qbits(__uint_as_float(v.x & 0xFFFF0000u), s);
-    const uint32_t b2 = qbits(bf16_bits_to_float(v.y & 0xFFFFu), s);
-    const uint32_t b3 = qbits(__uint_as_float(v.y & 0xFFFF0000u), s);
-    const uint32_t b4 = qbits(bf16_bits_to_float(v.z & 0xFFFFu), s);
-    const uint32_t b5 = qbits(__uint_as_float(v.z & 0xFFFF0000u), s);
-    const uint32_t b6 = qbits(bf16_bits_to_float(v.w & 0xFFFFu), s);
-    const uint32_t b7 = qbits(__uint_as_float(v.w & 0xFFFF0000u), s);
-    uint2 r;
-    r.x = __byte_perm(__byte_perm(b0, b1, 0x0040), __byte_perm(b2, b3, 0x0040), 0x5410);
-    r.y = __byte_perm(__byte_perm(b4, b5, 0x0040), __byte_perm(b6, b7, 0x0040), 0x5410);
-    return r;
-}
-
-__device__ __forceinline__ uint32_t absmax8_bits(const uint4 v) {
-    const uint32_t a = max(max(v.x & 0x7FFFu, v.x >> 16 & 0x7FFFu), max(v.y & 0x7FFFu, v.y >> 16 & 0x7FFFu));
-    const uint32_t b = max(max(v.z & 0x7FFFu, v.z >> 16 & 0x7FFFu), max(v.w & 0x7FFFu, v.w >> 16 & 0x7FFFu));
-    return max(a, b);
-}
-
-// Turns the natural-order words (lo = k..k+3, hi = k+4..k+7) held by lane pair
-// (2p, 2p+1) of one 16-group into that lane's 8 bytes of the permuted group.
-__device__ __forceinline__ uint2 permute_group_half(uint2 nat, int h) {
-    const uint32_t p01 = __byte_perm(nat.x, nat.y, 0x5140);  // pieces for words 0 and 1
-    const uint32_t p23 = __byte_perm(nat.x, nat.y, 0x7362);  // pieces for words 2 and 3
-    const uint32_t own = h ? p23 : p01;
-    const uint32_t send = h ? p01 : p23;
-    const uint32_t recv = __shfl_xor_sync(0xFFFFFFFFu, send, 1);
-    const uint32_t lo = h ? recv : own;  // pieces from the first 8 values of the group
-    const uint32_t hi = h ? own : recv;  // pieces from the last 8 values of the group
-    return make_uint2(__byte_perm(lo, hi, 0x5410), __byte_perm(lo, hi, 0x7632));
-}
 
 // Per-tensor activation scale ("BitNet 1-bit LLM推理优化" §2.2, I2_S; §3.2): the amax of the
 // whole input is the maximum of the partial maxima amax_parts_kernel wrote (whole warp).
@@ -130,7 +82,7 @@ __global__ void __launch_bounds__(kThreads) quant_rows_kernel(const uint16_t* __
         for (int u = 0; u < kRegPieces; ++u) mx = max(mx, absmax8_bits(v[u]));
         mx = __reduce_max_sync(0xFFFFFFFFu, mx);
         if (amax_parts) mx = parts_max(amax_parts, n_parts, lane);  // one scale per tensor
-        s = __fdiv_rn(127.0f, fmaxf(bf16_bits_to_float(mx), kEps));
+        s = __fdiv_rn(127.0f, fmaxf(bf16_lo(mx), kEps));
         if (lane == 0) {
             if (s_x) s_x[m] = s;
             if (r_x) r_x[m] = __frcp_rn(s);
@@ -165,7 +117,7 @@ __global__ void __launch_bounds__(kThreads) quant_rows_kernel(const uint16_t* __
         }
         mx = __reduce_max_sync(0xFFFFFFFFu, mx);
         if (amax_parts) mx = parts_max(amax_parts, n_parts, lane);  // one scale per tensor
-        s = __fdiv_rn(127.0f, fmaxf(bf16_bits_to_float(mx), kEps));
+        s = __fdiv_rn(127.0f, fmaxf(bf16_lo(mx), kEps));
         if (lane == 0) {
             if (s_x) s_x[m] = s;
             if (r_x) r_x[m] = __frcp_rn(s);
@@ -251,7 +203,7 @@ __global__ void __launch_bounds__(kLongThreads) quant_long_rows_kernel(
 #pragma unroll
     for (int w = 0; w < kLongRowThreads / 32; ++w) all = max(all, s_mx[row][w]);
     if (amax_parts) all = parts_max(amax_parts, n_parts, lane);  // one scale per tensor
-    const float s = __fdiv_rn(127.0f, fmaxf(bf16_bits_to_float(all), kEps));
+    const float s = __fdiv_rn(127.0f, fmaxf(bf16_lo(all), kEps));
     if (active && t == 0) {
         if (s_x) s_x[m] = s;
         if (r_x) r_x[m] = __frcp_rn(s);

@@ -204,3 +204,51 @@ def test_binding_rejects_wrong_shapes_before_the_call(bn):
     for i, call in enumerate(cases):
         with pytest.raises(ValueError):
             call()
+
+
+def test_plan_query_on_the_host(bn):
+    """bitnet_linear_plan runs without a device (148 SMs assumed) and reports the kernel
+    choices: the one-token kernels by size, the tensor-core tile width by token count, and
+    the same argument errors as the call it describes."""
+    assert bn.bitnet_linear_plan(1, 2560, [2560])["kernel"] == bn.KERNEL_GEMV
+    assert bn.bitnet_linear_plan(1, 2560, [2560], path=bn.PATH_MMA)["kernel"] == bn.KERNEL_MMA_GEMV
+    assert bn.bitnet_linear_plan(1, 2560, [2560, 640, 640, 6912, 6912])["kernel"] == \
+        bn.KERNEL_MMA_GEMV  # 11.3 MB: the warp-MMA GEMV
+    assert bn.bitnet_linear_plan(1, 4096, [4096, 1024, 1024, 14336, 14336])["kernel"] == \
+        bn.KERNEL_STREAM
+    assert bn.bitnet_linear_plan(3, 2560, [2560])["kernel"] == bn.KERNEL_GEMV
+    # rows longer than the warp-MMA kernel's largest slice: not available there
+    with pytest.raises(bn.BitnetError) as e:
+        bn.bitnet_linear_plan(1, 20480, [64], path=bn.PATH_MMA)
+    assert e.value.status == bn.ERR_UNSUPPORTED
+    p = bn.bitnet_linear_plan(4096, 4096, [4096, 1024, 1024, 14336, 14336])
+    assert p["kernel"] == bn.KERNEL_TC and p["tile_tokens"] == 192 and p["splits"] == 1
+    assert bn.bitnet_linear_plan(16, 2560, [2560])["tile_tokens"] == 16
+    assert bn.bitnet_linear_plan(5, 2560, [2560], workspace_bytes=0)["kernel"] == bn.KERNEL_GEMV
+    assert bn.bitnet_linear_plan(8, 2560, [6912], workspace_bytes=0)["kernel"] == bn.KERNEL_MMA_GEMV
+    with pytest.raises(bn.BitnetError) as e:
+        bn.bitnet_linear_plan(64, 2560, [2560], workspace_bytes=0)
+    assert e.value.status == bn.ERR_WORKSPACE
+    with pytest.raises(bn.BitnetError) as e:
+        bn.bitnet_linear_plan(1, 102, [64])  # K % 4 != 0
+    assert e.value.status == bn.ERR_SHAPE
+    with pytest.raises(bn.BitnetError) as e:
+        bn.bitnet_linear_plan(1, 2560, [100], swiglu=True)  # 2I must be a multiple of 32
+    assert e.value.status == bn.ERR_SHAPE
+
+
+def test_tensor_parallel_calls_argument_errors(bn):
+    lib = bn.lib
+    F = FAKE
+    assert lib.bitnet_act_amax(None, 1, 64, F, None) == bn.ERR_NULL
+    assert lib.bitnet_act_amax(F, 0, 64, F, None) == bn.ERR_SHAPE
+    assert lib.bitnet_act_amax(F, 1, 66, F, None) == bn.ERR_SHAPE
+    assert lib.bitnet_act_amax(F + 8, 1, 64, F, None) == bn.ERR_ALIGN
+    assert lib.bitnet_quant_act_amax(F, 1, 64, None, F, F, None) == bn.ERR_NULL
+    assert lib.bitnet_quant_act_amax(F, 1, 96, F, F, F, None) == bn.ERR_UNSUPPORTED
+    assert lib.bitnet_quant_act_amax(F, 1, 64, F, F + 4, F, None) == bn.ERR_ALIGN
+    assert lib.bitnet_dequant(F, 1, 8, F, None, 0, F, 0, None) == bn.ERR_NULL
+    assert lib.bitnet_dequant(F, 1, 0, F, F, 0, F, 0, None) == bn.ERR_SHAPE
+    assert lib.bitnet_dequant(F, 1, 8, F, F, 2, F, 0, None) == bn.ERR_UNSUPPORTED
+    assert lib.bitnet_dequant(F, 1, 8, F, F, 0, F, 7, None) == bn.ERR_UNSUPPORTED
+    assert lib.bitnet_dequant(F + 2, 1, 8, F, F, 0, F, 0, None) == bn.ERR_ALIGN
