@@ -134,9 +134,9 @@ bitnet_status plan_batch(const uint16_t* x_bf16, const int8_t* q_in, int64_t M, 
             p.proj[0].N = rows / 2;
         }
         // One token and a matrix too large for registers: stream it through a shared-memory
-        // ring. The warp-MMA GEMV where it measured faster than the dp4a GEMV in chains of
-        // calls on B200 (one token from kMmaMinBytesOneToken of packed weights, five to eight
-        // tokens above kMmaMinBytesFewTokens); the dp4a GEMV otherwise.
+        // ring. The warp-MMA GEMV where it measured faster than the dp4a GEMV on B200 (five to
+        // eight tokens above kMmaMinBytesFewTokens, reached without a workspace); the dp4a
+        // GEMV otherwise.
         const int64_t wbytes = rows * (K / 4);
         if (path == BITNET_PATH_MMA) {
             if (!gemv_mma_plan(p, tc_num_sms(), &pl->rt, &pl->grid, &pl->cpt))
@@ -144,9 +144,7 @@ bitnet_status plan_batch(const uint16_t* x_bf16, const int8_t* q_in, int64_t M, 
             pl->kernel = BITNET_KERNEL_MMA_GEMV;
             return BITNET_OK;
         }
-        const bool mma_pays = path == BITNET_PATH_AUTO &&
-                              (M == 1 ? wbytes >= kMmaMinBytesOneToken
-                                      : M >= 5 && wbytes > kMmaMinBytesFewTokens);
+        const bool mma_pays = path == BITNET_PATH_AUTO && M >= 5 && wbytes > kMmaMinBytesFewTokens;
         if (wbytes >= kStreamMinBytes &&
             gemv_stream_plan(p, &pl->n_stages, &pl->depth, &pl->stage_bytes)) {
             pl->kernel = BITNET_KERNEL_STREAM;

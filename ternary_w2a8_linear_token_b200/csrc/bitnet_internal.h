@@ -80,11 +80,12 @@ bool use_gemv(int64_t M, int64_t K, bitnet_path path, const void* ws, size_t ws_
 // where it does not apply (M > 8, or q of the tokens too large for shared memory); otherwise
 // the tiles per CTA, the grid and the packed chunks per lane.
 bool gemv_mma_plan(const GemvParams& p, int sms, int* rt, int* grid, int* cpt);
-// Where the warp-MMA GEMV runs (chains of calls on B200, 2B-4T and 8B-class shapes): one token
-// from 8 MiB of packed weights (17664 x 2560: 7.0 against 8.2 us per call for the dp4a GEMV;
-// 6912 x 2560: 4.3 against 4.1), five to eight tokens above 4 MiB (6912 x 2560 at 8 tokens:
-// 14.1 against 20.1 us; 4096 x 4096: 15.1 against 11.3). BITNET_PATH_MMA forces it.
-constexpr int64_t kMmaMinBytesOneToken = int64_t(8) << 20;
+// Where the warp-MMA GEMV runs under BITNET_PATH_AUTO: five to eight tokens (reached without a
+// workspace) above 4 MiB of packed weights (chains of calls on B200: 6912 x 2560 at 8 tokens
+// 14.1 against 20.1 us for the dp4a GEMV; 4096 x 4096, 4 MiB, 15.1 against 11.3). At one token
+// it lost to the dp4a GEMV everywhere but in chains of 11 MB batched calls (7.0 against 8.2 us),
+// and in the layer stacks, where it alternates with the dp4a GEMV, it lost there too (2B-4T
+// stack at M = 1: 465 against 431 us per pass); BITNET_PATH_MMA still forces it.
 constexpr int64_t kMmaMinBytesFewTokens = int64_t(4) << 20;
 cudaError_t launch_gemv_mma(const GemvParams& p, int rt, int grid, int cpt, int32_t* err,
                             cudaStream_t stream, bool pdl);

@@ -107,7 +107,6 @@ __global__ void __launch_bounds__(kMmaThreads) gemv_mma_kernel(const __grid_cons
     const int wrt = warp / ks;             // this warp's row tile within the CTA
     const int wks = warp - wrt * ks;       // and its K slice
     const int c0 = (wks * C) / ks, c1 = ((wks + 1) * C) / ks;
-    const int64_t tile = int64_t(blockIdx.x) * rt + wrt;
     const int64_t rows = SW ? 2 * p.total_rows : p.total_rows;  // packed rows in all
 
     // Base address of packed row r (null past the end); the batch's projections are laid
