@@ -65,11 +65,14 @@ def _load():
             lib.oracle_bitlinear_sampled.argtypes = [P, I64, I64, P, P, I, I64, P, I64, P, I64,
                                                      P, P, P, P, P, P, P]
             lib.oracle_swiglu.argtypes = [P, P, I64, P, P]
+            lib.oracle_pack_b3.argtypes = [P, I64, I64, P]
+            lib.oracle_unpack_b3.argtypes = [P, I64, I64, P]
             lib.oracle_quant_act_per_tensor.argtypes = [P, I64, I64, P, P]
             lib.oracle_quant_act_per_tensor.restype = ctypes.c_int
             for name in ("oracle_absmean_scale", "oracle_ternarize", "oracle_pack",
                          "oracle_unpack", "oracle_quant_act", "oracle_ternary_matmul",
-                         "oracle_dequant", "oracle_bitlinear_sampled", "oracle_swiglu"):
+                         "oracle_dequant", "oracle_bitlinear_sampled", "oracle_swiglu",
+                         "oracle_pack_b3", "oracle_unpack_b3"):
                 getattr(lib, name).restype = ctypes.c_int
             _lib = lib
     return _lib
@@ -124,6 +127,30 @@ def unpack(packed: np.ndarray, K: int) -> np.ndarray:
     N = packed.shape[0]
     t = np.empty((N, K), dtype=np.int8)
     _check(_load().oracle_unpack(_ptr(packed), N, K, _ptr(t)), "unpack")
+    return t
+
+
+def b3_row_bytes(K: int) -> int:
+    """Bytes of one row in the base-3 format: 16 per started chunk of 80 weights."""
+    return 16 * ((K + 79) // 80)
+
+
+def pack_b3(t: np.ndarray) -> np.ndarray:
+    """Five weights per byte in base 3 ("将 BitNet 三元查找表集成到自定义 Triton 内核中", step 1:
+    4-5 ternary values per byte): byte p of 80-weight chunk c holds k = 80c + 16d + p,
+    d = 0..4, as sum_d (t + 1) 3^d. Returns (N, b3_row_bytes(K)) uint8."""
+    t = np.ascontiguousarray(t, dtype=np.int8)
+    N, K = t.shape
+    p = np.empty((N, b3_row_bytes(K)), dtype=np.uint8)
+    _check(_load().oracle_pack_b3(_ptr(t), N, K, _ptr(p)), "pack_b3")
+    return p
+
+
+def unpack_b3(packed: np.ndarray, K: int) -> np.ndarray:
+    packed = np.ascontiguousarray(packed, dtype=np.uint8)
+    N = packed.shape[0]
+    t = np.empty((N, K), dtype=np.int8)
+    _check(_load().oracle_unpack_b3(_ptr(packed), N, K, _ptr(t)), "unpack_b3")
     return t
 
 

@@ -31,6 +31,8 @@
  *           or per-channel.
  *  [P2-2.2] same page, section 2.2 "I2_S（Int2 with Scale）内核": follows the
  *           per-tensor int8 activation quantisation BitNet b1.58 was trained with.
+ *  [P3-1]   "将 BitNet 三元查找表集成到自定义 Triton 内核中", step 1 of its recipe:
+ *           ternary values packed into uint8 bitmaps, 4-5 of them per byte.
  *
  * Readings where the pages are silent (each one is listed in the design notes):
  *  - code = t + 1 (00 = -1, 01 = 0, 10 = +1); code 11 never appears. Section 4.3
@@ -153,6 +155,63 @@ int oracle_unpack(const uint8_t* packed, int64_t N, int64_t K, int8_t* t) {
             unsigned code = (byte >> (2 * (k % 4))) & 3u;
             if (code == 3u) return ORACLE_BAD_DATA;
             t[n * K + k] = (int8_t)((int)code - 1);
+        }
+    }
+    return ORACLE_OK;
+}
+
+/* ---------------------------------------------------------------------------
+ * Base-3 packing, five weights per byte ([P3-1] "每个 8-bit 字节存储 4-5 个三元值":
+ * 3^5 = 243 <= 256, 1.6 bits per weight). The digit of a weight is its code t + 1,
+ * least significant digit first. The pages fix no layout; the one read here: a row
+ * is cut into chunks of 80 weights (16 bytes), and byte p (0..15) of chunk c holds
+ * the weights k = 80c + 16d + p for d = 0..4 as sum_d (t + 1) * 3^d. Weights past
+ * K count as t = 0. A row takes 16 * ceil(K / 80) bytes.
+ * ------------------------------------------------------------------------- */
+static int64_t b3_row_bytes(int64_t K) { return 16 * ((K + 79) / 80); }
+
+int oracle_pack_b3(const int8_t* t, int64_t N, int64_t K, uint8_t* packed) {
+    if (!t || !packed || N <= 0 || K <= 0) return ORACLE_BAD_ARG;
+    const int64_t rb = b3_row_bytes(K);
+    for (int64_t n = 0; n < N; ++n) {
+        for (int64_t j = 0; j < rb; ++j) {
+            const int64_t c = j / 16, p = j % 16;
+            unsigned byte = 0, place = 1;
+            for (int d = 0; d < 5; ++d) {
+                const int64_t k = 80 * c + 16 * d + p;
+                int w = 0;
+                if (k < K) {
+                    w = t[n * K + k];
+                    if (w < -1 || w > 1) return ORACLE_BAD_DATA;
+                }
+                byte += (unsigned)(w + 1) * place;
+                place *= 3u;
+            }
+            packed[n * rb + j] = (uint8_t)byte;
+        }
+    }
+    return ORACLE_OK;
+}
+
+/* Inverse of oracle_pack_b3. A byte above 242 (no five digits), or a padding weight
+ * that is not 0, is reported as bad data. */
+int oracle_unpack_b3(const uint8_t* packed, int64_t N, int64_t K, int8_t* t) {
+    if (!t || !packed || N <= 0 || K <= 0) return ORACLE_BAD_ARG;
+    const int64_t rb = b3_row_bytes(K);
+    for (int64_t n = 0; n < N; ++n) {
+        for (int64_t j = 0; j < rb; ++j) {
+            const int64_t c = j / 16, p = j % 16;
+            unsigned byte = packed[n * rb + j];
+            if (byte > 242u) return ORACLE_BAD_DATA;
+            for (int d = 0; d < 5; ++d) {
+                const int w = (int)(byte % 3u) - 1;
+                byte /= 3u;
+                const int64_t k = 80 * c + 16 * d + p;
+                if (k < K)
+                    t[n * K + k] = (int8_t)w;
+                else if (w != 0)
+                    return ORACLE_BAD_DATA;
+            }
         }
     }
     return ORACLE_OK;

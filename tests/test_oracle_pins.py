@@ -530,3 +530,59 @@ def test_bitlinear_per_tensor_act_matches_float_linear(oracle):
     m_idx, n_idx = np.array([0, 3, 4]), np.array([1, 7, 23])
     rs = oracle.bitlinear_sampled_per_tensor_act(x, oracle.pack(t), s_w, True, K, m_idx, n_idx)
     assert np.array_equal(rs["y"], r["y"][np.ix_(m_idx, n_idx)])
+
+
+# ---------------------------------------------------------------- base-3 packing (5 per byte)
+
+def test_pack_b3_hand_derived_bytes(oracle):
+    """The fixture's row (K = 80) packs to the bytes derived by hand from the layout."""
+    g = read_golden("pack_b3_example.txt")
+    t = np.zeros((1, 80), dtype=np.int8)
+    t[0, [int(v) for v in g["neg"]]] = -1
+    t[0, [int(v) for v in g["pos"]]] = 1
+    want = np.array([int(v) for v in g["bytes"]], dtype=np.uint8)
+    assert np.array_equal(oracle.pack_b3(t)[0], want)
+
+
+def test_pack_b3_digit_places(oracle):
+    """Each weight of a chunk moves its byte by 3^d in its own byte only: weight k = 16d + p of
+    chunk c sets digit d of byte 16c + p."""
+    K = 160
+    base = oracle.pack_b3(np.zeros((1, K), dtype=np.int8))[0].astype(np.int64)
+    assert np.all(base == 121)
+    for k in (0, 15, 16, 37, 79, 80, 101, 159):
+        c, r = divmod(k, 80)
+        d, p = divmod(r, 16)
+        for w, delta in ((1, 1), (-1, -1)):
+            t = np.zeros((1, K), dtype=np.int8)
+            t[0, k] = w
+            got = oracle.pack_b3(t)[0].astype(np.int64) - base
+            want = np.zeros_like(got)
+            want[16 * c + p] = delta * 3 ** d
+            assert np.array_equal(got, want), (k, w)
+
+
+@pytest.mark.parametrize("K", [64, 80, 100, 2560, 4096, 6912])
+def test_pack_b3_roundtrip_and_range(oracle, K):
+    g = np.random.default_rng(K)
+    t = g.integers(-1, 2, size=(7, K)).astype(np.int8)
+    p = oracle.pack_b3(t)
+    assert p.shape == (7, 16 * ((K + 79) // 80)) and int(p.max()) <= 242
+    assert np.array_equal(oracle.unpack_b3(p, K), t)
+    # 1.6 bits per weight, up to the padding of the last chunk
+    assert p.shape[1] * 8 <= 1.6 * K + 16 * 8
+
+
+def test_unpack_b3_rejects_bad_bytes_and_padding(oracle):
+    t = np.zeros((1, 64), dtype=np.int8)
+    p = oracle.pack_b3(t)
+    bad = p.copy()
+    bad[0, 3] = 243  # no five base-3 digits
+    with pytest.raises(oracle.OracleError):
+        oracle.unpack_b3(bad, 64)
+    pad = p.copy()
+    pad[0, 0] = 121 + 81  # digit 4 of byte 0 is weight k = 64, past K = 64: must stay 0
+    with pytest.raises(oracle.OracleError):
+        oracle.unpack_b3(pad, 64)
+    with pytest.raises(oracle.OracleError):
+        oracle.pack_b3(np.full((1, 64), 2, dtype=np.int8))
