@@ -295,6 +295,27 @@ bitnet_status bitnet_linear_noalloc(const uint16_t* x, int64_t M, int64_t K,
                                     bitnet_out_dtype out_dtype, void* stream);
 
 /*
+ * Base-3 weight format, five ternary weights per byte (page "将 BitNet 三元查找表集成到自定义
+ * Triton 内核中", step 1: 4-5 ternary values per 8-bit byte; 3^5 = 243 <= 256, so 1.6 bits
+ * per weight against 2). Row n is cut into chunks of 80 weights (16 bytes); byte p of chunk c
+ * holds weights k = 80c + 16d + p, d = 0..4, as sum_d (t + 1) * 3^d; weights past K count as
+ * 0. A row takes bitnet_b3_row_bytes(K) = 16 * ceil(K / 80) bytes.
+ *
+ * bitnet_pack_ternary_b3 — t (N, K) int8 in {-1, 0, +1} -> packed (N, bitnet_b3_row_bytes(K))
+ *   uint8, 16-byte aligned; K as for the other calls (a multiple of 64).
+ * bitnet_linear_b3 — bitnet_linear for one token (M = 1; BITNET_ERR_UNSUPPORTED otherwise)
+ *   on base-3 weights, K <= 16384: the same quantiser, contraction and epilogue arithmetic,
+ *   so its output equals bitnet_linear on the 2-bit packing of the same weights bit for bit.
+ *   y (1, N) 16-byte aligned. No workspace. Asynchronous on `stream`.
+ */
+int64_t bitnet_b3_row_bytes(int64_t K);
+bitnet_status bitnet_pack_ternary_b3(const int8_t* t, int64_t N, int64_t K, uint8_t* packed,
+                                     void* stream);
+bitnet_status bitnet_linear_b3(const uint16_t* x, int64_t M, int64_t K, const uint8_t* packed_b3,
+                               const float* s_w, bitnet_scale_mode mode, int64_t N, void* y,
+                               bitnet_out_dtype out_dtype, void* stream);
+
+/*
  * Tensor-parallel steps ("BitNet：1-bit LLM推理框架技术实战指南", section on the distributed
  * engine: a model split by layer or by tensor across devices). When a projection's K range is
  * split over ranks (rank r holds x[:, k0:k1] and packed[:, k0/4 : k1/4], k0 and k1 multiples

@@ -89,6 +89,10 @@ _SIGS = {
                                   ctypes.c_int),
     "bitnet_linear_swiglu": ([_P, _I64, _I64, _P, _P, ctypes.c_int, _I64, _P, _P, _SZ,
                              ctypes.c_int, _P], ctypes.c_int),
+    "bitnet_b3_row_bytes": ([_I64], _I64),
+    "bitnet_pack_ternary_b3": ([_P, _I64, _I64, _P, _P], ctypes.c_int),
+    "bitnet_linear_b3": ([_P, _I64, _I64, _P, _P, ctypes.c_int, _I64, _P, ctypes.c_int, _P],
+                         ctypes.c_int),
     "bitnet_act_amax": ([_P, _I64, _I64, _P, _P], ctypes.c_int),
     "bitnet_quant_act_amax": ([_P, _I64, _I64, _P, _P, _P, _P], ctypes.c_int),
     "bitnet_dequant": ([_P, _I64, _I64, _P, _P, ctypes.c_int, _P, ctypes.c_int, _P], ctypes.c_int),
@@ -383,6 +387,35 @@ def bitnet_linear_noalloc(x: torch.Tensor, packed: torch.Tensor, s_w: torch.Tens
                                      _dev(s_w, torch.float32, "s_w"), int(bool(per_row)), N,
                                      _dev(y, y.dtype, "y"), od, _stream(stream)),
            "bitnet_linear_noalloc")
+    return y
+
+
+def bitnet_pack_ternary_b3(t: torch.Tensor, stream=None) -> torch.Tensor:
+    """Ternary (N, K) int8 -> the base-3 format, five weights per byte (N, 16 ceil(K / 80))."""
+    N, K = t.shape
+    packed = torch.empty((N, int(lib.bitnet_b3_row_bytes(K))), dtype=torch.uint8, device=t.device)
+    _check(lib.bitnet_pack_ternary_b3(_dev(t, torch.int8, "t"), N, K, packed.data_ptr(),
+                                      _stream(stream)), "bitnet_pack_ternary_b3")
+    return packed
+
+
+def bitnet_linear_b3(x: torch.Tensor, packed_b3: torch.Tensor, s_w: torch.Tensor, per_row: bool,
+                     out_dtype: torch.dtype = torch.bfloat16, y: Optional[torch.Tensor] = None,
+                     stream=None) -> torch.Tensor:
+    """bitnet_linear for one token on base-3 weights (bitnet_pack_ternary_b3)."""
+    M, K = x.shape
+    N = packed_b3.shape[0]
+    if packed_b3.dim() != 2 or packed_b3.shape[1] != int(lib.bitnet_b3_row_bytes(K)):
+        raise ValueError("packed_b3 must be (N, bitnet_b3_row_bytes(K))")
+    if s_w.numel() != (N if per_row else 1):
+        raise ValueError("s_w must have N (per row) or 1 elements")
+    if y is None:
+        y = torch.empty((M, N), dtype=out_dtype, device=x.device)
+    _check_out(y, M, N)
+    od = OUT_BF16 if y.dtype == torch.bfloat16 else OUT_F32
+    _check(lib.bitnet_linear_b3(_x_ptr(x), M, K, _dev(packed_b3, torch.uint8, "packed_b3"),
+                                _dev(s_w, torch.float32, "s_w"), int(bool(per_row)), N,
+                                _dev(y, y.dtype, "y"), od, _stream(stream)), "bitnet_linear_b3")
     return y
 
 

@@ -577,6 +577,46 @@ bitnet_status bitnet_linear_swiglu(const uint16_t* x, int64_t M, int64_t K,
                      static_cast<cudaStream_t>(stream), /*swiglu=*/true);
 }
 
+int64_t bitnet_b3_row_bytes(int64_t K) { return K < 1 ? 0 : b3_row_bytes(K); }
+
+bitnet_status bitnet_pack_ternary_b3(const int8_t* t, int64_t N, int64_t K, uint8_t* packed,
+                                     void* stream) {
+    if (!t || !packed) return BITNET_ERR_NULL;
+    bitnet_status st = check_mk(1, K);
+    if (st != BITNET_OK) return st;
+    if ((st = check_n(N)) != BITNET_OK) return st;
+    if (!aligned(t, 16) || !aligned(packed, 16)) return BITNET_ERR_ALIGN;
+    return from_cuda(launch_pack_b3(t, N, K, packed, static_cast<cudaStream_t>(stream)));
+}
+
+bitnet_status bitnet_linear_b3(const uint16_t* x, int64_t M, int64_t K, const uint8_t* packed_b3,
+                               const float* s_w, bitnet_scale_mode mode, int64_t N, void* y,
+                               bitnet_out_dtype out_dtype, void* stream) {
+    if (!x || !packed_b3 || !s_w || !y) return BITNET_ERR_NULL;
+    bitnet_status st = check_mk(M, K);
+    if (st != BITNET_OK) return st;
+    if ((st = check_n(N)) != BITNET_OK) return st;
+    if (M != 1 || !gemv_b3_supported(K)) return BITNET_ERR_UNSUPPORTED;
+    if (mode != BITNET_SCALE_PER_TENSOR && mode != BITNET_SCALE_PER_ROW) return BITNET_ERR_UNSUPPORTED;
+    if (out_dtype != BITNET_OUT_BF16 && out_dtype != BITNET_OUT_F32) return BITNET_ERR_UNSUPPORTED;
+    if (!aligned(x, 16) || !aligned(packed_b3, 16) || !aligned(y, 16) || !aligned(s_w, 4))
+        return BITNET_ERR_ALIGN;
+    GemvParams p;
+    std::memset(&p, 0, sizeof(p));
+    p.x = x;
+    p.K = K;
+    p.M = 1;
+    p.nproj = 1;
+    p.out_kind = int(out_dtype);
+    p.total_rows = N;
+    p.proj[0].packed = packed_b3;
+    p.proj[0].s_w = s_w;
+    p.proj[0].y = y;
+    p.proj[0].N = N;
+    p.proj[0].per_row = mode == BITNET_SCALE_PER_ROW;
+    return from_cuda(launch_gemv_b3(p, tc_num_sms(), static_cast<cudaStream_t>(stream), true));
+}
+
 bitnet_status bitnet_act_amax(const uint16_t* x, int64_t M, int64_t K, float* amax, void* stream) {
     if (!x || !amax) return BITNET_ERR_NULL;
     bitnet_status st = check_mk(M, K);

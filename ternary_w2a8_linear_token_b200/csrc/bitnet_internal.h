@@ -118,6 +118,14 @@ int amax_parts_count(int64_t M, int64_t K);
 cudaError_t launch_amax_parts(const uint16_t* x, int64_t M, int64_t K, uint32_t* parts,
                               cudaStream_t stream, bool pdl);
 
+// ----------------------------------------------------------------------------- base-3 weights
+// Five ternary weights per byte (kernels_b3.cu): bytes per row, 16 per started 80-weight chunk.
+__host__ __device__ inline int64_t b3_row_bytes(int64_t K) { return 16 * ((K + 79) / 80); }
+cudaError_t launch_pack_b3(const int8_t* t, int64_t N, int64_t K, uint8_t* packed,
+                           cudaStream_t stream);
+bool gemv_b3_supported(int64_t K);
+cudaError_t launch_gemv_b3(const GemvParams& p, int sms, cudaStream_t stream, bool pdl);
+
 // ----------------------------------------------------------------------------- tensor parallel
 // The steps a rank runs when a projection's K range is split across ranks (kernels_tp.cu).
 cudaError_t launch_act_amax(const uint16_t* x, int64_t M, int64_t K, float* amax,

@@ -213,7 +213,7 @@ def test_plan_query_on_the_host(bn):
     assert bn.bitnet_linear_plan(1, 2560, [2560])["kernel"] == bn.KERNEL_GEMV
     assert bn.bitnet_linear_plan(1, 2560, [2560], path=bn.PATH_MMA)["kernel"] == bn.KERNEL_MMA_GEMV
     assert bn.bitnet_linear_plan(1, 2560, [2560, 640, 640, 6912, 6912])["kernel"] == \
-        bn.KERNEL_MMA_GEMV  # 11.3 MB: the warp-MMA GEMV
+        bn.KERNEL_GEMV  # 11.3 MB, below the streaming threshold
     assert bn.bitnet_linear_plan(1, 4096, [4096, 1024, 1024, 14336, 14336])["kernel"] == \
         bn.KERNEL_STREAM
     assert bn.bitnet_linear_plan(3, 2560, [2560])["kernel"] == bn.KERNEL_GEMV
@@ -252,3 +252,22 @@ def test_tensor_parallel_calls_argument_errors(bn):
     assert lib.bitnet_dequant(F, 1, 8, F, F, 2, F, 0, None) == bn.ERR_UNSUPPORTED
     assert lib.bitnet_dequant(F, 1, 8, F, F, 0, F, 7, None) == bn.ERR_UNSUPPORTED
     assert lib.bitnet_dequant(F + 2, 1, 8, F, F, 0, F, 0, None) == bn.ERR_ALIGN
+
+
+def test_b3_calls_argument_errors(bn):
+    lib, F = bn.lib, FAKE
+    assert lib.bitnet_b3_row_bytes(64) == 16 and lib.bitnet_b3_row_bytes(2560) == 512
+    assert lib.bitnet_b3_row_bytes(4096) == 832 and lib.bitnet_b3_row_bytes(0) == 0
+    assert lib.bitnet_pack_ternary_b3(None, 4, 64, F, None) == bn.ERR_NULL
+    assert lib.bitnet_pack_ternary_b3(F, 4, 66, F, None) == bn.ERR_SHAPE
+    assert lib.bitnet_pack_ternary_b3(F + 1, 4, 64, F, None) == bn.ERR_ALIGN
+    args = dict(x=F, M=1, K=64, p=F, s=F, mode=0, N=8, y=F, od=0)
+    def call(**kw):
+        a = dict(args, **kw)
+        return lib.bitnet_linear_b3(a["x"], a["M"], a["K"], a["p"], a["s"], a["mode"], a["N"],
+                                    a["y"], a["od"], None)
+    assert call(M=2) == bn.ERR_UNSUPPORTED      # one token only
+    assert call(K=16448) == bn.ERR_UNSUPPORTED  # K <= 16384
+    assert call(p=None) == bn.ERR_NULL
+    assert call(mode=3) == bn.ERR_UNSUPPORTED and call(od=5) == bn.ERR_UNSUPPORTED
+    assert call(y=F + 2) == bn.ERR_ALIGN
