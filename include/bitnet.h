@@ -358,6 +358,7 @@ bitnet_status bitnet_dequant(const int32_t* acc, int64_t M, int64_t N, const flo
 #define BITNET_KERNEL_MMA_GEMV 2 /* warp-level tensor-core GEMV (mma.sync), up to 8 tokens  */
 #define BITNET_KERNEL_STREAM 3 /* one-token streaming GEMV through a shared-memory ring      */
 #define BITNET_KERNEL_TC 4     /* quantiser kernel, then the tcgen05 tensor-core GEMM         */
+#define BITNET_KERNEL_GS 5     /* one-token grid-stride GEMV for large matrices               */
 typedef struct {
     int32_t kernel;        /* BITNET_KERNEL_*                                               */
     int32_t grid;          /* CTAs of the main kernel (0 for BITNET_KERNEL_GEMV)            */

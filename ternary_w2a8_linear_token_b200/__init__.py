@@ -64,7 +64,7 @@ class bitnet_plan(ctypes.Structure):
                 ("tile_rows", _I32), ("reserved", _I32 * 3)]
 
 
-KERNEL_GEMV, KERNEL_MMA_GEMV, KERNEL_STREAM, KERNEL_TC = 1, 2, 3, 4
+KERNEL_GEMV, KERNEL_MMA_GEMV, KERNEL_STREAM, KERNEL_TC, KERNEL_GS = 1, 2, 3, 4, 5
 
 _SIGS = {
     "bitnet_pack_weights": ([_P, _I64, _I64, ctypes.c_int, _P, _P, _P], ctypes.c_int),

@@ -133,8 +133,9 @@ bitnet_status plan_batch(const uint16_t* x_bf16, const int8_t* q_in, int64_t M, 
             p.total_rows = rows / 2;
             p.proj[0].N = rows / 2;
         }
-        // One token and a matrix too large for registers: stream it through a shared-memory
-        // ring. The warp-MMA GEMV where it measured faster than the dp4a GEMV on B200 (five to
+        // One token and a matrix too large for one wave of register-resident rows: the
+        // streaming kernel, or for the MLP's gate/up pairs with rows of at most kGsMaxK the
+        // grid-stride kernel (measured faster there on B200, slower on plain projections). The warp-MMA GEMV where it measured faster than the dp4a GEMV on B200 (five to
         // eight tokens above kMmaMinBytesFewTokens, reached without a workspace); the dp4a
         // GEMV otherwise.
         const int64_t wbytes = rows * (K / 4);
@@ -145,8 +146,13 @@ bitnet_status plan_batch(const uint16_t* x_bf16, const int8_t* q_in, int64_t M, 
             return BITNET_OK;
         }
         const bool mma_pays = path == BITNET_PATH_AUTO && M >= 5 && wbytes > kMmaMinBytesFewTokens;
-        if (wbytes >= kStreamMinBytes &&
-            gemv_stream_plan(p, &pl->n_stages, &pl->depth, &pl->stage_bytes)) {
+        if (wbytes >= kStreamMinBytes && swiglu && K <= kGsMaxK && gemv_gs_supported(p, false)) {
+            pl->kernel = BITNET_KERNEL_GS;
+            const int64_t per_cta = swiglu ? 16 : 32;
+            const int64_t want = (p.total_rows + per_cta - 1) / per_cta;
+            pl->grid = static_cast<int>(want < tc_num_sms() ? want : tc_num_sms());
+        } else if (wbytes >= kStreamMinBytes &&
+                   gemv_stream_plan(p, &pl->n_stages, &pl->depth, &pl->stage_bytes)) {
             pl->kernel = BITNET_KERNEL_STREAM;
             pl->grid = static_cast<int>(pl->n_stages < tc_num_sms() ? pl->n_stages : tc_num_sms());
         } else if (mma_pays && gemv_mma_plan(p, tc_num_sms(), &pl->rt, &pl->grid, &pl->cpt)) {
@@ -218,6 +224,8 @@ bitnet_status run_batch(const uint16_t* x_bf16, const int8_t* q_in, int64_t M, i
     bitnet_status pst = plan_batch(x_bf16, q_in, M, K, b, out_kind, workspace, workspace_bytes,
                                    path, swiglu, act_per_tensor, &pl);
     if (pst != BITNET_OK) return pst;
+    if (pl.kernel == BITNET_KERNEL_GS)
+        return from_cuda(launch_gemv_gs(pl.gp, /*b3=*/false, tc_num_sms(), stream, /*pdl=*/true));
     if (pl.kernel == BITNET_KERNEL_STREAM) {
         int32_t* err = device_error_word();
         if (!err) return BITNET_ERR_CUDA;
@@ -596,7 +604,7 @@ bitnet_status bitnet_linear_b3(const uint16_t* x, int64_t M, int64_t K, const ui
     bitnet_status st = check_mk(M, K);
     if (st != BITNET_OK) return st;
     if ((st = check_n(N)) != BITNET_OK) return st;
-    if (M != 1 || !gemv_b3_supported(K)) return BITNET_ERR_UNSUPPORTED;
+    if (M != 1 || K > 16384) return BITNET_ERR_UNSUPPORTED;
     if (mode != BITNET_SCALE_PER_TENSOR && mode != BITNET_SCALE_PER_ROW) return BITNET_ERR_UNSUPPORTED;
     if (out_dtype != BITNET_OUT_BF16 && out_dtype != BITNET_OUT_F32) return BITNET_ERR_UNSUPPORTED;
     if (!aligned(x, 16) || !aligned(packed_b3, 16) || !aligned(y, 16) || !aligned(s_w, 4))
@@ -614,7 +622,8 @@ bitnet_status bitnet_linear_b3(const uint16_t* x, int64_t M, int64_t K, const ui
     p.proj[0].y = y;
     p.proj[0].N = N;
     p.proj[0].per_row = mode == BITNET_SCALE_PER_ROW;
-    return from_cuda(launch_gemv_b3(p, tc_num_sms(), static_cast<cudaStream_t>(stream), true));
+    return from_cuda(launch_gemv_gs(p, /*b3=*/true, tc_num_sms(), static_cast<cudaStream_t>(stream),
+                                    true));
 }
 
 bitnet_status bitnet_act_amax(const uint16_t* x, int64_t M, int64_t K, float* amax, void* stream) {

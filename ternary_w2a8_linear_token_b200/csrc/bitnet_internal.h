@@ -123,8 +123,16 @@ cudaError_t launch_amax_parts(const uint16_t* x, int64_t M, int64_t K, uint32_t*
 __host__ __device__ inline int64_t b3_row_bytes(int64_t K) { return 16 * ((K + 79) / 80); }
 cudaError_t launch_pack_b3(const int8_t* t, int64_t N, int64_t K, uint8_t* packed,
                            cudaStream_t stream);
-bool gemv_b3_supported(int64_t K);
-cudaError_t launch_gemv_b3(const GemvParams& p, int sms, cudaStream_t stream, bool pdl);
+// Grid-stride one-token GEMV (kernels_gemv_gs.cu) for large matrices, 2-bit or base-3 (b3)
+// weights: one 16-warp CTA per SM, each warp a ring of row pairs in registers.
+bool gemv_gs_supported(const GemvParams& p, bool b3);
+cudaError_t launch_gemv_gs(const GemvParams& p, bool b3, int sms, cudaStream_t stream, bool pdl);
+// The grid-stride kernel replaces the streaming one for one-token SwiGLU calls from
+// kStreamMinBytes with rows of at most this many K values (two chunks per lane, four row pairs
+// in flight per warp). On B200 (µs per call): 8B-class gate/up + SwiGLU 28672 x 4096 12.3
+// against 13.8; plain projections lost or tied (35.7 MB 8B q/k/v/gate/up batch 17.4 against
+// 15.9; 50011 x 1024 17.4 against 14.7; 14336 x 4096 and a 14.6 MB 2B-4T batch equal).
+constexpr int64_t kGsMaxK = 4096;
 
 // ----------------------------------------------------------------------------- tensor parallel
 // The steps a rank runs when a projection's K range is split across ranks (kernels_tp.cu).

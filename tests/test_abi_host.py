@@ -215,7 +215,9 @@ def test_plan_query_on_the_host(bn):
     assert bn.bitnet_linear_plan(1, 2560, [2560, 640, 640, 6912, 6912])["kernel"] == \
         bn.KERNEL_GEMV  # 11.3 MB, below the streaming threshold
     assert bn.bitnet_linear_plan(1, 4096, [4096, 1024, 1024, 14336, 14336])["kernel"] == \
-        bn.KERNEL_STREAM
+        bn.KERNEL_STREAM  # 35.6 MB: the streaming GEMV
+    assert bn.bitnet_linear_plan(1, 4096, [28672], swiglu=True)["kernel"] == bn.KERNEL_GS
+    assert bn.bitnet_linear_plan(1, 14336, [4096])["kernel"] == bn.KERNEL_STREAM  # longer rows
     assert bn.bitnet_linear_plan(3, 2560, [2560])["kernel"] == bn.KERNEL_GEMV
     # rows longer than the warp-MMA kernel's largest slice: not available there
     with pytest.raises(bn.BitnetError) as e:

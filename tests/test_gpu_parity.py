@@ -260,20 +260,23 @@ def test_8b_stack_projection_sampled(bn, oracle):
 
 
 # One token and at least 12 MiB of packed weights per call: the streaming GEMV (producer warp,
-# shared-memory ring of 16-row stages). Ragged projections (N not a multiple of 16), every
-# chunks-per-lane class, per-row scales, fp32 output, whole outputs against the oracle.
-STREAM_CASES = [  # (Ns of the batch, K, per_row)
-    ((2560, 640, 640, 6912, 6912, 2560, 2560), 2560, False),  # 2B-4T projections, batched
-    ((4096, 14336 + 7), 4096, True),              # ragged last stage
-    ((4096,), 14336, True),                       # 8B down projection, K = 14336
-    ((9001,), 6912, False),                       # 4 chunks per lane, ragged
-    ((3000, 50011), 1024, True),                  # 1 chunk per lane
+# shared-memory ring of 16-row stages; the grid-stride GEMV takes only SwiGLU calls, tested in
+# test_gpu_swiglu). Ragged projections (N not a multiple of 16), every chunks-per-lane class,
+# per-row scales, fp32 output, whole outputs against the oracle.
+STREAM_CASES = [  # (Ns of the batch, K, per_row, kernel)
+    ((2560, 640, 640, 6912, 6912, 2560, 2560), 2560, False, "stream"),  # 2B-4T projections
+    ((4096, 14336 + 7), 4096, True, "stream"),    # ragged last rows
+    ((4096,), 14336, True, "stream"),             # 8B down projection, K = 14336
+    ((9001,), 6912, False, "stream"),             # 4 chunks per lane, ragged
+    ((3000, 50011), 1024, True, "stream"),        # 1 chunk per lane
 ]
 
 
-@pytest.mark.parametrize("Ns,K,per_row", STREAM_CASES)
-def test_stream_gemv_matches_oracle(bn, oracle, Ns, K, per_row):
+@pytest.mark.parametrize("Ns,K,per_row,kernel", STREAM_CASES)
+def test_stream_gemv_matches_oracle(bn, oracle, Ns, K, per_row, kernel):
     assert sum(Ns) * K // 4 >= 12 << 20
+    want = bn.KERNEL_GS if kernel == "gs" else bn.KERNEL_STREAM
+    assert bn.bitnet_linear_plan(1, K, list(Ns))["kernel"] == want
     g = synth.rng(0, 99, len(Ns), K, synth.KIND_T)
     x = synth.normal_x(1, K, g)
     projs, refs = [], []

@@ -164,7 +164,7 @@ def test_swiglu_8b_mlp_per_row_sampled(bn, oracle):
 
 
 def test_swiglu_8b_mlp_decode_stream(bn, oracle):
-    """8B-class MLP gate/up at M = 1 (29 MB interleaved, the streaming GEMV), per-row scales,
+    """8B-class MLP gate/up at M = 1 (29 MB interleaved, the grid-stride GEMV), per-row scales,
     every output."""
     Wg = synth.stack8b_latent(0, "gate")
     Wu = synth.stack8b_latent(0, "up")
@@ -177,3 +177,20 @@ def test_swiglu_8b_mlp_decode_stream(bn, oracle):
     torch.cuda.synchronize()
     ref = oracle.swiglu_gate_up(x, pg, sg, pu, su, True, 4096)
     assert_swiglu_within_bound(bits_from_bf16_tensor(h), ref, oracle, where="8B decode")
+
+
+def test_swiglu_one_token_grid_stride_per_tensor(bn, oracle):
+    """One token, 10000 output pairs at K = 2560 (12.8 MB interleaved: the grid-stride GEMV's
+    SwiGLU pairing), per-tensor gate and up scales: within the bound, and bit-equal to the
+    tensor-core path (same arithmetic)."""
+    I, K = 10000, 2560
+    assert bn.bitnet_linear_plan(1, K, [2 * I], swiglu=True)["kernel"] == bn.KERNEL_GS
+    x, tg, tu, sg, su = _mlp(1, I, K, False)
+    pg, pu, packed_gu, s_gu = _device_weights(bn, oracle, tg, tu, sg, su, False)
+    xd = bf16_tensor_from_bits(x)
+    h = bn.bitnet_linear_swiglu(xd, packed_gu, s_gu, False)
+    torch.cuda.synchronize()
+    ref = oracle.swiglu_gate_up(x, pg, sg, pu, su, False, K)
+    assert_swiglu_within_bound(bits_from_bf16_tensor(h), ref, oracle, where="grid-stride SwiGLU")
+    h_tc = bn.bitnet_linear_swiglu(xd, packed_gu, s_gu, False, path=bn.PATH_TC)
+    assert torch.equal(h.view(torch.int16), h_tc.view(torch.int16))
