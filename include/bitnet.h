@@ -268,6 +268,40 @@ bitnet_status bitnet_linear_swiglu(const uint16_t* x, int64_t M, int64_t K,
                                    void* stream);
 
 /*
+ * The SwiGLU -> down projection hand-off (page "BitNet-Triton", section "技术架构：融合内核的
+ * 三重优化", item 3 "融合激活量化": the activation quantiser belongs with the producer of its
+ * input; "BitNet 深度实战" section 3.2, BitLlamaMLP: down(silu(gate(x)) * up(x))).
+ * The down projection quantises h per token, and a token's amax runs over all I outputs of h,
+ * which the gate/up kernel computes in different CTAs. So the gate/up epilogue writes, beside
+ * h, the maxima of |h| over every block of 16 outputs, and the down projection's quantiser
+ * takes each token's amax from those I/16 values instead of reducing the row of h.
+ *
+ * hmax / xmax layout: (M, K/16) uint16, row-major; entry [m, b] holds the bf16 bit pattern,
+ * sign cleared, of max |x[m, 16b .. 16b + 15]|. |x| ordered as an unsigned integer is exact,
+ * so the amax, and therefore q, s_x and y, equal the plain per-token path's bit for bit.
+ *
+ * bitnet_linear_swiglu_hmax — bitnet_linear_swiglu that also writes hmax (M, I/16), 2-byte
+ *   aligned. Always runs the tensor-core path (workspace as bitnet_linear_ex for that path;
+ *   any M); BITNET_ERR_NULL for a null hmax, other errors as bitnet_linear_swiglu.
+ * bitnet_linear_hmax — bitnet_linear on the tensor-core path whose quantiser reads xmax
+ *   (M, K/16, 8-byte aligned) for each token's amax. xmax must be the block maxima of this x:
+ *   the library does not check them, and other values give other scales.
+ * bitnet_quant_act_hmax — bitnet_quant_act with the amax taken from xmax: q (M, K) int8
+ *   natural layout, s_x (M) fp32.
+ */
+bitnet_status bitnet_linear_swiglu_hmax(const uint16_t* x, int64_t M, int64_t K,
+                                        const uint8_t* packed_gu, const float* s_w_gu,
+                                        bitnet_scale_mode mode, int64_t I, uint16_t* h,
+                                        uint16_t* hmax, void* workspace, size_t workspace_bytes,
+                                        void* stream);
+bitnet_status bitnet_linear_hmax(const uint16_t* x, const uint16_t* xmax, int64_t M, int64_t K,
+                                 const uint8_t* packed, const float* s_w, bitnet_scale_mode mode,
+                                 int64_t N, void* y, bitnet_out_dtype out_dtype, void* workspace,
+                                 size_t workspace_bytes, void* stream);
+bitnet_status bitnet_quant_act_hmax(const uint16_t* x, const uint16_t* xmax, int64_t M,
+                                    int64_t K, int8_t* q, float* s_x, void* stream);
+
+/*
  * bitnet_linear_noalloc — bitnet_linear for callers that cannot allocate device memory.
  * The pages have no counterpart to this call; it exists for callers such as a serving
  * loop in which cudaMalloc could synchronise the device and stall other streams, or a

@@ -182,6 +182,21 @@ def quant_act_per_tensor(x_bf16_bits: np.ndarray):
     return q, s
 
 
+def block_absmax_bits(x_bf16_bits: np.ndarray, block: int = 16) -> np.ndarray:
+    """Maxima of |x| over consecutive blocks of ``block`` values along each row, as bf16 bit
+    patterns (M, K / block) uint16: the hand-off from the SwiGLU producer to the down
+    projection's quantiser ("BitNet-Triton", "技术架构：融合内核的三重优化" item 3: the
+    activation quantiser belongs with the producer of its input). |x| of a bf16 pattern is the
+    pattern with the sign bit cleared; for non-NaN values those patterns order as unsigned
+    integers exactly as the magnitudes do, so the block maximum is exact, and the maximum over
+    a row's blocks is the row's amax of ``quant_act``."""
+    x = np.ascontiguousarray(x_bf16_bits, dtype=np.uint16)
+    M, K = x.shape
+    if K % block:
+        raise ValueError(f"K = {K} is not a multiple of the block {block}")
+    return (x & np.uint16(0x7FFF)).reshape(M, K // block, block).max(axis=2).astype(np.uint16)
+
+
 def ternary_matmul(q: np.ndarray, t: np.ndarray) -> np.ndarray:
     """int32 acc[m,n] = sum_k q[m,k] t[n,k] by add / subtract / skip ("BitNet 深度实战", §4.4)."""
     q = np.ascontiguousarray(q, dtype=np.int8)

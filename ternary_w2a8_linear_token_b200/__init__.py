@@ -89,6 +89,11 @@ _SIGS = {
                                   ctypes.c_int),
     "bitnet_linear_swiglu": ([_P, _I64, _I64, _P, _P, ctypes.c_int, _I64, _P, _P, _SZ,
                              ctypes.c_int, _P], ctypes.c_int),
+    "bitnet_linear_swiglu_hmax": ([_P, _I64, _I64, _P, _P, ctypes.c_int, _I64, _P, _P, _P, _SZ,
+                                   _P], ctypes.c_int),
+    "bitnet_linear_hmax": ([_P, _P, _I64, _I64, _P, _P, ctypes.c_int, _I64, _P, ctypes.c_int, _P,
+                            _SZ, _P], ctypes.c_int),
+    "bitnet_quant_act_hmax": ([_P, _P, _I64, _I64, _P, _P, _P], ctypes.c_int),
     "bitnet_b3_row_bytes": ([_I64], _I64),
     "bitnet_pack_ternary_b3": ([_P, _I64, _I64, _P, _P], ctypes.c_int),
     "bitnet_linear_b3": ([_P, _I64, _I64, _P, _P, ctypes.c_int, _I64, _P, ctypes.c_int, _P],
@@ -363,6 +368,75 @@ def bitnet_linear_swiglu(x: torch.Tensor, packed_gu: torch.Tensor, s_w_gu: torch
                                     _dev(h, torch.bfloat16, "h"), wp, wb, path, _stream(stream)),
            "bitnet_linear_swiglu")
     return h
+
+
+def _check_xmax(xmax: torch.Tensor, M: int, K: int):
+    if tuple(xmax.shape) != (M, K // SWIGLU_BLOCK) or not xmax.is_contiguous():
+        raise ValueError(f"xmax must be contiguous ({M}, {K // SWIGLU_BLOCK}), got "
+                         f"{tuple(xmax.shape)}")
+    return _dev(xmax, torch.int16, "xmax")
+
+
+def bitnet_linear_swiglu_hmax(x: torch.Tensor, packed_gu: torch.Tensor, s_w_gu: torch.Tensor,
+                              per_row: bool, h: Optional[torch.Tensor] = None,
+                              hmax: Optional[torch.Tensor] = None,
+                              workspace: Optional[torch.Tensor] = None, stream=None):
+    """bitnet_linear_swiglu on the tensor-core path that also returns hmax (M, I/16) int16:
+    the bf16 bits of max |h| over each block of 16 outputs, for bitnet_linear_hmax."""
+    M, K = x.shape
+    if packed_gu.dim() != 2 or packed_gu.shape[1] * 4 != K or packed_gu.shape[0] % 2:
+        raise ValueError(f"packed_gu must be (2I, K/4) = (2I, {K // 4}), got "
+                         f"{tuple(packed_gu.shape)}")
+    I = packed_gu.shape[0] // 2
+    want = 2 * I if per_row else 2
+    if s_w_gu.numel() != want:
+        raise ValueError(f"s_w_gu must have {want} elements, got {s_w_gu.numel()}")
+    if h is None:
+        h = torch.empty((M, I), dtype=torch.bfloat16, device=x.device)
+    if hmax is None:
+        hmax = torch.empty((M, I // SWIGLU_BLOCK), dtype=torch.int16, device=x.device)
+    if tuple(h.shape) != (M, I):
+        raise ValueError(f"h must be ({M}, {I}), got {tuple(h.shape)}")
+    hm = _check_xmax(hmax, M, I)
+    wp, wb, _keep = _ws_args(workspace, M, K, PATH_TC, x.device)
+    _check(lib.bitnet_linear_swiglu_hmax(_x_ptr(x), M, K, _dev(packed_gu, torch.uint8, "packed_gu"),
+                                         _dev(s_w_gu, torch.float32, "s_w_gu"),
+                                         int(bool(per_row)), I, _dev(h, torch.bfloat16, "h"),
+                                         hm, wp, wb, _stream(stream)),
+           "bitnet_linear_swiglu_hmax")
+    return h, hmax
+
+
+def bitnet_linear_hmax(x: torch.Tensor, xmax: torch.Tensor, packed: torch.Tensor,
+                       s_w: torch.Tensor, per_row: bool, out_dtype: torch.dtype = torch.bfloat16,
+                       y: Optional[torch.Tensor] = None,
+                       workspace: Optional[torch.Tensor] = None, stream=None):
+    """bitnet_linear on the tensor-core path with each token's amax taken from xmax, the
+    (M, K/16) block maxima of |x| (as bitnet_linear_swiglu_hmax returns them for h)."""
+    M, K = x.shape
+    N = _check_proj(packed, s_w, per_row, K)
+    xm = _check_xmax(xmax, M, K)
+    if y is None:
+        y = torch.empty((M, N), dtype=out_dtype, device=x.device)
+    _check_out(y, M, N)
+    od = OUT_BF16 if y.dtype == torch.bfloat16 else OUT_F32
+    wp, wb, _keep = _ws_args(workspace, M, K, PATH_TC, x.device)
+    _check(lib.bitnet_linear_hmax(_x_ptr(x), xm, M, K, _dev(packed, torch.uint8, "packed"),
+                                  _dev(s_w, torch.float32, "s_w"), int(bool(per_row)), N,
+                                  _dev(y, y.dtype, "y"), od, wp, wb, _stream(stream)),
+           "bitnet_linear_hmax")
+    return y
+
+
+def bitnet_quant_act_hmax(x: torch.Tensor, xmax: torch.Tensor, stream=None):
+    """bitnet_quant_act with each token's amax taken from xmax (M, K/16)."""
+    M, K = x.shape
+    xm = _check_xmax(xmax, M, K)
+    q = torch.empty((M, K), dtype=torch.int8, device=x.device)
+    s_x = torch.empty(M, dtype=torch.float32, device=x.device)
+    _check(lib.bitnet_quant_act_hmax(_x_ptr(x), xm, M, K, q.data_ptr(), s_x.data_ptr(),
+                                     _stream(stream)), "bitnet_quant_act_hmax")
+    return q, s_x
 
 
 NOALLOC_SCRATCH_BYTES = 16 * 1024 * 1024

@@ -216,14 +216,18 @@ bitnet_status plan_batch(const uint16_t* x_bf16, const int8_t* q_in, int64_t M, 
 
 // Runs a validated batch. x_bf16 or q_in (int8, contraction-only) is the input. swiglu: the
 // batch is one interleaved gate/up matrix of N = 2I rows whose output is h (M, I) bf16.
+// Tensor-core path only: xmax, the (M, K/16) block maxima of |x| that the quantiser reduces
+// instead of x's rows; hmax, the (M, I/16) block maxima of |h| the SwiGLU epilogue writes.
 bitnet_status run_batch(const uint16_t* x_bf16, const int8_t* q_in, int64_t M, int64_t K,
                         const Batch& b, int out_kind, void* workspace, size_t workspace_bytes,
                         bitnet_path path, cudaStream_t stream, bool swiglu = false,
-                        bool act_per_tensor = false) {
+                        bool act_per_tensor = false, const uint16_t* xmax = nullptr,
+                        uint16_t* hmax = nullptr) {
     Plan pl;
     bitnet_status pst = plan_batch(x_bf16, q_in, M, K, b, out_kind, workspace, workspace_bytes,
                                    path, swiglu, act_per_tensor, &pl);
     if (pst != BITNET_OK) return pst;
+    if (pl.kernel != BITNET_KERNEL_TC && (xmax || hmax)) return BITNET_ERR_UNSUPPORTED;
     if (pl.kernel == BITNET_KERNEL_GS)
         return from_cuda(launch_gemv_gs(pl.gp, /*b3=*/false, tc_num_sms(), stream, /*pdl=*/true));
     if (pl.kernel == BITNET_KERNEL_STREAM) {
@@ -286,6 +290,7 @@ bitnet_status run_batch(const uint16_t* x_bf16, const int8_t* q_in, int64_t M, i
             return BITNET_ERR_CUDA;
         p.proj[0].tma_store = 1;
         p.swiglu = 1;
+        p.hmax = hmax;
     }
     for (int i = 0; i < b.nproj && !swiglu; ++i) {
         const uint64_t N = uint64_t(b.proj[i].N);
@@ -326,7 +331,7 @@ bitnet_status run_batch(const uint16_t* x_bf16, const int8_t* q_in, int64_t M, i
     cudaError_t e = launch_quant(x_bf16, q_in, M, K, q_ws, q_in ? nullptr : s_x,
                                  q_in ? nullptr : r_x, /*permuted=*/1, stream, /*pdl=*/true, zero,
                                  zero_bytes, qsum, per_tensor ? amax_parts : nullptr,
-                                 per_tensor ? amax_parts_count(M, K) : 0);
+                                 per_tensor ? amax_parts_count(M, K) : 0, xmax);
     if (e != cudaSuccess) return BITNET_ERR_CUDA;
     return from_cuda(launch_tc_gemm(p, bn, stream, /*pdl=*/true));
 }
@@ -583,6 +588,63 @@ bitnet_status bitnet_linear_swiglu(const uint16_t* x, int64_t M, int64_t K,
     if ((st = validate_batch(x, M, K, &pr, 1, /*out_kind=*/0, &b)) != BITNET_OK) return st;
     return run_batch(x, nullptr, M, K, b, 0, workspace, workspace_bytes, path,
                      static_cast<cudaStream_t>(stream), /*swiglu=*/true);
+}
+
+bitnet_status bitnet_linear_swiglu_hmax(const uint16_t* x, int64_t M, int64_t K,
+                                        const uint8_t* packed_gu, const float* s_w_gu,
+                                        bitnet_scale_mode mode, int64_t I, uint16_t* h,
+                                        uint16_t* hmax, void* workspace, size_t workspace_bytes,
+                                        void* stream) {
+    if (!h || !hmax) return BITNET_ERR_NULL;
+    bitnet_status st = check_n(I);
+    if (st != BITNET_OK) return st;
+    if (I % kSwigluBlock != 0 || 2 * I >= (int64_t(1) << 31)) return BITNET_ERR_SHAPE;
+    if (!aligned(hmax, 2)) return BITNET_ERR_ALIGN;
+    bitnet_proj pr;
+    pr.packed = packed_gu;
+    pr.s_w = s_w_gu;
+    pr.mode = int32_t(mode);
+    pr.reserved = 0;
+    pr.N = 2 * I;
+    pr.y = h;
+    Batch b;
+    if ((st = validate_batch(x, M, K, &pr, 1, /*out_kind=*/0, &b)) != BITNET_OK) return st;
+    return run_batch(x, nullptr, M, K, b, 0, workspace, workspace_bytes, BITNET_PATH_TC,
+                     static_cast<cudaStream_t>(stream), /*swiglu=*/true, false, nullptr, hmax);
+}
+
+bitnet_status bitnet_linear_hmax(const uint16_t* x, const uint16_t* xmax, int64_t M, int64_t K,
+                                 const uint8_t* packed, const float* s_w, bitnet_scale_mode mode,
+                                 int64_t N, void* y, bitnet_out_dtype out_dtype, void* workspace,
+                                 size_t workspace_bytes, void* stream) {
+    if (out_dtype != BITNET_OUT_BF16 && out_dtype != BITNET_OUT_F32) return BITNET_ERR_UNSUPPORTED;
+    if (!xmax) return BITNET_ERR_NULL;
+    if (!aligned(xmax, 8)) return BITNET_ERR_ALIGN;
+    bitnet_proj pr;
+    pr.packed = packed;
+    pr.s_w = s_w;
+    pr.mode = int32_t(mode);
+    pr.reserved = 0;
+    pr.N = N;
+    pr.y = y;
+    Batch b;
+    bitnet_status st = validate_batch(x, M, K, &pr, 1, int(out_dtype), &b);
+    if (st != BITNET_OK) return st;
+    return run_batch(x, nullptr, M, K, b, int(out_dtype), workspace, workspace_bytes,
+                     BITNET_PATH_TC, static_cast<cudaStream_t>(stream), /*swiglu=*/false, false,
+                     xmax, nullptr);
+}
+
+bitnet_status bitnet_quant_act_hmax(const uint16_t* x, const uint16_t* xmax, int64_t M,
+                                    int64_t K, int8_t* q, float* s_x, void* stream) {
+    if (!x || !xmax || !q || !s_x) return BITNET_ERR_NULL;
+    bitnet_status st = check_mk(M, K);
+    if (st != BITNET_OK) return st;
+    if (!aligned(x, 16) || !aligned(xmax, 8) || !aligned(q, 16) || !aligned(s_x, 4))
+        return BITNET_ERR_ALIGN;
+    return from_cuda(launch_quant(x, nullptr, M, K, q, s_x, nullptr, /*permuted=*/0,
+                                  static_cast<cudaStream_t>(stream), /*pdl=*/false, nullptr, 0,
+                                  nullptr, nullptr, 0, xmax));
 }
 
 int64_t bitnet_b3_row_bytes(int64_t K) { return K < 1 ? 0 : b3_row_bytes(K); }

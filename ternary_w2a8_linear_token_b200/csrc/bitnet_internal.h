@@ -109,10 +109,13 @@ cudaError_t launch_gemv_stream(const GemvParams& p, int64_t n_stages, int depth,
 // over its CTAs (the split-K area of the GEMM that follows), or null.
 // amax_parts / n_parts: when set, every token uses the one scale of the whole input, whose
 // amax is the maximum of these partial maxima (written by launch_amax_parts).
+// tok_parts: when set, token m's amax is the maximum of tok_parts[m * K/16 .. + K/16), the
+// maxima of |x| over its blocks of 16 values (bf16 bits) written by x's producer.
 cudaError_t launch_quant(const uint16_t* x, const int8_t* q_in, int64_t M, int64_t K, int8_t* q,
                          float* s_x, float* r_x, int permuted, cudaStream_t stream, bool pdl,
                          void* zero = nullptr, int64_t zero_bytes = 0, int32_t* qsum = nullptr,
-                         const uint32_t* amax_parts = nullptr, int n_parts = 0);
+                         const uint32_t* amax_parts = nullptr, int n_parts = 0,
+                         const uint16_t* tok_parts = nullptr);
 // Partial maxima of |x| over all of x (M, K) into parts[0 .. amax_parts_count(M, K)).
 int amax_parts_count(int64_t M, int64_t K);
 cudaError_t launch_amax_parts(const uint16_t* x, int64_t M, int64_t K, uint32_t* parts,
@@ -173,6 +176,7 @@ struct alignas(64) TcParams {
     int32_t* split_acc;   // split-K: int32 accumulation tile per tile, [tile][token][row]
     int32_t splits;       // K splits per tile (1 = none)
     int32_t swiglu;       // 1: interleaved gate/up rows, outputs h = SwiGLU (bf16, M x N/2)
+    uint16_t* hmax;       // SwiGLU: when set, (M, N/32) maxima of |h| over blocks of 16 outputs
     int64_t K;
     int32_t M;
     int32_t nproj;

@@ -8,7 +8,9 @@
 // 4096 < K <= 14336 take four warps each, also in registers; longer rows take one warp and
 // two passes (the second an L1/L2 hit). With a per-tensor scale ("BitNet 1-bit LLM推理优化"
 // section 2.2, I2_S), amax_parts_kernel first writes partial maxima of the whole input and
-// every warp reduces those instead of its row. Two output layouts:
+// every warp reduces those instead of its row; with block maxima from x's producer (the
+// SwiGLU epilogue's maxima of |h| over 16 outputs), every warp reduces its token's I/16
+// maxima instead. Two output layouts:
 //  - natural (M, K) int8, the public bitnet_quant_act result;
 //  - permuted, the operand layout of the tensor-core path: inside every group of 16
 //    values along K, byte 4i + b holds k = 4b + i. That is the order in which a packed
@@ -35,6 +37,22 @@ __device__ __forceinline__ uint32_t parts_max(const uint32_t* __restrict__ parts
     return __reduce_max_sync(0xFFFFFFFFu, m);
 }
 
+// A token's amax from the maxima of its K / 16 blocks of 16 values (bf16 magnitude bits), as
+// the SwiGLU epilogue writes them for its output h (whole warp). K % 64 == 0, so a token's
+// K / 16 values start on an 8-byte boundary and are read four at a time.
+__device__ __forceinline__ uint32_t tok_parts_max(const uint16_t* __restrict__ parts, int64_t K,
+                                                  int lane) {
+    const uint2* p = reinterpret_cast<const uint2*>(parts);
+    const int64_t n = K / 64;
+    uint32_t m = 0;  // two 16-bit maxima
+#pragma unroll 4
+    for (int64_t i = lane; i < n; i += 32) {
+        const uint2 w = p[i];
+        m = __vmaxu2(m, __vmaxu2(w.x, w.y));
+    }
+    return __reduce_max_sync(0xFFFFFFFFu, max(m & 0xFFFFu, m >> 16));
+}
+
 // One warp per token row; each lane keeps 8 loads in flight. Pass 1 finds amax, pass 2
 // re-reads the row (an L1/L2 hit) and writes q.
 constexpr int kRowsPerCta = kThreads / 32;
@@ -52,7 +70,7 @@ __global__ void __launch_bounds__(kThreads) quant_rows_kernel(const uint16_t* __
                                                               int64_t zero_words,
                                                               int32_t* __restrict__ qsum,
                                                               const uint32_t* __restrict__ amax_parts,
-                                                              int n_parts) {
+                                                              int n_parts, const uint16_t* __restrict__ tok_parts) {
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const int64_t m = int64_t(blockIdx.x) * kRowsPerCta + warp;
@@ -80,8 +98,14 @@ __global__ void __launch_bounds__(kThreads) quant_rows_kernel(const uint16_t* __
         uint32_t mx = 0;
 #pragma unroll
         for (int u = 0; u < kRegPieces; ++u) mx = max(mx, absmax8_bits(v[u]));
-        mx = __reduce_max_sync(0xFFFFFFFFu, mx);
-        if (amax_parts) mx = parts_max(amax_parts, n_parts, lane);  // one scale per tensor
+        // The token's amax: its row's, the whole input's (per-tensor parts) or the maximum of
+        // the block maxima that x's producer wrote.
+        if (tok_parts)
+            mx = tok_parts_max(tok_parts + m * (K / 16), K, lane);
+        else if (amax_parts)
+            mx = parts_max(amax_parts, n_parts, lane);
+        else
+            mx = __reduce_max_sync(0xFFFFFFFFu, mx);
         s = __fdiv_rn(127.0f, fmaxf(bf16_lo(mx), kEps));
         if (lane == 0) {
             if (s_x) s_x[m] = s;
@@ -115,8 +139,12 @@ __global__ void __launch_bounds__(kThreads) quant_rows_kernel(const uint16_t* __
 #pragma unroll
             for (int u = 0; u < kUnroll; ++u) mx = max(mx, absmax8_bits(v[u]));
         }
-        mx = __reduce_max_sync(0xFFFFFFFFu, mx);
-        if (amax_parts) mx = parts_max(amax_parts, n_parts, lane);  // one scale per tensor
+        if (tok_parts)
+            mx = tok_parts_max(tok_parts + m * (K / 16), K, lane);
+        else if (amax_parts)
+            mx = parts_max(amax_parts, n_parts, lane);
+        else
+            mx = __reduce_max_sync(0xFFFFFFFFu, mx);
         s = __fdiv_rn(127.0f, fmaxf(bf16_lo(mx), kEps));
         if (lane == 0) {
             if (s_x) s_x[m] = s;
@@ -170,7 +198,7 @@ __global__ void __launch_bounds__(kLongThreads) quant_long_rows_kernel(
     const uint16_t* __restrict__ x, int64_t M, int64_t K, int8_t* __restrict__ q,
     float* __restrict__ s_x, float* __restrict__ r_x, int permuted, uint4* __restrict__ zero,
     int64_t zero_words, int32_t* __restrict__ qsum, const uint32_t* __restrict__ amax_parts,
-    int n_parts) {
+    int n_parts, const uint16_t* __restrict__ tok_parts) {
     __shared__ uint32_t s_mx[kLongRows][kLongRowThreads / 32];
     __shared__ int32_t s_qs[kLongRows][kLongRowThreads / 32];
     const int row = threadIdx.x / kLongRowThreads;
@@ -193,16 +221,21 @@ __global__ void __launch_bounds__(kLongThreads) quant_long_rows_kernel(
         const int64_t c = int64_t(u) * kLongRowThreads + t;
         v[u] = (active && c < pieces) ? xr[c] : make_uint4(0u, 0u, 0u, 0u);
     }
-    uint32_t mx = 0;
-#pragma unroll
-    for (int u = 0; u < kLongPieces; ++u) mx = max(mx, absmax8_bits(v[u]));
-    mx = __reduce_max_sync(0xFFFFFFFFu, mx);
-    if (lane == 0) s_mx[row][t >> 5] = mx;
-    __syncthreads();
     uint32_t all = 0;
+    if (tok_parts) {
+        // the block maxima written by x's producer: no reduction across the row's warps
+        all = tok_parts_max(tok_parts + (active ? m : 0) * (K / 16), K, lane);
+    } else {
+        uint32_t mx = 0;
 #pragma unroll
-    for (int w = 0; w < kLongRowThreads / 32; ++w) all = max(all, s_mx[row][w]);
-    if (amax_parts) all = parts_max(amax_parts, n_parts, lane);  // one scale per tensor
+        for (int u = 0; u < kLongPieces; ++u) mx = max(mx, absmax8_bits(v[u]));
+        mx = __reduce_max_sync(0xFFFFFFFFu, mx);
+        if (lane == 0) s_mx[row][t >> 5] = mx;
+        __syncthreads();
+#pragma unroll
+        for (int w = 0; w < kLongRowThreads / 32; ++w) all = max(all, s_mx[row][w]);
+        if (amax_parts) all = parts_max(amax_parts, n_parts, lane);  // one scale per tensor
+    }
     const float s = __fdiv_rn(127.0f, fmaxf(bf16_lo(all), kEps));
     if (active && t == 0) {
         if (s_x) s_x[m] = s;
@@ -296,7 +329,7 @@ cudaError_t launch_amax_parts(const uint16_t* x, int64_t M, int64_t K, uint32_t*
 cudaError_t launch_quant(const uint16_t* x, const int8_t* q_in, int64_t M, int64_t K, int8_t* q,
                          float* s_x, float* r_x, int permuted, cudaStream_t stream, bool pdl,
                          void* zero, int64_t zero_bytes, int32_t* qsum,
-                         const uint32_t* amax_parts, int n_parts) {
+                         const uint32_t* amax_parts, int n_parts, const uint16_t* __restrict__ tok_parts) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>((M + kRowsPerCta - 1) / kRowsPerCta));
     cfg.blockDim = dim3(kThreads);
@@ -312,11 +345,11 @@ cudaError_t launch_quant(const uint16_t* x, const int8_t* q_in, int64_t M, int64
         cfg.blockDim = dim3(kLongThreads);
         return cudaLaunchKernelEx(&cfg, quant_long_rows_kernel, x, M, K, q, s_x, r_x, permuted,
                                   static_cast<uint4*>(zero), zero_bytes / 16, qsum, amax_parts,
-                                  n_parts);
+                                  n_parts, tok_parts);
     }
     return cudaLaunchKernelEx(&cfg, quant_rows_kernel, x, q_in, M, K, q, s_x, r_x, permuted,
                               static_cast<uint4*>(zero), zero_bytes / 16, qsum, amax_parts,
-                              n_parts);
+                              n_parts, tok_parts);
 }
 
 }  // namespace bitnet

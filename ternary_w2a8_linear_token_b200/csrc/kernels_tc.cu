@@ -224,6 +224,37 @@ __device__ __forceinline__ void stage_cols(int out_kind, uint8_t* buf, int lane,
     }
 }
 
+// Column maxima over a half warp: lanes 16h .. 16h + 15 each hold N values (one per column)
+// of 16-bit magnitudes (bf16 bits, sign cleared here). Each exchange step halves the columns a
+// lane keeps, swapping the other half with its partner, until one column is left; the
+// remaining steps reduce it. On return v[0] holds the maximum of column c over the 16 lanes
+// (the returned c); lanes that differ only in their low 4 - log2(N) bits hold the same column.
+template <int N>
+__device__ __forceinline__ int half_warp_column_max(uint32_t* v, int lane) {
+    static_assert(N >= 1 && N <= 16 && (N & (N - 1)) == 0, "N is a power of two up to 16");
+#pragma unroll
+    for (int c = 0; c < N; ++c) v[c] &= 0x7FFFu;
+    int col = 0;
+#pragma unroll
+    for (int step = 0; step < 4; ++step) {
+        const int o = 8 >> step;
+        const int n = N >> step;  // columns still held
+        if (n > 1) {
+            const bool upper = (lane & o) != 0;
+#pragma unroll
+            for (int i = 0; i < n / 2; ++i) {
+                const uint32_t send = upper ? v[i] : v[i + n / 2];
+                const uint32_t keep = upper ? v[i + n / 2] : v[i];
+                v[i] = max(keep, __shfl_xor_sync(0xFFFFFFFFu, send, o));
+            }
+            if (upper) col += n / 2;
+        } else {
+            v[0] = max(v[0], __shfl_xor_sync(0xFFFFFFFFu, v[0], o));
+        }
+    }
+    return col;
+}
+
 // Dequantisation factors of kHC consecutive tokens from the tile's shared table (a
 // broadcast read: every lane reads the same addresses). The table holds s_w * (1/s_x) for
 // a per-tensor scale and 1/s_x for per-row scales, where this lane's row scale sw is
@@ -641,6 +672,14 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
                             bulk_commit_group();
                         }
                         ++staged_stores;
+                        if (p.hmax && x < (pr.N >> 1)) {  // warp-uniform
+                            // Maxima of |h| over this warp's 16 outputs, per token: half-warp
+                            // column maxima, stored as bf16 bits at hmax[token][x / 16].
+                            const int c = half_warp_column_max<kHalf>(v, lane);
+                            const int64_t m = int64_t(y) + c + (gate_lane ? 0 : kHalf);
+                            if ((lane & (kSwigluBlock / kHalf - 1)) == 0 && m < p.M)
+                                p.hmax[m * (pr.N >> 5) + (x >> 4)] = uint16_t(v[0]);
+                        }
                     } else if (staged) {
                         // 2-byte outputs alternate between the two 1 KB halves of the staging
                         // tile; 4-byte outputs use all 2 KB, so the previous store must have

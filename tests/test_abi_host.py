@@ -273,3 +273,35 @@ def test_b3_calls_argument_errors(bn):
     assert call(p=None) == bn.ERR_NULL
     assert call(mode=3) == bn.ERR_UNSUPPORTED and call(od=5) == bn.ERR_UNSUPPORTED
     assert call(y=F + 2) == bn.ERR_ALIGN
+
+
+def test_hand_off_calls_argument_errors(bn):
+    """bitnet_linear_swiglu_hmax, bitnet_linear_hmax and bitnet_quant_act_hmax check pointers,
+    shapes and alignment before touching the device, and always need the tensor-core
+    workspace (any M)."""
+    lib, F = bn.lib, FAKE
+
+    def sw(x=F, M=4, K=512, pgu=F, s=F, mode=0, I=64, h=F, hm=F, ws=None, wb=0):
+        return lib.bitnet_linear_swiglu_hmax(x, M, K, pgu, s, mode, I, h, hm, ws, wb, None)
+
+    assert sw(hm=None) == bn.ERR_NULL and sw(h=None) == bn.ERR_NULL and sw(x=None) == bn.ERR_NULL
+    assert sw(I=24) == bn.ERR_SHAPE and sw(M=0) == bn.ERR_SHAPE
+    assert sw(K=96) == bn.ERR_UNSUPPORTED and sw(mode=4) == bn.ERR_UNSUPPORTED
+    assert sw(hm=F + 1) == bn.ERR_ALIGN and sw(h=F + 2) == bn.ERR_ALIGN
+    assert sw(M=1) == bn.ERR_WORKSPACE and sw(M=300, ws=F, wb=16) == bn.ERR_WORKSPACE
+
+    def lin(x=F, xm=F, M=4, K=512, p=F, s=F, mode=0, N=64, y=F, od=0, ws=None, wb=0):
+        return lib.bitnet_linear_hmax(x, xm, M, K, p, s, mode, N, y, od, ws, wb, None)
+
+    assert lin(xm=None) == bn.ERR_NULL and lin(p=None) == bn.ERR_NULL
+    assert lin(M=0) == bn.ERR_SHAPE and lin(K=96) == bn.ERR_UNSUPPORTED
+    assert lin(od=3) == bn.ERR_UNSUPPORTED and lin(mode=2) == bn.ERR_UNSUPPORTED
+    assert lin(xm=F + 4) == bn.ERR_ALIGN and lin(x=F + 2) == bn.ERR_ALIGN
+    assert lin(M=2) == bn.ERR_WORKSPACE
+
+    def qa(x=F, xm=F, M=2, K=512, q=F, s=F):
+        return lib.bitnet_quant_act_hmax(x, xm, M, K, q, s, None)
+
+    assert qa(xm=None) == bn.ERR_NULL and qa(q=None) == bn.ERR_NULL
+    assert qa(M=0) == bn.ERR_SHAPE and qa(K=96) == bn.ERR_UNSUPPORTED
+    assert qa(xm=F + 2) == bn.ERR_ALIGN and qa(q=F + 8) == bn.ERR_ALIGN

@@ -586,3 +586,40 @@ def test_unpack_b3_rejects_bad_bytes_and_padding(oracle):
         oracle.unpack_b3(pad, 64)
     with pytest.raises(oracle.OracleError):
         oracle.pack_b3(np.full((1, 64), 2, dtype=np.int8))
+
+
+# ---------------------------------------------------------------- SwiGLU -> down hand-off
+
+def test_block_absmax_hand_example(oracle):
+    """Two blocks of 16: block 0 holds -3.0 (bf16 0xC040 -> |x| = 0x4040), block 1 holds
+    0.5 as its largest magnitude next to -0.25 (0x3F00); sign and position do not matter."""
+    xs = np.zeros((2, 32), dtype=np.float32)
+    xs[0, 3], xs[0, 15], xs[0, 20], xs[0, 31] = 1.0, -3.0, 0.5, -0.25
+    xs[1, 16] = -0.0
+    xs[1, 0] = 2.0 ** -130  # a subnormal bf16 still orders as its magnitude
+    got = oracle.block_absmax_bits(synth.to_bf16_bits(xs))
+    assert got.dtype == np.uint16 and got.shape == (2, 2)
+    assert got[0].tolist() == [0x4040, 0x3F00]
+    assert got[1].tolist() == [int(synth.to_bf16_bits(np.array([2.0 ** -130], np.float32))[0]), 0]
+
+
+def test_block_absmax_brute_force_and_quant_scale(oracle):
+    """Against a float loop over every block, and the maximum over a row's blocks gives the
+    scale oracle.quant_act computes from the row (the quantiser's amax, reached two ways)."""
+    g = np.random.default_rng(11)
+    M, K = 5, 96
+    x = synth.to_bf16_bits(g.standard_normal((M, K)).astype(np.float32)
+                           * g.uniform(1e-3, 40, size=(M, 1)).astype(np.float32))
+    x[2] = 0
+    got = oracle.block_absmax_bits(x)
+    xf = synth.bf16_bits_to_f32(x)
+    for m in range(M):
+        for b in range(K // 16):
+            want = max(abs(float(v)) for v in xf[m, 16 * b:16 * b + 16])
+            assert float(synth.bf16_bits_to_f32(got[m:m + 1, b:b + 1])[0, 0]) == want
+    amax = synth.bf16_bits_to_f32(got.max(axis=1, keepdims=True))[:, 0]
+    s_from_blocks = np.float32(127.0) / np.maximum(amax, np.float32(1e-5))
+    _, s = oracle.quant_act(x)
+    assert np.array_equal(s_from_blocks.astype(np.float32), s)
+    with pytest.raises(ValueError):
+        oracle.block_absmax_bits(x[:, :40])
