@@ -48,6 +48,11 @@ INT8_PER_BF16 = 2.0
 # shapes (2560 x 2560, 640 x 2560, 6912 x 2560, 2560 x 6912 at M = 1: 1662976, 430336,
 # 4447744, 4455168 bytes), averaged; the kernel has not changed since.
 GEMV_DECODE_TRAFFIC_BYTES = 2749056
+# DRAM bytes per prefill GEMM launch (tc_gemm_kernel, M = 2048), read + write, from one ncu
+# capture of the four shapes (6979328, 5748736, 9764352, 18681344 bytes), averaged. The bf16
+# outputs stay in L2 while the kernel runs (written back after it ends), so this is below the
+# algorithmic bytes: packed weights + int8 tokens + outputs.
+GEMM_PREFILL_TRAFFIC_BYTES = 10293440
 
 
 def decode_bytes(M, N, K):
@@ -586,7 +591,14 @@ def run_ours(args):
                             "with 1% x20 outlier channels, ternary P(0)=0.5",
                 "roofline": {"bound": "tensor", "achieved": local_tops, "peak": int8_peak,
                              "unit": "TOPS", "frac": local_tops / int8_peak,
-                             "traffic": None,
+                             "traffic": GEMM_PREFILL_TRAFFIC_BYTES
+                             if args.prefill_m == PREFILL_M else None,
+                             "traffic_src": "ncu dram__bytes_read.sum + dram__bytes_write.sum "
+                                            "per tc_gemm_kernel launch at M=2048, one capture "
+                                            "of the four shapes, mean",
+                             "algorithmic_bytes_per_launch": sum(
+                                 c["N"] * c["K"] // 4 + args.prefill_m * c["K"]
+                                 + 2 * args.prefill_m * c["N"] for c in pcalls) / len(pcalls),
                              "peak_src": peaks["int8_src"],
                              "frac_vs_measured_int8": (local_tops / int8_probe["burst_tops"]
                                                        if int8_probe.get("burst_tops") else None),
