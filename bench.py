@@ -694,6 +694,7 @@ def run_ours(args):
             "e2e": {"value": e2e_gbs, "unit": "GB/s",
                     "h2d_bytes_per_step": int(h_x.numel() * 2),
                     "d2h_bytes_per_step": int(h_y.numel() * 2)},
+            "cpu_baseline": cpu,
             "gpu_launches": args.steps * launches_per_step * 2 + args.steps * 7 * len(pcalls)
                             + stack_launches,
             "clocks": clk.summary(),
@@ -706,7 +707,6 @@ def run_ours(args):
             "gemm": gemm,
             "stacks": stacks,
             "mlp": mlp,
-            "cpu_baseline": cpu,
         }
         print(json.dumps(line), flush=True)
     del g_dec, g_e2e, g_pre
