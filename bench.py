@@ -497,6 +497,34 @@ def measure_int8_peak(torch, dev, seconds: float = 1.5):
                    f"for {seconds} s"}
 
 
+def measure_int_rates(bn, torch, dev):
+    """Issue rates of the one-token GEMV's product instructions on this GPU (the library's
+    probe kernels: dp4a only, legacy mma.sync m16n8k32 s8 only), 8 CTAs of 256 threads per
+    SM, ~10 ms per launch, best of 3; int8 ops = 2 per multiply-add."""
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    blocks = sms * 8
+    out = torch.empty(blocks, dtype=torch.int32, device=dev)
+    st = torch.cuda.current_stream().cuda_stream
+    res = {"how": f"bitnet_probe_int_rate, {blocks} CTAs x 256 threads, best of 3"}
+    for name, kind, iters in (("dp4a", 0, 1 << 16), ("mma_sync_s8", 1, 1 << 15)):
+        if bn.lib.bitnet_probe_int_rate(kind, blocks, 64, out.data_ptr(), st) != bn.OK:
+            return {"error": f"probe {name} failed to launch"}
+        best = float("inf")
+        for _ in range(3):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            bn.lib.bitnet_probe_int_rate(kind, blocks, iters, out.data_ptr(), st)
+            e1.record()
+            torch.cuda.synchronize()
+            best = min(best, e0.elapsed_time(e1) * 1e-3)
+        ops = bn.lib.bitnet_probe_int_ops(kind, blocks, iters)
+        per_instr = 8 * 32 if kind == 0 else 2 * 16 * 8 * 32  # ops per warp instruction
+        res[f"{name}_tops"] = ops / best / 1e12
+        res[f"{name}_warp_instr_per_sm_per_ns"] = ops / per_instr / best / sms / 1e9
+    assert bn.bitnet_check_device_errors() == 0
+    return res
+
+
 # ---------------------------------------------------------------------------- main arm
 def run_ours(args):
     import torch
@@ -515,6 +543,7 @@ def run_ours(args):
     # The GEMM's denominator: the larger of the measured int8 rate (cuBLASLt through
     # torch._int_mm) and the nominal int8 : bf16 ratio times the measured bf16 peak.
     int8_probe = measure_int8_peak(torch, dev) if args.only == "all" else {}
+    int_rates = measure_int_rates(bn, torch, dev) if args.only == "all" else None
     nominal = peaks["bf16_tflops"] * INT8_PER_BF16
     measured = int8_probe.get("burst_tops", 0.0)
     peaks["int8_tops"] = max(measured, nominal)
@@ -704,6 +733,7 @@ def run_ours(args):
             if gemm and f"m{PREFILL_M_SMALL}" in gemm else None,
             "int8_peak": dict(int8_probe, used_tops=peaks["int8_tops"], used_src=peaks["int8_src"])
             if int8_probe else None,
+            "int_rates": int_rates,
             "gemm": gemm,
             "stacks": stacks,
             "mlp": mlp,

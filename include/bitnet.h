@@ -431,6 +431,23 @@ bitnet_status bitnet_check_device_errors(int32_t* flags);
  */
 bitnet_status bitnet_selftest_wait_timeout(int64_t limit_ns, void* stream);
 
+/*
+ * Arithmetic rate probes for the roofline of the one-token GEMV (diagnostics; the pages have
+ * no counterpart). bitnet_probe_int_rate launches `blocks` CTAs of 256 threads that issue only
+ * dp4a (BITNET_PROBE_DP4A: eight independent chains per thread) or only warp-level
+ * mma.sync m16n8k32 s8 x s8 -> s32 (BITNET_PROBE_MMA_S8: four independent accumulator tiles
+ * per warp), `iters` rounds each; out receives one int32 per CTA (blocks elements, device).
+ * Asynchronous on `stream`: the caller times the launch (CUDA events) and divides
+ * bitnet_probe_int_ops(kind, blocks, iters) integer operations (2 per multiply-add) by it.
+ * Errors: BITNET_ERR_UNSUPPORTED for another kind, BITNET_ERR_SHAPE for blocks outside
+ * [1, 65535] or iters outside [1, 2^24], BITNET_ERR_NULL for a null out.
+ */
+#define BITNET_PROBE_DP4A 0
+#define BITNET_PROBE_MMA_S8 1
+bitnet_status bitnet_probe_int_rate(int32_t kind, int32_t blocks, int64_t iters, int32_t* out,
+                                    void* stream);
+int64_t bitnet_probe_int_ops(int32_t kind, int32_t blocks, int64_t iters);
+
 /* Human-readable name of a status code (static storage). */
 const char* bitnet_status_string(bitnet_status status);
 

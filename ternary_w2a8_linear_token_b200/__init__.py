@@ -105,6 +105,8 @@ _SIGS = {
                             ctypes.POINTER(bitnet_plan)], ctypes.c_int),
     "bitnet_check_device_errors": ([ctypes.POINTER(_I32)], ctypes.c_int),
     "bitnet_selftest_wait_timeout": ([_I64, _P], ctypes.c_int),
+    "bitnet_probe_int_rate": ([_I32, _I32, _I64, _P, _P], ctypes.c_int),
+    "bitnet_probe_int_ops": ([_I32, _I32, _I64], _I64),
     "bitnet_status_string": ([ctypes.c_int], ctypes.c_char_p),
     "bitnet_version": ([], _I32),
 }

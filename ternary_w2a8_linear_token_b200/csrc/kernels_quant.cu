@@ -213,6 +213,7 @@ __global__ void __launch_bounds__(kLongThreads) quant_long_rows_kernel(
     for (int64_t i = int64_t(blockIdx.x) * kLongThreads + threadIdx.x; i < zero_words;
          i += int64_t(gridDim.x) * kLongThreads)
         zero[i] = make_uint4(0u, 0u, 0u, 0u);
+    if (int64_t(blockIdx.x) * kLongRows >= M) return;  // a CTA added for the clearing only
 
     const uint4* xr = reinterpret_cast<const uint4*>(x + (active ? m : 0) * K);
     uint4 v[kLongPieces];
@@ -269,6 +270,7 @@ __global__ void __launch_bounds__(kLongThreads) quant_long_rows_kernel(
 // integers): CTA b writes the maximum of its grid-stride share to parts[b]. The per-tensor
 // quantiser then reduces the parts; no zeroing or atomics are needed.
 constexpr int kAmaxThreads = 256;
+constexpr int64_t kZeroBytesPerCta = 16 * 1024;  // split-K area cleared per quantiser CTA
 constexpr int kAmaxUnroll = 4;
 
 __global__ void __launch_bounds__(kAmaxThreads) amax_parts_kernel(const uint4* __restrict__ x,
@@ -340,8 +342,14 @@ cudaError_t launch_quant(const uint16_t* x, const int8_t* q_in, int64_t M, int64
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = pdl ? 1 : 0;
+    // Few tokens may come with a large split-K area to clear: add CTAs so that no CTA clears
+    // more than kZeroBytesPerCta (the clearing is a grid-stride loop; the added CTAs quantise
+    // nothing).
+    const int64_t zero_ctas = (zero_bytes + kZeroBytesPerCta - 1) / kZeroBytesPerCta;
+    if (zero_ctas > int64_t(cfg.gridDim.x)) cfg.gridDim.x = static_cast<unsigned>(zero_ctas);
     if (q_in == nullptr && K > int64_t(32) * kRegPieces * 8 && K <= kLongMaxK) {
-        cfg.gridDim = dim3(static_cast<unsigned>((M + kLongRows - 1) / kLongRows));
+        const int64_t rows_ctas = (M + kLongRows - 1) / kLongRows;
+        cfg.gridDim = dim3(static_cast<unsigned>(rows_ctas > zero_ctas ? rows_ctas : zero_ctas));
         cfg.blockDim = dim3(kLongThreads);
         return cudaLaunchKernelEx(&cfg, quant_long_rows_kernel, x, M, K, q, s_x, r_x, permuted,
                                   static_cast<uint4*>(zero), zero_bytes / 16, qsum, amax_parts,

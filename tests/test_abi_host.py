@@ -305,3 +305,16 @@ def test_hand_off_calls_argument_errors(bn):
     assert qa(xm=None) == bn.ERR_NULL and qa(q=None) == bn.ERR_NULL
     assert qa(M=0) == bn.ERR_SHAPE and qa(K=96) == bn.ERR_UNSUPPORTED
     assert qa(xm=F + 2) == bn.ERR_ALIGN and qa(q=F + 8) == bn.ERR_ALIGN
+
+
+def test_probe_calls_argument_errors_and_op_counts(bn):
+    lib, F = bn.lib, FAKE
+    assert lib.bitnet_probe_int_rate(2, 8, 16, F, None) == bn.ERR_UNSUPPORTED
+    assert lib.bitnet_probe_int_rate(0, 0, 16, F, None) == bn.ERR_SHAPE
+    assert lib.bitnet_probe_int_rate(1, 8, 0, F, None) == bn.ERR_SHAPE
+    assert lib.bitnet_probe_int_rate(0, 8, 1 << 25, F, None) == bn.ERR_SHAPE
+    assert lib.bitnet_probe_int_rate(0, 8, 16, None, None) == bn.ERR_NULL
+    # 256 threads x 8 chains x 4 multiply-adds; 8 warps x 4 tiles x 16*8*32 multiply-adds
+    assert lib.bitnet_probe_int_ops(0, 1, 1) == 256 * 8 * 8
+    assert lib.bitnet_probe_int_ops(1, 3, 5) == 8 * 4 * 16 * 8 * 32 * 2 * 3 * 5
+    assert lib.bitnet_probe_int_ops(7, 1, 1) == 0

@@ -203,3 +203,14 @@ def test_decode_chain_of_calls(bn, oracle, path):
         got = bits_from_bf16_tensor(y)
         assert_bf16_within_1ulp(got, ref["y"], oracle, "chain")
         xin = got  # the next call reads exactly what this one wrote
+
+
+def test_int_rate_probes_run_clean(bn):
+    """The arithmetic rate probes behind the bench's int_rates launch, finish and leave the
+    watchdog word clear."""
+    out = torch.empty(16, dtype=torch.int32, device="cuda")
+    for kind in (0, 1):
+        assert bn.lib.bitnet_probe_int_rate(kind, 16, 256, out.data_ptr(),
+                                            torch.cuda.current_stream().cuda_stream) == bn.OK
+    torch.cuda.synchronize()
+    assert bn.bitnet_check_device_errors() == 0

@@ -43,3 +43,4 @@ def test_bounded_wait_expires_and_is_reported(bn, oracle):
     ref = oracle.bitlinear(x, oracle.pack(t), s_w, False, K)
     assert_bf16_within_1ulp(bits_from_bf16_tensor(y), ref["y"], oracle, "after self-test")
     assert bn.bitnet_check_device_errors() == 0
+
