@@ -143,3 +143,32 @@ def stack8b_latent(layer: int, name: str, seed: int = 0):
 
 def stack8b_x(M: int, K: int, seed: int = 0, which: int = 0):
     return normal_x(M, K, rng(seed, 5, 1000 + which, 0, KIND_X))
+
+
+# ---------------------------------------------------------------- device-side draws
+# For workloads too large to draw on the host in a test (billions of values): the same
+# distributions drawn by torch's seeded generator on the device, in row chunks so that no
+# temporary exceeds about a gigabyte. Deterministic for a given (seed, shape, chunk_rows).
+
+def device_normal_bf16(M: int, K: int, seed: int, device, chunk_rows: int = 1 << 17):
+    """x ~ N(0, 1) drawn in fp32 on the device and cast to bf16 there (RNE): (M, K) bf16."""
+    g = torch.Generator(device=device).manual_seed(seed)
+    out = torch.empty((M, K), dtype=torch.bfloat16, device=device)
+    for r0 in range(0, M, chunk_rows):
+        r1 = min(M, r0 + chunk_rows)
+        out[r0:r1] = torch.randn((r1 - r0, K), generator=g, device=device).to(torch.bfloat16)
+    return out
+
+
+def device_ternary_chunks(N: int, K: int, seed: int, device, chunk_rows: int = 1 << 17):
+    """Ternary rows drawn on the device, P(0) = 0.4, P(+1) = P(-1) = 0.3 (as ``ternary``),
+    yielded as (row0, int8 tensor (rows, K)) chunks in row order."""
+    g = torch.Generator(device=device).manual_seed(seed)
+    for r0 in range(0, N, chunk_rows):
+        r1 = min(N, r0 + chunk_rows)
+        r = torch.randint(0, 10, (r1 - r0, K), generator=g, device=device, dtype=torch.int8)
+        t = torch.ones_like(r)
+        t[r >= 7] = -1
+        t[r < 4] = 0
+        del r
+        yield r0, t

@@ -21,6 +21,7 @@ Functions keep the C names:
 from __future__ import annotations
 
 import ctypes
+import functools
 import os
 from typing import Optional, Sequence
 
@@ -219,10 +220,23 @@ def bitnet_quant_act_ex(x: torch.Tensor, act: int = ACT_PER_TOKEN, stream=None):
     return q, s_x
 
 
+@functools.lru_cache(maxsize=4096)
+def _takes_tc_path(M: int, K: int, path: int) -> bool:
+    """Whether a call of this shape runs the tensor-core path (and so needs a workspace): the
+    library's own plan query, which also covers rows too long for the GEMV."""
+    if path == PATH_TC:
+        return True
+    if path != PATH_AUTO:
+        return False
+    pl = bitnet_plan()
+    arr = (_I64 * 1)(64)
+    st = lib.bitnet_linear_plan(M, K, arr, 1, 0, workspace_size(M, K), path, ctypes.byref(pl))
+    return st == OK and pl.kernel == KERNEL_TC
+
+
 def _ws_args(workspace: Optional[torch.Tensor], M: int, K: int, path: int, device):
-    need_tc = path == PATH_TC or (path == PATH_AUTO and M > GEMV_AUTO_M)
     if workspace is None:
-        if not need_tc:
+        if not _takes_tc_path(M, K, path):
             return None, 0, None
         workspace = make_workspace(M, K, device)
     return workspace.data_ptr(), workspace.numel() * workspace.element_size(), workspace

@@ -219,6 +219,11 @@ def test_plan_query_on_the_host(bn):
     assert bn.bitnet_linear_plan(1, 4096, [28672], swiglu=True)["kernel"] == bn.KERNEL_GS
     assert bn.bitnet_linear_plan(1, 14336, [4096])["kernel"] == bn.KERNEL_STREAM  # longer rows
     assert bn.bitnet_linear_plan(3, 2560, [2560])["kernel"] == bn.KERNEL_GEMV
+    # one token past the GEMV's longest row (K = 32768) takes the tensor-core path, so the
+    # binding supplies a workspace for it
+    assert bn.bitnet_linear_plan(1, 32768, [300])["kernel"] == bn.KERNEL_GEMV
+    assert bn.bitnet_linear_plan(1, 32832, [300])["kernel"] == bn.KERNEL_TC
+    assert bn._takes_tc_path(1, 32832, bn.PATH_AUTO) and not bn._takes_tc_path(1, 32768, bn.PATH_AUTO)
     # rows longer than the warp-MMA kernel's largest slice: not available there
     with pytest.raises(bn.BitnetError) as e:
         bn.bitnet_linear_plan(1, 20480, [64], path=bn.PATH_MMA)
