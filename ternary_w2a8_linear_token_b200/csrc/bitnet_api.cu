@@ -135,7 +135,8 @@ bitnet_status plan_batch(const uint16_t* x_bf16, const int8_t* q_in, int64_t M, 
         }
         // One token and a matrix too large for one wave of register-resident rows: the
         // streaming kernel, or for the MLP's gate/up pairs with rows of at most kGsMaxK the
-        // grid-stride kernel (measured faster there on B200, slower on plain projections). The warp-MMA GEMV where it measured faster than the dp4a GEMV on B200 (five to
+        // grid-stride kernel (measured faster there on B200, slower on plain projections).
+        // The warp-MMA GEMV where it measured faster than the dp4a GEMV on B200 (five to
         // eight tokens above kMmaMinBytesFewTokens, reached without a workspace); the dp4a
         // GEMV otherwise.
         const int64_t wbytes = rows * (K / 4);

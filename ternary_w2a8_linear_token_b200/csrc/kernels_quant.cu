@@ -70,7 +70,8 @@ __global__ void __launch_bounds__(kThreads) quant_rows_kernel(const uint16_t* __
                                                               int64_t zero_words,
                                                               int32_t* __restrict__ qsum,
                                                               const uint32_t* __restrict__ amax_parts,
-                                                              int n_parts, const uint16_t* __restrict__ tok_parts) {
+                                                              int n_parts,
+                                                              const uint16_t* __restrict__ tok_parts) {
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const int64_t m = int64_t(blockIdx.x) * kRowsPerCta + warp;
@@ -331,7 +332,7 @@ cudaError_t launch_amax_parts(const uint16_t* x, int64_t M, int64_t K, uint32_t*
 cudaError_t launch_quant(const uint16_t* x, const int8_t* q_in, int64_t M, int64_t K, int8_t* q,
                          float* s_x, float* r_x, int permuted, cudaStream_t stream, bool pdl,
                          void* zero, int64_t zero_bytes, int32_t* qsum,
-                         const uint32_t* amax_parts, int n_parts, const uint16_t* __restrict__ tok_parts) {
+                         const uint32_t* amax_parts, int n_parts, const uint16_t* tok_parts) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>((M + kRowsPerCta - 1) / kRowsPerCta));
     cfg.blockDim = dim3(kThreads);
