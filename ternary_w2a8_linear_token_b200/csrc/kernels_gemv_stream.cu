@@ -198,7 +198,7 @@ __global__ void __launch_bounds__(kStreamThreads, 1)
 
     // Sum over this lane's chunks of one packed row in shared memory: sum_k q * code.
     auto row_dot = [&](const uint8_t* row) -> int32_t {
-        int32_t a0 = 0, a1 = 0;
+        int32_t a0 = 0, a1 = 0, a2 = 0, a3 = 0;  // four independent dp4a chains
 #pragma unroll
         for (int c = 0; c < CPL; ++c) {
             const int chunk = lane + 32 * c;
@@ -210,12 +210,12 @@ __global__ void __launch_bounds__(kStreamThreads, 1)
                     const uint4 qv = QREG ? qreg[QREG ? c : 0][j] : s_q[j * C + chunk];
                     a0 = __dp4a(int(word & 0x03030303u), int(qv.x), a0);
                     a1 = __dp4a(int((word >> 2) & 0x03030303u), int(qv.y), a1);
-                    a0 = __dp4a(int((word >> 4) & 0x03030303u), int(qv.z), a0);
-                    a1 = __dp4a(int((word >> 6) & 0x03030303u), int(qv.w), a1);
+                    a2 = __dp4a(int((word >> 4) & 0x03030303u), int(qv.z), a2);
+                    a3 = __dp4a(int((word >> 6) & 0x03030303u), int(qv.w), a3);
                 }
             }
         }
-        return a0 + a1;
+        return (a0 + a1) + (a2 + a3);
     };
 
     int i = 0;
@@ -242,21 +242,21 @@ __global__ void __launch_bounds__(kStreamThreads, 1)
                 if (p.swiglu) sb[u] = pr.per_row ? pr.s_w[r + kSwigluBlock] : pr.s_w[1];
             }
         }
+        // All of this warp's row sums first, as independent chains (the dp4a chains of one
+        // row alone leave most issue slots idle), then the warp reductions. A unit past the
+        // end of a short last stage reads stale bytes of its slot and is discarded.
+        int32_t part[UPW], part2[UPW];
+#pragma unroll
+        for (int u = 0; u < UPW; ++u) {
+            const int lr = p.swiglu ? 2 * kSwigluBlock * u + cw : kConsumers * u + cw;
+            part[u] = row_dot(base + lr * row_bytes);
+            part2[u] = p.swiglu ? row_dot(base + (lr + kSwigluBlock) * row_bytes) : 0;
+        }
         int32_t tot[UPW], tot2[UPW];
 #pragma unroll
         for (int u = 0; u < UPW; ++u) {
-            tot[u] = tot2[u] = 0;
-            if (!valid[u]) continue;  // warp-uniform
-            if (p.swiglu) {
-                const int lr = 2 * kSwigluBlock * u + cw;
-                tot[u] = __reduce_add_sync(0xFFFFFFFFu, row_dot(base + lr * row_bytes)) - qs_tot;
-                tot2[u] = __reduce_add_sync(0xFFFFFFFFu,
-                                            row_dot(base + (lr + kSwigluBlock) * row_bytes)) -
-                          qs_tot;
-            } else {
-                const int lr = kConsumers * u + cw;
-                tot[u] = __reduce_add_sync(0xFFFFFFFFu, row_dot(base + lr * row_bytes)) - qs_tot;
-            }
+            tot[u] = __reduce_add_sync(0xFFFFFFFFu, part[u]) - qs_tot;
+            tot2[u] = p.swiglu ? __reduce_add_sync(0xFFFFFFFFu, part2[u]) - qs_tot : 0;
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty[slot]);  // this warp is done reading the slot
