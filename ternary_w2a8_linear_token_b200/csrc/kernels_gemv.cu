@@ -325,7 +325,10 @@ cudaError_t launch_one(const GemvParams& p, cudaStream_t stream, bool pdl) {
 // programmatic dependent launch, loads its weights while this one finishes) and take two
 // rows per warp for short rows once the grid would exceed one CTA per SM; more rows per
 // warp lengthen the work left after the wait for the previous grid, which costs more than
-// it saves (measured on B200). Four or eight tokens run one CTA per SM and take as many
+// it saves (measured on B200) — except where two rows per warp would need more than two
+// CTAs per SM: four rows keep such a matrix in one wave (the 2B-4T layer's batched
+// q/k/v/gate/up, 17664 x 2560 at one token: 8.2 -> 6.7 µs per call; 6912 x 2560, which two
+// rows per warp already fit in one wave, 4.1 -> 4.8 µs with four). Four or eight tokens run one CTA per SM and take as many
 // rows per warp as let one wave cover every row: a second wave would repeat each CTA's
 // quantisation of the tokens and its whole dependent chain. Register-resident weights cap
 // the rows per warp.
@@ -335,6 +338,7 @@ cudaError_t launch_cpl(const GemvParams& p, cudaStream_t stream, bool pdl) {
     if (p.swiglu) return launch_one<MT, CPL, 2, true>(p, stream, pdl);  // one pair per warp
     if constexpr (MT <= 2) {
         if constexpr (CPL <= 2) {
+            if (p.total_rows > 4 * slots) return launch_one<MT, CPL, 4>(p, stream, pdl);
             if (p.total_rows > slots) return launch_one<MT, CPL, 2>(p, stream, pdl);
         }
     } else {

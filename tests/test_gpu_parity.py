@@ -127,6 +127,7 @@ I32_CASES = [  # (M, N, K): tile multiples, ragged tails and the minimum K
     (256, 256, 2560), (257, 129, 512), (600, 200, 448),
     (300, 384, 2560), (1000, 640, 2560),  # 128-token tiles past M = 128
     (48, 256, 4160), (20, 200, 1088),  # split-K with 64- and 32-token tiles, K not a stage multiple
+    (1, 10001, 1024), (2, 9600, 2560),  # the GEMV at four rows per warp
 ]
 
 
@@ -179,6 +180,8 @@ LINEAR_CASES = [  # (M, N, K, per_row)
     (129, 131, 640, True), (300, 256, 512, False), (200, 640, 1024, True),
     (40, 300, 4096, True),  # split-K, ragged tokens and rows
     (4, 200, 4096, False), (8, 100, 2048, True),  # GEMV shared memory at exactly 48 KB dynamic
+    # one or two tokens past two CTAs per SM at two rows per warp: four rows per warp
+    (1, 17664, 2560, False), (2, 12000, 4096, True), (1, 9473, 512, True),
 ]
 
 
