@@ -31,11 +31,12 @@ constexpr int kThreads = kWarps * 32;
 
 // MT: token capacity (compile time); p.M <= MT tokens are real, the rest are zero.
 // CPL: 16-byte chunks per lane (K <= CPL * 32 * 64). RW: weight rows per warp.
-// SW: SwiGLU of an interleaved gate/up matrix; each warp takes one output pair, the gate
-// row and the up row of output j (RW = 2), and writes h = SwiGLU(g, u).
+// SW: SwiGLU of an interleaved gate/up matrix; each warp takes RW / 2 output pairs, the gate
+// row and the up row of each output j (rows 2p and 2p + 1 of the warp), and writes
+// h = SwiGLU(g, u).
 template <int MT, int CPL, int RW, bool SW>
 __global__ void __launch_bounds__(kThreads, MT <= 2 ? 2 : 1) gemv_w2a8_kernel(const __grid_constant__ GemvParams p) {
-    static_assert(!SW || RW == 2, "a SwiGLU warp holds one gate row and one up row");
+    static_assert(!SW || RW == 2 || RW == 4, "a SwiGLU warp holds one or two gate/up pairs");
     extern __shared__ uint4 s_q[];  // [MT][4][C] permuted q: word i of group 4c + j
     __shared__ uint32_t s_red[kWarps][MT];  // per-warp amax bits
     __shared__ int32_t s_qsum[kWarps][MT];  // per-warp partial sums of q
@@ -58,8 +59,9 @@ __global__ void __launch_bounds__(kThreads, MT <= 2 ? 2 : 1) gemv_w2a8_kernel(co
         pj[r] = 0;
         if constexpr (SW) {
             // output pair j: gate row 32 (j / 16) + j % 16, up row 16 further
-            const int64_t j = int64_t(blockIdx.x) * kWarps + warp;
-            gr[r] = (j / kSwigluBlock) * (2 * kSwigluBlock) + j % kSwigluBlock + r * kSwigluBlock;
+            const int64_t j = (int64_t(blockIdx.x) * kWarps + warp) * (RW / 2) + r / 2;
+            gr[r] = (j / kSwigluBlock) * (2 * kSwigluBlock) + j % kSwigluBlock +
+                    (r & 1) * kSwigluBlock;
             rvalid[r] = j < p.total_rows;
         } else {
             gr[r] = (int64_t(blockIdx.x) * kWarps + warp) * RW + r;
@@ -79,7 +81,7 @@ __global__ void __launch_bounds__(kThreads, MT <= 2 ? 2 : 1) gemv_w2a8_kernel(co
         sw[r] = 0.0f;
         if (rvalid[r] && p.out_kind != 2)  // per-tensor SwiGLU scales are {s_gate, s_up}
             sw[r] = p.proj[pj[r]].per_row ? p.proj[pj[r]].s_w[nrow[r]]
-                                          : p.proj[pj[r]].s_w[SW ? r : 0];
+                                          : p.proj[pj[r]].s_w[SW ? (r & 1) : 0];
     }
 
     pdl_trigger();
@@ -239,18 +241,26 @@ __global__ void __launch_bounds__(kThreads, MT <= 2 ? 2 : 1) gemv_w2a8_kernel(co
         qs_tot[m] = t;
     }
     if constexpr (SW) {
-        // g and u of this warp's output pair for every token; lane m writes token m's h.
-        const int64_t j = int64_t(blockIdx.x) * kWarps + warp;
+        // g and u of this warp's output pairs for every token; lane pp * MT + m writes
+        // token m's h of pair pp.
 #pragma unroll
-        for (int m = 0; m < MT; ++m) {
-            const int32_t tg = __reduce_add_sync(0xFFFFFFFFu, acc[0][m][0] + acc[0][m][1]);
-            const int32_t tu = __reduce_add_sync(0xFFFFFFFFu, acc[1][m][0] + acc[1][m][1]);
-            if (lane == m && rvalid[0] && m < Mreal) {
-                const float rx = __frcp_rn(s_tok[m]);
-                const float g = __fmul_rn(__int2float_rn(tg - qs_tot[m]), __fmul_rn(sw[0], rx));
-                const float u = __fmul_rn(__int2float_rn(tu - qs_tot[m]), __fmul_rn(sw[1], rx));
-                static_cast<uint16_t*>(p.proj[0].y)[int64_t(m) * p.proj[0].N + j] =
-                    swiglu_bf16_bits(g, u);
+        for (int pp = 0; pp < RW / 2; ++pp) {
+            const int64_t j = (int64_t(blockIdx.x) * kWarps + warp) * (RW / 2) + pp;
+#pragma unroll
+            for (int m = 0; m < MT; ++m) {
+                const int32_t tg =
+                    __reduce_add_sync(0xFFFFFFFFu, acc[2 * pp][m][0] + acc[2 * pp][m][1]);
+                const int32_t tu =
+                    __reduce_add_sync(0xFFFFFFFFu, acc[2 * pp + 1][m][0] + acc[2 * pp + 1][m][1]);
+                if (lane == pp * MT + m && rvalid[2 * pp] && m < Mreal) {
+                    const float rx = __frcp_rn(s_tok[m]);
+                    const float g =
+                        __fmul_rn(__int2float_rn(tg - qs_tot[m]), __fmul_rn(sw[2 * pp], rx));
+                    const float u =
+                        __fmul_rn(__int2float_rn(tu - qs_tot[m]), __fmul_rn(sw[2 * pp + 1], rx));
+                    static_cast<uint16_t*>(p.proj[0].y)[int64_t(m) * p.proj[0].N + j] =
+                        swiglu_bf16_bits(g, u);
+                }
             }
         }
     } else {
@@ -307,7 +317,8 @@ cudaError_t launch_one(const GemvParams& p, cudaStream_t stream, bool pdl) {
                                              static_cast<int>(smem));
         if (e != cudaSuccess) return e;
     }
-    const int64_t rows_per_cta = SW ? int64_t(kWarps) : int64_t(kWarps) * RW;  // SW: pairs
+    // rows of the grid per CTA (SwiGLU: output pairs)
+    const int64_t rows_per_cta = SW ? int64_t(kWarps) * (RW / 2) : int64_t(kWarps) * RW;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>((p.total_rows + rows_per_cta - 1) / rows_per_cta));
     cfg.blockDim = dim3(kThreads);
@@ -335,7 +346,12 @@ cudaError_t launch_one(const GemvParams& p, cudaStream_t stream, bool pdl) {
 template <int MT, int CPL>
 cudaError_t launch_cpl(const GemvParams& p, cudaStream_t stream, bool pdl) {
     const int64_t slots = int64_t(num_sms()) * kWarps;  // warps of one CTA per SM
-    if (p.swiglu) return launch_one<MT, CPL, 2, true>(p, stream, pdl);  // one pair per warp
+    if (p.swiglu) {  // one gate/up pair per warp; two where one would need a second wave
+        if constexpr (MT <= 2 && CPL <= 2) {
+            if (p.total_rows > 2 * slots) return launch_one<MT, CPL, 4, true>(p, stream, pdl);
+        }
+        return launch_one<MT, CPL, 2, true>(p, stream, pdl);
+    }
     if constexpr (MT <= 2) {
         if constexpr (CPL <= 2) {
             if (p.total_rows > 4 * slots) return launch_one<MT, CPL, 4>(p, stream, pdl);

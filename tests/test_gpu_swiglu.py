@@ -80,6 +80,8 @@ SWIGLU_CASES = [
     (3, 48, 2560, True, "gemv"),
     (4, 208, 4096, False, "gemv"),
     (8, 160, 2560, True, "gemv"),
+    (1, 4816, 2560, False, "gemv"),  # two gate/up pairs per warp, ragged last CTA
+    (2, 4816, 1024, True, "gemv"),
     (8, 160, 2560, True, "tc"),
     (16, 144, 512, False, "tc"),
     (37, 208, 2560, True, "tc"),
