@@ -80,8 +80,10 @@ typedef enum {
 typedef enum {
     BITNET_PATH_AUTO = 0, /* GEMV for M <= BITNET_GEMV_AUTO_M; for M up to                */
                           /* BITNET_GEMV_MAX_M the tensor-core GEMM when the workspace    */
-                          /* holds it, else the GEMV; tensor-core GEMM above. Among the   */
-                          /* GEMVs, the kernel measured fastest for the size.             */
+                          /* holds it, else the GEMV; tensor-core GEMM above, and for     */
+                          /* rows longer than the GEMV takes (K > 32768 at one token,     */
+                          /* bitnet_linear_plan tells). Among the GEMVs, the kernel       */
+                          /* measured fastest for the size.                               */
     BITNET_PATH_GEMV = 1, /* force the dp4a GEMV with fused activation quantisation (the  */
                           /* streaming variant at one token from 12 MiB of weights)       */
     BITNET_PATH_TC = 2,   /* force the tcgen05 GEMM (needs the workspace)                 */
