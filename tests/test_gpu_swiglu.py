@@ -82,6 +82,7 @@ SWIGLU_CASES = [
     (8, 160, 2560, True, "gemv"),
     (1, 4816, 2560, False, "gemv"),  # two gate/up pairs per warp, ragged last CTA
     (2, 4816, 1024, True, "gemv"),
+    (1, 1024, 6912, True, "gemv"),  # four chunks per lane
     (8, 160, 2560, True, "tc"),
     (16, 144, 512, False, "tc"),
     (37, 208, 2560, True, "tc"),
@@ -195,4 +196,22 @@ def test_swiglu_one_token_grid_stride_per_tensor(bn, oracle):
     ref = oracle.swiglu_gate_up(x, pg, sg, pu, su, False, K)
     assert_swiglu_within_bound(bits_from_bf16_tensor(h), ref, oracle, where="grid-stride SwiGLU")
     h_tc = bn.bitnet_linear_swiglu(xd, packed_gu, s_gu, False, path=bn.PATH_TC)
+    assert torch.equal(h.view(torch.int16), h_tc.view(torch.int16))
+
+
+@pytest.mark.parametrize("per_row", [False, True])
+def test_swiglu_one_token_streaming_long_rows(bn, oracle, per_row):
+    """One token, rows longer than the grid-stride kernel takes (K = 8192) and 13.1 MB of
+    interleaved gate/up weights: the streaming GEMV's SwiGLU pairing. Within the bound, and
+    bit-equal to the tensor-core path (same arithmetic)."""
+    I, K = 3200, 8192
+    assert bn.bitnet_linear_plan(1, K, [2 * I], swiglu=True)["kernel"] == bn.KERNEL_STREAM
+    x, tg, tu, sg, su = _mlp(1, I, K, per_row, seed=3)
+    pg, pu, packed_gu, s_gu = _device_weights(bn, oracle, tg, tu, sg, su, per_row)
+    xd = bf16_tensor_from_bits(x)
+    h = bn.bitnet_linear_swiglu(xd, packed_gu, s_gu, per_row)
+    torch.cuda.synchronize()
+    ref = oracle.swiglu_gate_up(x, pg, sg, pu, su, per_row, K)
+    assert_swiglu_within_bound(bits_from_bf16_tensor(h), ref, oracle, where="streaming SwiGLU")
+    h_tc = bn.bitnet_linear_swiglu(xd, packed_gu, s_gu, per_row, path=bn.PATH_TC)
     assert torch.equal(h.view(torch.int16), h_tc.view(torch.int16))
