@@ -72,3 +72,26 @@ __device__ __forceinline__ uint2 permute_group_half(uint2 nat, int h) {
 }
 
 }  // namespace bitnet
+
+// Sum over one packed weight word (16 codes c = t + 1) times the token's permuted q (one
+// uint4, word i against the codes at bits 2i..2i+1 of every byte). The codes are masked in
+// place instead of shifted down: byte values c * 4^i with c in {0, 1, 2}, unsigned, against
+// signed q, so acc.{x, y, z, w} collect 4^i * sum c q for i = 0 .. 3 with one AND and one dp4a
+// per four weights; code_dot_total divides the factors back out, exactly (each sum is a
+// multiple of its 4^i; |64 sum c q| stays far inside int32 for a lane's share of a row).
+__device__ __forceinline__ int dp4a_u8s8(uint32_t a, uint32_t b, int c) {
+    int d;
+    asm("dp4a.u32.s32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+    return d;
+}
+
+__device__ __forceinline__ void code_dot_acc(uint32_t word, const uint4 q, int4& acc) {
+    acc.x = dp4a_u8s8(word & 0x03030303u, q.x, acc.x);
+    acc.y = dp4a_u8s8(word & 0x0C0C0C0Cu, q.y, acc.y);
+    acc.z = dp4a_u8s8(word & 0x30303030u, q.z, acc.z);
+    acc.w = dp4a_u8s8(word & 0xC0C0C0C0u, q.w, acc.w);
+}
+
+__device__ __forceinline__ int code_dot_total(const int4 acc) {
+    return (acc.x + (acc.y >> 2)) + ((acc.z >> 4) + (acc.w >> 6));
+}

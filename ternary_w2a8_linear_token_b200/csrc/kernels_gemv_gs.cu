@@ -60,14 +60,6 @@ __device__ __forceinline__ void decode_b3_chunk(const uint4 v, uint32_t (&w)[5])
     }
 }
 
-// sum over the 16 weights of one 2-bit-format word of code * q (q permuted, one uint4).
-__device__ __forceinline__ int word_dot(uint32_t word, const uint4 q, int acc) {
-    acc = __dp4a(int(word & 0x03030303u), int(q.x), acc);
-    acc = __dp4a(int((word >> 2) & 0x03030303u), int(q.y), acc);
-    acc = __dp4a(int((word >> 4) & 0x03030303u), int(q.z), acc);
-    return __dp4a(int((word >> 6) & 0x03030303u), int(q.w), acc);
-}
-
 // One row of a pair in flight: this lane's chunks and, for lane 0, the row's scale.
 template <int CPL>
 struct RowBuf {
@@ -175,7 +167,7 @@ __global__ void __launch_bounds__(kGsThreads, 1) gemv_gs_kernel(const __grid_con
     const float rx = __frcp_rn(s);
 
     auto row_dot = [&](const RowBuf<CPL>& buf) -> int {
-        int a0 = 0, a1 = 0;
+        int4 a0 = make_int4(0, 0, 0, 0), a1 = make_int4(0, 0, 0, 0);
 #pragma unroll
         for (int i = 0; i < CPL; ++i) {
             const int c = lane + 32 * i;
@@ -193,15 +185,12 @@ __global__ void __launch_bounds__(kGsThreads, 1) gemv_gs_kernel(const __grid_con
                 for (int d = 0; d < G; ++d) {
                     if (!B3 || G * c + d < groups) {  // base-3 padding groups carry no q
                         const uint4 q = s_q[d * C + c];
-                        if (d & 1)
-                            a1 = word_dot(wd[d], q, a1);
-                        else
-                            a0 = word_dot(wd[d], q, a0);
+                        code_dot_acc(wd[d], q, (d & 1) ? a1 : a0);
                     }
                 }
             }
         }
-        return a0 + a1;
+        return code_dot_total(a0) + code_dot_total(a1);
     };
     auto store_row = [&](int64_t r, int32_t acc, float sw) {
         int pj = 0;

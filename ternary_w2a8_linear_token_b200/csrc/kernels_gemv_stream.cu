@@ -13,9 +13,11 @@
 //  - one CTA per SM, persistent over stages s = blockIdx.x, blockIdx.x + gridDim.x, ...;
 //    a stage is 16 * UPW consecutive rows of one projection (16 * UPW output pairs, 32 * UPW
 //    interleaved rows, for SwiGLU), one contiguous span of the (N, K/4) packed matrix, and
-//    each consumer warp takes UPW of its units: at one token the kernel is bound by issue
-//    slots (11 instructions per 16 weights), so the per-stage bookkeeping is spread over
-//    several rows;
+//    each consumer warp takes UPW of its units: at one token the consumers' instruction
+//    stream bounds the kernel (8 instructions per 16 weights: the codes are masked in place,
+//    see code_dot_acc, and issued at about one instruction every other cycle per scheduler),
+//    so the per-stage bookkeeping is spread over several rows, which are summed as
+//    independent chains;
 //  - full/empty mbarriers per ring slot, every wait bounded (the library's watchdog);
 //  - the consumers quantise x once per CTA into shared memory in the permuted in-group
 //    order (see kernels_quant.cu) and keep their lanes' share of q in registers (K <= 4096)
@@ -198,7 +200,7 @@ __global__ void __launch_bounds__(kStreamThreads, 1)
 
     // Sum over this lane's chunks of one packed row in shared memory: sum_k q * code.
     auto row_dot = [&](const uint8_t* row) -> int32_t {
-        int32_t a0 = 0, a1 = 0, a2 = 0, a3 = 0;  // four independent dp4a chains
+        int4 acc = make_int4(0, 0, 0, 0);  // four independent dp4a chains
 #pragma unroll
         for (int c = 0; c < CPL; ++c) {
             const int chunk = lane + 32 * c;
@@ -208,14 +210,11 @@ __global__ void __launch_bounds__(kStreamThreads, 1)
                 for (int j = 0; j < 4; ++j) {
                     const uint32_t word = j == 0 ? wv.x : j == 1 ? wv.y : j == 2 ? wv.z : wv.w;
                     const uint4 qv = QREG ? qreg[QREG ? c : 0][j] : s_q[j * C + chunk];
-                    a0 = __dp4a(int(word & 0x03030303u), int(qv.x), a0);
-                    a1 = __dp4a(int((word >> 2) & 0x03030303u), int(qv.y), a1);
-                    a2 = __dp4a(int((word >> 4) & 0x03030303u), int(qv.z), a2);
-                    a3 = __dp4a(int((word >> 6) & 0x03030303u), int(qv.w), a3);
+                    code_dot_acc(word, qv, acc);
                 }
             }
         }
-        return (a0 + a1) + (a2 + a3);
+        return code_dot_total(acc);
     };
 
     int i = 0;
