@@ -195,41 +195,53 @@ __global__ void __launch_bounds__(kThreads, MT <= 2 ? 2 : 1) gemv_w2a8_kernel(co
 
     // ---- 3. dp4a over the register-resident chunks: sum_k q * code, two independent
     //         accumulator chains per output
-    int32_t acc[RW][MT][2];
+    // One token: the codes are masked in place (code_dot_acc, one AND per four weights and
+    // four accumulators); more tokens share one shifted unpack of each word instead (and
+    // would need more registers for the accumulators than two CTAs per SM leave).
+    constexpr bool kMasked = MT == 1;
+    int4 acc[RW][MT];
 #pragma unroll
     for (int r = 0; r < RW; ++r)
 #pragma unroll
-        for (int m = 0; m < MT; ++m) acc[r][m][0] = acc[r][m][1] = 0;
+        for (int m = 0; m < MT; ++m) acc[r][m] = make_int4(0, 0, 0, 0);
 #pragma unroll
     for (int c = 0; c < CPL; ++c) {
         const int chunk = lane + 32 * c;
         if (chunk < C) {
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
+                uint32_t word[RW];
                 int e[RW][4];
 #pragma unroll
                 for (int r = 0; r < RW; ++r) {
-                    const uint32_t word = j == 0 ? w[r][c].x : j == 1 ? w[r][c].y
-                                        : j == 2 ? w[r][c].z : w[r][c].w;
-                    e[r][0] = int(word & 0x03030303u);
-                    e[r][1] = int((word >> 2) & 0x03030303u);
-                    e[r][2] = int((word >> 4) & 0x03030303u);
-                    e[r][3] = int((word >> 6) & 0x03030303u);
+                    word[r] = j == 0 ? w[r][c].x : j == 1 ? w[r][c].y
+                            : j == 2 ? w[r][c].z : w[r][c].w;
+                    if constexpr (!kMasked) {
+                        e[r][0] = int(word[r] & 0x03030303u);
+                        e[r][1] = int((word[r] >> 2) & 0x03030303u);
+                        e[r][2] = int((word[r] >> 4) & 0x03030303u);
+                        e[r][3] = int((word[r] >> 6) & 0x03030303u);
+                    }
                 }
 #pragma unroll
                 for (int m = 0; m < MT; ++m) {
                     const uint4 qv = s_q[(m * 4 + j) * C + chunk];
 #pragma unroll
                     for (int r = 0; r < RW; ++r) {
-                        acc[r][m][0] = __dp4a(e[r][0], int(qv.x), acc[r][m][0]);
-                        acc[r][m][1] = __dp4a(e[r][1], int(qv.y), acc[r][m][1]);
-                        acc[r][m][0] = __dp4a(e[r][2], int(qv.z), acc[r][m][0]);
-                        acc[r][m][1] = __dp4a(e[r][3], int(qv.w), acc[r][m][1]);
+                        if constexpr (kMasked) {
+                            code_dot_acc(word[r], qv, acc[r][m]);
+                        } else {
+                            acc[r][m].x = __dp4a(e[r][0], int(qv.x), acc[r][m].x);
+                            acc[r][m].y = __dp4a(e[r][1], int(qv.y), acc[r][m].y);
+                            acc[r][m].x = __dp4a(e[r][2], int(qv.z), acc[r][m].x);
+                            acc[r][m].y = __dp4a(e[r][3], int(qv.w), acc[r][m].y);
+                        }
                     }
                 }
             }
         }
     }
+    auto dot_total = [](const int4 a) { return kMasked ? code_dot_total(a) : a.x + a.y; };
 
     // ---- 4. reduce across the warp, remove the code offset (sum q), dequantise, write
     int32_t qs_tot[MT];
@@ -249,9 +261,9 @@ __global__ void __launch_bounds__(kThreads, MT <= 2 ? 2 : 1) gemv_w2a8_kernel(co
 #pragma unroll
             for (int m = 0; m < MT; ++m) {
                 const int32_t tg =
-                    __reduce_add_sync(0xFFFFFFFFu, acc[2 * pp][m][0] + acc[2 * pp][m][1]);
+                    __reduce_add_sync(0xFFFFFFFFu, dot_total(acc[2 * pp][m]));
                 const int32_t tu =
-                    __reduce_add_sync(0xFFFFFFFFu, acc[2 * pp + 1][m][0] + acc[2 * pp + 1][m][1]);
+                    __reduce_add_sync(0xFFFFFFFFu, dot_total(acc[2 * pp + 1][m]));
                 if (lane == pp * MT + m && rvalid[2 * pp] && m < Mreal) {
                     const float rx = __frcp_rn(s_tok[m]);
                     const float g =
@@ -268,7 +280,7 @@ __global__ void __launch_bounds__(kThreads, MT <= 2 ? 2 : 1) gemv_w2a8_kernel(co
         for (int r = 0; r < RW; ++r) {
 #pragma unroll
             for (int m = 0; m < MT; ++m) {
-                const int32_t total = __reduce_add_sync(0xFFFFFFFFu, acc[r][m][0] + acc[r][m][1]);
+                const int32_t total = __reduce_add_sync(0xFFFFFFFFu, dot_total(acc[r][m]));
                 if (lane == r * MT + m && rvalid[r] && m < Mreal) {
                     const GemvProj& pr = p.proj[pj[r]];
                     const int32_t v = total - qs_tot[m];
