@@ -46,8 +46,8 @@ INT8_PER_BF16 = 2.0
 
 # DRAM bytes per decode-sweep GEMV launch, read + write, from one ncu capture of the four
 # shapes with the current kernel (2560 x 2560, 640 x 2560, 6912 x 2560, 2560 x 6912 at M = 1:
-# 1662464, 430592, 4447488, 4454912 bytes), averaged.
-GEMV_DECODE_TRAFFIC_BYTES = 2748864
+# 1659648, 430592, 4455424, 4454912 bytes), averaged.
+GEMV_DECODE_TRAFFIC_BYTES = 2750144
 # DRAM bytes per prefill GEMM launch (tc_gemm_kernel, M = 2048), read + write, from one ncu
 # capture of the four shapes (6979328, 5748736, 9764352, 18681344 bytes), averaged. The bf16
 # outputs stay in L2 while the kernel runs (written back after it ends), so this is below the

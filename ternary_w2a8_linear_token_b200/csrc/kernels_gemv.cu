@@ -346,7 +346,10 @@ cudaError_t launch_one(const GemvParams& p, cudaStream_t stream, bool pdl) {
 
 // Rows per warp. One or two tokens run two CTAs per SM (so the next grid, started early by
 // programmatic dependent launch, loads its weights while this one finishes) and take two
-// rows per warp for short rows once the grid would exceed one CTA per SM; more rows per
+// rows per warp once the grid would exceed two CTAs per SM, or one CTA per SM for rows of at
+// least 1 KB (measured on B200 at one token: 2560 x 2560 runs faster with one row per warp
+// on 160 CTAs, 3.08 -> 3.02 µs per call and the decode sweep 3.36 -> 3.22, 4096 x 4096
+// slower, 3.38 -> 3.58); more rows per
 // warp lengthen the work left after the wait for the previous grid, which costs more than
 // it saves (measured on B200) — except where two rows per warp would need more than two
 // CTAs per SM: four rows keep such a matrix in one wave (the 2B-4T layer's batched
@@ -367,7 +370,8 @@ cudaError_t launch_cpl(const GemvParams& p, cudaStream_t stream, bool pdl) {
     if constexpr (MT <= 2) {
         if constexpr (CPL <= 2) {
             if (p.total_rows > 4 * slots) return launch_one<MT, CPL, 4>(p, stream, pdl);
-            if (p.total_rows > slots) return launch_one<MT, CPL, 2>(p, stream, pdl);
+            if (p.total_rows > 2 * slots || (p.total_rows > slots && p.K >= 4096))
+                return launch_one<MT, CPL, 2>(p, stream, pdl);
         }
     } else {
         const int64_t need = (p.total_rows + slots - 1) / slots;
