@@ -397,10 +397,10 @@ bitnet_status bitnet_dequant(const int32_t* acc, int64_t M, int64_t N, const flo
 #define BITNET_KERNEL_GS 5     /* one-token grid-stride GEMV for large matrices               */
 typedef struct {
     int32_t kernel;        /* BITNET_KERNEL_*                                               */
-    int32_t grid;          /* CTAs of the main kernel (0 for BITNET_KERNEL_GEMV)            */
+    int32_t grid;          /* CTAs of the main kernel                                       */
     int32_t tile_tokens;   /* tensor-core path: tokens per tile (16 .. 192), else 0         */
     int32_t splits;        /* tensor-core path: K splits per tile (1 = none), else 0        */
-    int32_t tile_rows;     /* warp-MMA GEMV: weight rows per CTA, else 0                     */
+    int32_t tile_rows;     /* GEMV and warp-MMA GEMV: weight rows per CTA, else 0            */
     int32_t reserved[3];
 } bitnet_plan;
 bitnet_status bitnet_linear_plan(int64_t M, int64_t K, const int64_t* Ns, int32_t nproj,

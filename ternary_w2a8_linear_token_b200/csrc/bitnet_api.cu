@@ -757,10 +757,16 @@ bitnet_status bitnet_linear_plan(int64_t M, int64_t K, const int64_t* Ns, int32_
     if (st != BITNET_OK) return st;
     std::memset(plan, 0, sizeof(*plan));
     plan->kernel = pl.kernel;
-    plan->grid = pl.kernel == BITNET_KERNEL_GEMV ? 0 : pl.grid;
+    plan->grid = pl.grid;
     plan->tile_tokens = pl.kernel == BITNET_KERNEL_TC ? pl.bn : 0;
     plan->splits = pl.kernel == BITNET_KERNEL_TC ? pl.splits : 0;
     plan->tile_rows = pl.kernel == BITNET_KERNEL_MMA_GEMV ? 16 * pl.rt : 0;
+    if (pl.kernel == BITNET_KERNEL_GEMV) {  // 16 warps of rw rows (SwiGLU: rw / 2 pairs) each
+        const int rw = gemv_rows_per_warp(pl.gp, tc_num_sms());
+        const int64_t units = swiglu ? 16 * (rw / 2) : 16 * rw;
+        plan->tile_rows = 16 * rw;
+        plan->grid = static_cast<int32_t>((pl.gp.total_rows + units - 1) / units);
+    }
     return BITNET_OK;
 }
 

@@ -71,6 +71,9 @@ struct GemvParams {
 
 cudaError_t launch_gemv(const GemvParams& p, cudaStream_t stream, bool pdl);
 bool gemv_supported(int64_t M, int64_t K);
+// Rows per warp the dp4a GEMV takes for this call on a GPU of `sms` SMs (SwiGLU: 2 per
+// gate/up pair): the launch's choice, also reported by the plan query.
+int gemv_rows_per_warp(const GemvParams& p, int sms);
 // The kernel-path choice of bitnet_linear / bitnet_linear_batch: true when a call with this
 // token count, width, path and workspace runs the GEMV (which uses no workspace).
 bool use_gemv(int64_t M, int64_t K, bitnet_path path, const void* ws, size_t ws_bytes);

@@ -344,42 +344,26 @@ cudaError_t launch_one(const GemvParams& p, cudaStream_t stream, bool pdl) {
     return cudaLaunchKernelEx(&cfg, kern, q);
 }
 
-// Rows per warp. One or two tokens run two CTAs per SM (so the next grid, started early by
-// programmatic dependent launch, loads its weights while this one finishes) and take two
-// rows per warp once the grid would exceed two CTAs per SM, or one CTA per SM for rows of at
-// least 1 KB (measured on B200 at one token: 2560 x 2560 runs faster with one row per warp
-// on 160 CTAs, 3.08 -> 3.02 µs per call and the decode sweep 3.36 -> 3.22, 4096 x 4096
-// slower, 3.38 -> 3.58); more rows per
-// warp lengthen the work left after the wait for the previous grid, which costs more than
-// it saves (measured on B200) — except where two rows per warp would need more than two
-// CTAs per SM: four rows keep such a matrix in one wave (the 2B-4T layer's batched
-// q/k/v/gate/up, 17664 x 2560 at one token: 8.2 -> 6.7 µs per call; 6912 x 2560, which two
-// rows per warp already fit in one wave, 4.1 -> 4.8 µs with four). Four or eight tokens run one CTA per SM and take as many
-// rows per warp as let one wave cover every row: a second wave would repeat each CTA's
-// quantisation of the tokens and its whole dependent chain. Register-resident weights cap
-// the rows per warp.
 template <int MT, int CPL>
 cudaError_t launch_cpl(const GemvParams& p, cudaStream_t stream, bool pdl) {
-    const int64_t slots = int64_t(num_sms()) * kWarps;  // warps of one CTA per SM
-    if (p.swiglu) {  // one gate/up pair per warp; two where one would need a second wave
+    const int rw = gemv_rows_per_warp(p, num_sms());
+    if (p.swiglu) {
         if constexpr (MT <= 2 && CPL <= 2) {
-            if (p.total_rows > 2 * slots) return launch_one<MT, CPL, 4, true>(p, stream, pdl);
+            if (rw == 4) return launch_one<MT, CPL, 4, true>(p, stream, pdl);
         }
         return launch_one<MT, CPL, 2, true>(p, stream, pdl);
     }
     if constexpr (MT <= 2) {
         if constexpr (CPL <= 2) {
-            if (p.total_rows > 4 * slots) return launch_one<MT, CPL, 4>(p, stream, pdl);
-            if (p.total_rows > 2 * slots || (p.total_rows > slots && p.K >= 4096))
-                return launch_one<MT, CPL, 2>(p, stream, pdl);
+            if (rw == 4) return launch_one<MT, CPL, 4>(p, stream, pdl);
+            if (rw == 2) return launch_one<MT, CPL, 2>(p, stream, pdl);
         }
     } else {
-        const int64_t need = (p.total_rows + slots - 1) / slots;
         if constexpr (CPL <= 2 && MT <= 4) {
-            if (need >= 3) return launch_one<MT, CPL, 3>(p, stream, pdl);
+            if (rw == 3) return launch_one<MT, CPL, 3>(p, stream, pdl);
         }
         if constexpr (CPL <= 2 || (MT <= 4 && CPL <= 4)) {
-            if (need >= 2) return launch_one<MT, CPL, 2>(p, stream, pdl);
+            if (rw == 2) return launch_one<MT, CPL, 2>(p, stream, pdl);
         }
     }
     return launch_one<MT, CPL, 1>(p, stream, pdl);
@@ -397,6 +381,41 @@ cudaError_t launch_mt(const GemvParams& p, cudaStream_t stream, bool pdl) {
 }
 
 }  // namespace
+
+// Rows per warp of the dp4a GEMV (SwiGLU: 2 per gate/up pair). One or two tokens run two CTAs
+// per SM (so the next grid, started early by programmatic dependent launch, loads its weights
+// while this one finishes) and take two rows per warp once the grid would exceed two CTAs per
+// SM, or one CTA per SM for rows of at least 1 KB (measured on B200 at one token: 2560 x 2560
+// runs faster with one row per warp on 160 CTAs, 3.08 -> 3.02 µs per call and the decode sweep
+// 3.36 -> 3.22; 4096 x 4096 slower, 3.38 -> 3.58). More rows per warp lengthen the work left
+// after the wait for the previous grid, which costs more than it saves (measured on B200),
+// except where two rows per warp would need more than two CTAs per SM: four rows keep such a
+// matrix in one wave (the 2B-4T layer's batched q/k/v/gate/up, 17664 x 2560 at one token:
+// 8.2 -> 6.7 µs per call; 6912 x 2560, which two rows per warp already fit in one wave,
+// 4.1 -> 4.8 µs with four); the SwiGLU variant likewise takes two pairs per warp once one pair
+// would need more than two CTAs per SM. Four or eight tokens run one CTA per SM and take as
+// many rows per warp (up to 3) as let one wave cover every row: a second wave would repeat
+// each CTA's quantisation of the tokens and its whole dependent chain. Register-resident
+// weights cap the rows per warp (the chunk counts below).
+int gemv_rows_per_warp(const GemvParams& p, int sms) {
+    const int64_t C = p.K >> 6;
+    const int64_t c32 = (C + 31) / 32;  // chunks per lane, rounded up as the kernels are
+    const int cpl = c32 <= 1 ? 1 : c32 <= 2 ? 2 : c32 <= 4 ? 4 : c32 <= 8 ? 8 : 16;
+    const int mt = p.M <= 1 ? 1 : p.M <= 2 ? 2 : p.M <= 4 ? 4 : 8;
+    const int64_t slots = int64_t(sms) * kWarps;  // warps of one CTA per SM
+    if (p.swiglu) return (mt <= 2 && cpl <= 2 && p.total_rows > 2 * slots) ? 4 : 2;
+    if (mt <= 2) {
+        if (cpl <= 2) {
+            if (p.total_rows > 4 * slots) return 4;
+            if (p.total_rows > 2 * slots || (p.total_rows > slots && p.K >= 4096)) return 2;
+        }
+        return 1;
+    }
+    const int64_t need = (p.total_rows + slots - 1) / slots;
+    if (cpl <= 2 && mt <= 4 && need >= 3) return 3;
+    if ((cpl <= 2 || (mt <= 4 && cpl <= 4)) && need >= 2) return 2;
+    return 1;
+}
 
 bool gemv_supported(int64_t M, int64_t K) {
     const int64_t mt = M <= 1 ? 1 : M <= 2 ? 2 : M <= 4 ? 4 : 8;

@@ -224,6 +224,22 @@ def test_plan_query_on_the_host(bn):
     assert bn.bitnet_linear_plan(1, 32768, [300])["kernel"] == bn.KERNEL_GEMV
     assert bn.bitnet_linear_plan(1, 32832, [300])["kernel"] == bn.KERNEL_TC
     assert bn._takes_tc_path(1, 32832, bn.PATH_AUTO) and not bn._takes_tc_path(1, 32768, bn.PATH_AUTO)
+    # one-token GEMV rows per warp (tile_rows = 16 warps x rows), as the kernels were timed:
+    # one row for 640-byte rows up to two CTAs per SM, two for 1 KB rows past one CTA per SM,
+    # four past two CTAs per SM at two; SwiGLU: two gate/up pairs per warp past two CTAs per SM
+    def rows(M, K, Ns, swiglu=False):
+        pl = bn.bitnet_linear_plan(M, K, Ns, swiglu=swiglu)
+        assert pl["kernel"] == bn.KERNEL_GEMV
+        return pl["tile_rows"], pl["grid"]
+    assert rows(1, 2560, [2560]) == (16, 160)
+    assert rows(1, 2560, [640]) == (16, 40)
+    assert rows(1, 4096, [4096]) == (32, 128)
+    assert rows(1, 2560, [6912]) == (32, 216)
+    assert rows(1, 6912, [2560]) == (16, 160)
+    assert rows(1, 2560, [17664]) == (64, 276)
+    assert rows(1, 2560, [13824], swiglu=True) == (64, 216)
+    assert rows(1, 4096, [2048], swiglu=True) == (32, 64)
+    assert rows(4, 2560, [2560]) == (32, 80)
     # rows longer than the warp-MMA kernel's largest slice: not available there
     with pytest.raises(bn.BitnetError) as e:
         bn.bitnet_linear_plan(1, 20480, [64], path=bn.PATH_MMA)
