@@ -193,8 +193,8 @@ __global__ void __launch_bounds__(kThreads, MT <= 2 ? 2 : 1) gemv_w2a8_kernel(co
     }
     __syncthreads();
 
-    // ---- 3. dp4a over the register-resident chunks: sum_k q * code, two independent
-    //         accumulator chains per output
+    // ---- 3. dp4a over the register-resident chunks: sum_k q * code, independent
+    //         accumulator chains per output (four at one token, two otherwise)
     // One token: the codes are masked in place (code_dot_acc, one AND per four weights and
     // four accumulators); more tokens share one shifted unpack of each word instead (and
     // would need more registers for the accumulators than two CTAs per SM leave).
