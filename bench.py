@@ -472,7 +472,7 @@ def measure_int8_peak(torch, dev, seconds: float = 1.5):
     try:
         for _ in range(3):
             torch._int_mm(a, b)
-    except RuntimeError as e:  # no int8 GEMM in this build
+    except RuntimeError as e:  # torch without an int8 GEMM
         return {"error": repr(e)[:200]}
     torch.cuda.synchronize()
     best = float("inf")
