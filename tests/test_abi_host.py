@@ -339,3 +339,21 @@ def test_probe_calls_argument_errors_and_op_counts(bn):
     assert lib.bitnet_probe_int_ops(0, 1, 1) == 256 * 8 * 8
     assert lib.bitnet_probe_int_ops(1, 3, 5) == 8 * 4 * 16 * 8 * 32 * 2 * 3 * 5
     assert lib.bitnet_probe_int_ops(7, 1, 1) == 0
+
+
+def test_binding_signatures_match_the_header(bn):
+    """Every call the header declares has a ctypes signature in the binding with the same
+    number of parameters and a matching return type (int status, int64, size_t or string)."""
+    src = re.sub(r"/\*.*?\*/", "", open(HEADER, encoding="utf-8").read(), flags=re.S)
+    decls = re.findall(r"\b(bitnet_status|int64_t|size_t|int32_t|const char\s*\*)\s+"
+                       r"(bitnet_[a-z0-9_]+)\s*\(([^;]*?)\)\s*;", src, flags=re.S)
+    assert len(decls) == len(declared_functions())
+    ret_types = {"bitnet_status": ctypes.c_int, "int64_t": ctypes.c_int64,
+                 "size_t": ctypes.c_size_t, "int32_t": ctypes.c_int32}
+    for ret, name, args in decls:
+        a = args.strip()
+        n = 0 if a in ("", "void") else len([x for x in a.split(",") if x.strip()])
+        argtypes, restype = bn._SIGS[name]
+        assert len(argtypes) == n, name
+        want = ctypes.c_char_p if ret.startswith("const char") else ret_types[ret]
+        assert restype is want, name
